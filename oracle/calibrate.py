@@ -1,0 +1,125 @@
+"""WUSH / WUS / Hadamard / identity block transforms from second moments (oracle).
+
+Cites:
+  * WUSH news article, paragraph 3: WUSH is built from the Cholesky factor of the
+    weights (W), the SVD components (U, S) and a Hadamard matrix (H), from the
+    second-order statistics of weights and activations; it is non-orthogonal and
+    block-diagonal.
+  * WUSH news article, paragraph 6 (deployment workflow): collect the second
+    moments of weights and activations from calibration data, compute the
+    transforms (Cholesky and SVD, in parallel over blocks), apply the transform
+    to the input activations at inference.
+  * WUSH news article, paragraph 5: WUS (no Hadamard component) is evaluated
+    beside WUSH on NVFP4.
+  * AI Radio episode, "The gist": a Hadamard backbone combined with a
+    data-dependent second-moment component, non-orthogonal.
+  * AI Radio episode, "Problem Setup and Goal": T_W and T_X are chosen so that
+    q(T_W W)^T q(T_X X) approximates W^T X.
+
+Reading (the pages print no formula). Per d_in block j of width b:
+    Sigma_X = X_j X_j^T / n_calib,   Sigma_W = W_j W_j^T / d_out     (b x b)
+    W' = lower Cholesky factor of Sigma_W
+    W'^T Sigma_X W' = U diag(lambda) U^T,  S = diag(sqrt(lambda))
+        (this is the SVD of W'^T X_j / sqrt(n) without forming it)
+    T_X = Hn S^(-1/2) U^T W'^T,     T_W = T_X^(-T) = Hn S^(1/2) U^T W'^(-1)
+with Hn = H_b / sqrt(b).  WUS drops Hn; "hadamard" is T_X = T_W = Hn; "identity"
+is I.  The factors are listed in the order in which they act on x (W, U, S, H),
+T_W^T T_X = I so the product is lossless before rounding, and the transformed
+moments balance: T_X Sigma_X T_X^T = T_W Sigma_W T_W^T = Hn S Hn^T.
+
+Conventions the pages leave open: eigenvalues in descending order; each column
+of U is negated if needed so that its largest-magnitude entry is positive (ties
+to the lowest index); eigenvalues are floored at 1e-12 * max(lambda); a failed
+Cholesky is retried once on Sigma_W + 1e-8 * mean(diag(Sigma_W)) I.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from .transforms import normalized_hadamard
+
+KINDS = ("identity", "hadamard", "wus", "wush")
+
+
+class NotPositiveDefinite(ValueError):
+    pass
+
+
+def block_moments(x_rows: np.ndarray, b: int) -> np.ndarray:
+    """Per-block second moments (1/rows) sum_r x_j x_j^T, as [d_in/b, b, b] fp64.
+
+    x_rows: [rows, d_in] -- calibration tokens of X, or the d_out rows of W^T.
+    """
+    x = np.asarray(x_rows, dtype=np.float64)
+    rows, d_in = x.shape
+    xb = x.reshape(rows, d_in // b, b)
+    return np.einsum("rjk,rjl->jkl", xb, xb) / rows
+
+
+def _cholesky(sigma_w: np.ndarray) -> np.ndarray:
+    try:
+        return np.linalg.cholesky(sigma_w)
+    except np.linalg.LinAlgError:
+        jitter = 1e-8 * np.mean(np.diag(sigma_w))
+        try:
+            return np.linalg.cholesky(sigma_w + jitter * np.eye(len(sigma_w)))
+        except np.linalg.LinAlgError as e:
+            raise NotPositiveDefinite(str(e)) from e
+
+
+def _sorted_eig(m: np.ndarray):
+    """Eigenpairs of a symmetric matrix, descending, with the sign convention above."""
+    lam, u = np.linalg.eigh(m)
+    order = np.argsort(-lam, kind="stable")
+    lam = lam[order]
+    u = u[:, order].copy()
+    for c in range(u.shape[1]):
+        i = int(np.argmax(np.abs(u[:, c])))     # first index of the max magnitude
+        if u[i, c] < 0:
+            u[:, c] = -u[:, c]
+    lam = np.maximum(lam, 1e-12 * max(lam[0], 0.0))
+    return lam, u
+
+
+def block_transform_pair(sigma_x: np.ndarray, sigma_w: np.ndarray, kind: str):
+    """(T_X, T_W) for one b x b block from its two second moments, fp64."""
+    b = sigma_x.shape[0]
+    if kind == "identity":
+        return np.eye(b), np.eye(b)
+    hn = normalized_hadamard(b)
+    if kind == "hadamard":
+        return hn.copy(), hn.copy()
+    if kind not in ("wus", "wush"):
+        raise ValueError(kind)
+    wp = _cholesky(sigma_w)
+    m = wp.T @ sigma_x @ wp
+    lam, u = _sorted_eig(m)
+    s = np.sqrt(lam)
+    left = hn if kind == "wush" else np.eye(b)
+    t_x = left @ np.diag(s ** -0.5) @ u.T @ wp.T
+    t_w = left @ np.diag(s ** 0.5) @ u.T @ np.linalg.inv(wp)
+    return t_x, t_w
+
+
+def transforms_from_moments(sigma_x: np.ndarray, sigma_w: np.ndarray, kind: str):
+    """(T_X, T_W) as [d_in/b, b, b] fp64 from per-block moments [d_in/b, b, b]."""
+    pairs = [block_transform_pair(sx, sw, kind) for sx, sw in zip(sigma_x, sigma_w)]
+    return np.stack([p[0] for p in pairs]), np.stack([p[1] for p in pairs])
+
+
+def calibrate(x_calib: np.ndarray, w_rows: np.ndarray, b: int, kind: str):
+    """(T_X, T_W) fp64 [d_in/b, b, b] from calibration tokens [n, d_in] and W^T [d_out, d_in]."""
+    return transforms_from_moments(block_moments(x_calib, b), block_moments(w_rows, b), kind)
+
+
+def nvfp4_global_scale(y_rows: np.ndarray) -> np.float32:
+    """Per-tensor NVFP4 scale s_g = amax / (6 * 448), returned as fp32.
+
+    Reading: the pages name NVFP4 only; the per-tensor fp32 scale is chosen so
+    that the largest calibration value maps to the largest E2M1 magnitude (6)
+    times the largest UE4M3 block scale (448).  For activations it is taken once
+    from the transformed calibration tokens (static), for weights from the
+    transformed weight tensor itself.
+    """
+    amax = float(np.max(np.abs(np.asarray(y_rows, dtype=np.float64))))
+    return np.float32(amax / (6.0 * 448.0))
