@@ -1,0 +1,197 @@
+"""Python binding of libwush.so: the B200 WUSH transform-then-quantize linear layer.
+
+Argument marshalling only: every step of the path runs in the library (host
+calibration in C++, everything else in sm_100a CUDA kernels).  Functions carry
+the C names declared in include/wush.h; device buffers are torch CUDA tensors
+(PyTorch provides memory and streams, nothing else), host buffers are numpy
+arrays.  A missing library raises ImportError: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libwush.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is not built; run `python -m activation_quantization_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+FORMATS = {"mxfp4": 0, "nvfp4": 1, "int4": 2}
+TRANSFORMS = {"identity": 0, "hadamard": 1, "wus": 2, "wush": 3}
+IN_BF16, IN_FP32 = 0, 1
+
+_i64, _i32, _f32, _vp, _sz = ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+
+_SIGNATURES = {
+    "wush_status_string": (ctypes.c_char_p, [_i32]),
+    "wush_block_size": (_i32, [_i32]),
+    "wush_calibrate": (_i32, [_vp, _i64, _vp, _i64, _i64, _i32, _i32, _vp, _vp]),
+    "wush_calibrate_from_moments": (_i32, [_vp, _vp, _i64, _i32, _i32, _vp, _vp]),
+    "wush_codes_bytes": (_sz, [_i64, _i64, _i32]),
+    "wush_scales_bytes": (_sz, [_i64, _i64, _i32]),
+    "wush_transform_quant": (_i32, [_vp, _i32, _i64, _i64, _vp, _i32, _i32, _f32, _vp, _vp, _vp, _vp]),
+    "wush_transform_amax": (_i32, [_vp, _i32, _i64, _i64, _vp, _i32, _i32, _vp, _vp]),
+    "wush_qgemm": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _f32, _vp, _vp]),
+    "itq3_quantize_weights": (_i32, [_vp, _i64, _i64, _vp, _vp]),
+    "itq3_dequant_gemv": (_i32, [_vp, _vp, _vp, _i64, _i64, _i64, _i32, _vp, _vp, _vp]),
+    "wush_check_device_status": (_i32, [_vp]),
+    "wush_debug_set_wait_limit": (_i32, [_i64]),
+}
+
+EXPORTED = []
+for _name, (_res, _args) in _SIGNATURES.items():
+    _fn = getattr(_lib, _name, None)
+    if _fn is None:
+        continue
+    _fn.restype = _res
+    _fn.argtypes = _args
+    EXPORTED.append(_name)
+
+
+class WushError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn}: {_lib.wush_status_string(status).decode()} ({status})")
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise WushError(fn, status)
+
+
+def _enum(table, v):
+    return table[v] if isinstance(v, str) else int(v)
+
+
+def _ptr(t):
+    """Device pointer of a torch tensor (None -> NULL)."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+def _host(a, dtype):
+    a = np.ascontiguousarray(a, dtype=dtype)
+    return a, a.ctypes.data
+
+
+# --------------------------------------------------------------------------- host
+
+def wush_block_size(fmt) -> int:
+    return _lib.wush_block_size(_enum(FORMATS, fmt))
+
+
+def wush_calibrate(x_calib: np.ndarray, w: np.ndarray, block: int, kind):
+    """(t_x, t_w) fp32 [d_in/block, block, block] from calibration tokens [n, d_in] and W^T [d_out, d_in]."""
+    x, xp = _host(x_calib, np.float32)
+    wt, wp = _host(w, np.float32)
+    d_in = x.shape[1]
+    if wt.shape[1] != d_in:
+        raise ValueError("d_in mismatch")
+    tx = np.empty((d_in // block, block, block), np.float32)
+    tw = np.empty_like(tx)
+    _check("wush_calibrate", _lib.wush_calibrate(xp, x.shape[0], wp, wt.shape[0], d_in, block,
+                                                 _enum(TRANSFORMS, kind), tx.ctypes.data, tw.ctypes.data))
+    return tx, tw
+
+
+def wush_calibrate_from_moments(sigma_x: np.ndarray, sigma_w: np.ndarray, kind):
+    sx, sxp = _host(sigma_x, np.float64)
+    sw, swp = _host(sigma_w, np.float64)
+    nb, b, _ = sx.shape
+    tx = np.empty((nb, b, b), np.float32)
+    tw = np.empty_like(tx)
+    _check("wush_calibrate_from_moments",
+           _lib.wush_calibrate_from_moments(sxp, swp, nb * b, b, _enum(TRANSFORMS, kind),
+                                            tx.ctypes.data, tw.ctypes.data))
+    return tx, tw
+
+
+def itq3_quantize_weights(w_fp16: np.ndarray):
+    """(packed codes uint8 [d_out * d_in * 3 / 8], scales fp16 [d_out, d_in/256]) from fp16 W [d_out, d_in]."""
+    w, wp = _host(w_fp16, np.float16)
+    d_out, d_in = w.shape
+    codes = np.empty(d_out * d_in * 3 // 8, np.uint8)
+    scales = np.empty((d_out, d_in // 256), np.float16)
+    _check("itq3_quantize_weights",
+           _lib.itq3_quantize_weights(wp, d_out, d_in, codes.ctypes.data, scales.ctypes.data))
+    return codes, scales
+
+
+# --------------------------------------------------------------------------- device
+
+def wush_codes_bytes(rows: int, d_in: int, fmt) -> int:
+    return _lib.wush_codes_bytes(rows, d_in, _enum(FORMATS, fmt))
+
+
+def wush_scales_bytes(rows: int, d_in: int, fmt) -> int:
+    return _lib.wush_scales_bytes(rows, d_in, _enum(FORMATS, fmt))
+
+
+def alloc_quant_outputs(rows: int, d_in: int, fmt, device="cuda"):
+    """Empty (codes, scales) uint8 CUDA tensors sized for wush_transform_quant."""
+    import torch
+    codes = torch.empty(wush_codes_bytes(rows, d_in, fmt), dtype=torch.uint8, device=device)
+    scales = torch.empty(max(wush_scales_bytes(rows, d_in, fmt), 16), dtype=torch.uint8, device=device)
+    return codes, scales
+
+
+def wush_transform_quant(x, t, kind, fmt, codes, scales, global_scale: float = 0.0, y_debug=None,
+                         stream=None):
+    """x: CUDA [rows, d_in] bf16 or fp32; t: CUDA fp32 [d_in/b, b, b] or None."""
+    import torch
+    x_dtype = IN_FP32 if x.dtype == torch.float32 else IN_BF16
+    if x.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("x must be bf16 or fp32")
+    rows, d_in = x.shape
+    _check("wush_transform_quant",
+           _lib.wush_transform_quant(_ptr(x), x_dtype, rows, d_in, _ptr(t), _enum(TRANSFORMS, kind),
+                                     _enum(FORMATS, fmt), float(global_scale), _ptr(codes), _ptr(scales),
+                                     _ptr(y_debug), _stream(stream)))
+
+
+def wush_transform_amax(x, t, kind, block: int, amax_out, stream=None):
+    import torch
+    x_dtype = IN_FP32 if x.dtype == torch.float32 else IN_BF16
+    rows, d_in = x.shape
+    _check("wush_transform_amax",
+           _lib.wush_transform_amax(_ptr(x), x_dtype, rows, d_in, _ptr(t), _enum(TRANSFORMS, kind), block,
+                                    _ptr(amax_out), _stream(stream)))
+
+
+def wush_qgemm(a_codes, a_scales, b_codes, b_scales, M: int, N: int, K: int, fmt, alpha: float, y,
+               stream=None):
+    _check("wush_qgemm",
+           _lib.wush_qgemm(_ptr(a_codes), _ptr(a_scales), _ptr(b_codes), _ptr(b_scales), M, N, K,
+                           _enum(FORMATS, fmt), float(alpha), _ptr(y), _stream(stream)))
+
+
+def itq3_dequant_gemv(codes, scales, x, d_out: int, mode: int, y, workspace=None, stream=None):
+    tokens, d_in = x.shape
+    _check("itq3_dequant_gemv",
+           _lib.itq3_dequant_gemv(_ptr(codes), _ptr(scales), _ptr(x), tokens, d_out, d_in, int(mode),
+                                  _ptr(workspace), _ptr(y), _stream(stream)))
+
+
+def wush_check_device_status(stream=None) -> int:
+    return _lib.wush_check_device_status(_stream(stream))
+
+
+def wush_debug_set_wait_limit(max_polls: int):
+    _check("wush_debug_set_wait_limit", _lib.wush_debug_set_wait_limit(int(max_polls)))

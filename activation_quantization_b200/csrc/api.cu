@@ -1,0 +1,33 @@
+// Status strings, the device error word and the diagnostics entry points.
+#include "common.cuh"
+
+namespace wush {
+// Poll limit for bounded mbarrier waits in the GEMM (0 = default); see wush.h.
+int64_t g_wait_limit_override = 0;
+}  // namespace wush
+
+extern "C" const char* wush_status_string(int status) {
+  switch (status) {
+    case WUSH_OK: return "ok";
+    case WUSH_ERR_INVALID_ARG: return "invalid argument";
+    case WUSH_ERR_UNSUPPORTED: return "unsupported format, transform or size";
+    case WUSH_ERR_NOT_SPD: return "weight second moment is not positive definite";
+    case WUSH_ERR_CUDA: return "CUDA error";
+    case WUSH_ERR_TIMEOUT: return "a bounded device wait gave up";
+    case WUSH_ERR_BUFFER_TOO_SMALL: return "buffer too small";
+    default: return "unknown status";
+  }
+}
+
+extern "C" int wush_check_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return WUSH_ERR_CUDA;
+  int word = 0;
+  if (wush::read_and_clear_error_word(&word) != cudaSuccess) return WUSH_ERR_CUDA;
+  return word == 0 ? WUSH_OK : WUSH_ERR_TIMEOUT;
+}
+
+extern "C" int wush_debug_set_wait_limit(int64_t max_polls) {
+  if (max_polls < 0) return WUSH_ERR_INVALID_ARG;
+  wush::g_wait_limit_override = max_polls;
+  return WUSH_OK;
+}

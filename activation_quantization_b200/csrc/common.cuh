@@ -1,0 +1,39 @@
+// Shared device helpers of the CUDA library (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "wush.h"
+
+namespace wush {
+
+// Bits of the device error word that kernels with bounded waits set when a wait
+// gives up (see wush_check_device_status).  The word lives in qgemm.cu.
+enum : int { kErrTimeoutBarrier = 1, kErrTimeoutTmem = 2 };
+
+// Reads the device error word of the GEMM translation unit into *word and clears
+// it; returns a cudaError_t as int.
+int read_and_clear_error_word(int* word);
+
+// Poll limit for bounded mbarrier waits (0 = the built-in default).
+extern int64_t g_wait_limit_override;
+
+inline int launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? WUSH_OK : WUSH_ERR_CUDA;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Byte offset of scale (r, c) in the block-scaled MMA scale-factor tile layout:
+// 128-row x 4-column atoms of 512 bytes, (r, c) at (r%32)*16 + (r/32)*4 + c inside
+// an atom, atoms ordered row-block-major.
+__host__ __device__ __forceinline__ int64_t sf_offset(int64_t r, int64_t c, int64_t n_atom_cols) {
+  return ((r >> 7) * n_atom_cols + (c >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (c & 3);
+}
+
+}  // namespace wush

@@ -1,0 +1,306 @@
+// Block-scaled FP4 GEMM on tcgen05 tensor cores: y = alpha * dq(A) dq(B)^T.
+//
+// AI Radio episode "WUSH: Near-Optimal Adaptive Transforms for LLM Quantization",
+// "Conclusion": the W4A4 layer runs an FP4 MatMul (up to 5.8x per layer over
+// BF16).  A holds the quantised activations [M = tokens, K = d_in], B the
+// quantised weights [N = d_out, K]; both are packed E2M1 codes, K contiguous, with
+// block scales in the MMA scale-factor tile layout written by
+// wush_transform_quant: UE8M0 per 32 (MXFP4, kind::mxf4, block32) or UE4M3 per 16
+// (NVFP4, kind::mxf4nvf4, block16).  Products of codes and scales are exact;
+// accumulation is fp32 in TMEM.
+//
+// One CTA computes one 128 x BN output tile (BN = 256, or 128 when N % 256 != 0)
+// with 4 warps:
+//   warp 0  TMA producer: per 256-wide k-tile, one 2D TMA load of the A tile
+//           (128 rows x 128 bytes, 128-byte swizzle), one of the B tile, and
+//           untiled bulk copies of the matching 512-byte scale atoms, all
+//           completing on the stage's "full" mbarrier;
+//   warp 1  allocates TMEM; one elected thread copies the stage's scale atoms
+//           into TMEM (tcgen05.cp 32x128b.warpx4) and issues the four K=64
+//           block-scaled MMAs, then commits the stage back to the producer;
+//   warps 0-3  epilogue: tcgen05.ld of the fp32 accumulator rows, times alpha,
+//           stored to y.
+// Every mbarrier wait is bounded (poll count, wall time, and a shared abort
+// flag); a wait that gives up records a device error word and the CTA drains
+// and frees its TMEM before returning.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace wush {
+
+static __device__ int g_error_word = 0;
+
+int read_and_clear_error_word(int* word) {
+  cudaError_t e = cudaMemcpyFromSymbol(word, g_error_word, sizeof(int));
+  if (e != cudaSuccess) return e;
+  if (*word) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_error_word, &zero, sizeof(int));
+  }
+  return e;
+}
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kBM = 128;
+constexpr int kBK = 256;             // fp4 elements per k-tile = 128 bytes per row
+constexpr int kBKBytes = kBK / 2;
+constexpr int kStages = 4;
+constexpr int kThreads = 128;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSfaCol = 256;    // TMEM column of the A scale factors
+constexpr uint32_t kSfbCol = 288;    // TMEM column of the B scale factors
+constexpr int64_t kDefaultPolls = int64_t(1) << 40;
+constexpr uint64_t kDeadlineNs = 4000000000ull;  // 4 s of wall time per wait
+
+template <int BN, bool NV>
+struct Cfg {
+  static constexpr int kAtomsK = NV ? 4 : 2;             // 512-byte scale atoms per row block per k-tile
+  static constexpr int kRowAtomsB = BN / 128;
+  static constexpr int kABytes = kBM * kBKBytes;         // 16 KB
+  static constexpr int kBBytes = BN * kBKBytes;          // 32 KB or 16 KB
+  static constexpr int kSfaBytes = kAtomsK * 512;
+  static constexpr int kSfbBytes = kRowAtomsB * kAtomsK * 512;
+  static constexpr int kStageBytes = ((kABytes + kBBytes + kSfaBytes + kSfbBytes + 1023) / 1024) * 1024;
+  static constexpr int kTxBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+};
+
+template <int BN, bool NV>
+__global__ void __launch_bounds__(kThreads, 1)
+    qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                 const uint8_t* __restrict__ sfa, const uint8_t* __restrict__ sfb, float* __restrict__ y,
+                 int M, int N, int K, float alpha, int64_t max_polls, int debug_never) {
+  using C = Cfg<BN, NV>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * C::kStageBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* acc_full = empty + kStages;
+  uint64_t* never = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const int n_blk = blockIdx.x;
+  const int m_blk = blockIdx.y;
+  const int k_tiles = K / kBK;
+  const int n_acols = (K / (NV ? 16 : 32) + 3) / 4;     // scale atoms per 128-row block
+  const uint64_t deadline = globaltimer_ns() + kDeadlineNs;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(never, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tmap_a);
+    prefetch_tmap(&tmap_b);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (elect_one()) {
+      for (int kt = 0; kt < k_tiles; ++kt) {
+        const int s = kt % kStages;
+        const uint32_t ph = (kt / kStages) & 1;
+        if (!mbar_wait_bounded(&empty[s], ph ^ 1, max_polls, deadline, abort_flag)) {
+          if (!*abort_flag) { *abort_flag = 1; atomicOr(&g_error_word, 1 << kErrTimeoutBarrier); }
+          break;
+        }
+        uint8_t* st = smem + s * C::kStageBytes;
+        uint8_t* sa = st;
+        uint8_t* sb = sa + C::kABytes;
+        uint8_t* ssfa = sb + C::kBBytes;
+        uint8_t* ssfb = ssfa + C::kSfaBytes;
+        mbar_arrive_expect_tx(&full[s], C::kTxBytes);
+        tma_load_2d(sa, &tmap_a, kt * kBKBytes, m_blk * kBM, &full[s]);
+        tma_load_2d(sb, &tmap_b, kt * kBKBytes, n_blk * BN, &full[s]);
+        bulk_load(ssfa, sfa + (static_cast<int64_t>(m_blk) * n_acols + kt * C::kAtomsK) * 512, C::kSfaBytes,
+                  &full[s]);
+#pragma unroll
+        for (int h = 0; h < C::kRowAtomsB; ++h)
+          bulk_load(ssfb + h * C::kAtomsK * 512,
+                    sfb + (static_cast<int64_t>(n_blk * C::kRowAtomsB + h) * n_acols + kt * C::kAtomsK) * 512,
+                    C::kAtomsK * 512, &full[s]);
+      }
+    }
+  } else if (warp == 1) {
+    if (elect_one()) {
+      bool ok = true;
+      if (debug_never) {
+        // test hook: wait on a barrier nothing arrives on, to exercise the give-up path
+        ok = mbar_wait_bounded(never, 0, max_polls, deadline, abort_flag);
+      }
+      const uint32_t tsfa = tmem + kSfaCol;
+      const uint32_t tsfb = tmem + kSfbCol;
+      for (int kt = 0; ok && kt < k_tiles; ++kt) {
+        const int s = kt % kStages;
+        const uint32_t ph = (kt / kStages) & 1;
+        if (!mbar_wait_bounded(&full[s], ph, max_polls, deadline, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        uint8_t* st = smem + s * C::kStageBytes;
+        const uint32_t sa = smem_u32(st);
+        const uint32_t sb = sa + C::kABytes;
+        const uint32_t ssfa = sb + C::kBBytes;
+        const uint32_t ssfb = ssfa + C::kSfaBytes;
+#pragma unroll
+        for (int a = 0; a < C::kAtomsK; ++a) {
+          tc_cp_32x128b_warpx4(tsfa + 4 * a, desc_sf_atom(ssfa + a * 512));
+#pragma unroll
+          for (int h = 0; h < C::kRowAtomsB; ++h)
+            tc_cp_32x128b_warpx4(tsfb + 4 * (C::kRowAtomsB * a + h), desc_sf_atom(ssfb + (h * C::kAtomsK + a) * 512));
+        }
+#pragma unroll
+        for (int kk = 0; kk < kBK / 64; ++kk) {
+          const int atom = NV ? kk : kk / 2;
+          const uint32_t sf_id = NV ? 0u : 2u * (kk & 1);
+          const uint32_t idesc = idesc_block_scaled_e2m1(kBM, BN, NV ? 0u : 1u, sf_id, sf_id);
+          const uint64_t ad = desc_kmajor_sw128(sa + kk * 32);
+          const uint64_t bd = desc_kmajor_sw128(sb + kk * 32);
+          mma_block_scaled<NV>(tmem, ad, bd, idesc, (kt | kk) ? 1u : 0u,
+                               (tsfa + 4 * atom) | (sf_id << 30),
+                               (tsfb + 4 * C::kRowAtomsB * atom) | (sf_id << 30));
+        }
+        tc_commit(&empty[s]);
+      }
+      if (ok) {
+        tc_commit(acc_full);
+      } else if (!*abort_flag) {
+        *abort_flag = 1;
+        atomicOr(&g_error_word, 1 << kErrTimeoutBarrier);
+      }
+    }
+  }
+  __syncwarp();
+
+  // epilogue: every warp drains its 32 TMEM lanes (rows 32*warp .. 32*warp + 31)
+  bool have_acc = mbar_wait_bounded(acc_full, 0, max_polls, deadline, abort_flag);
+  if (!have_acc && !*abort_flag) {
+    *abort_flag = 1;
+    atomicOr(&g_error_word, 1 << kErrTimeoutBarrier);
+  }
+  have_acc = __all_sync(0xffffffffu, have_acc);
+  if (have_acc) {
+    tc_fence_after();
+    const int row = m_blk * kBM + warp * 32 + lane;
+    float* yrow = y + static_cast<int64_t>(row) * N + static_cast<int64_t>(n_blk) * BN;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      uint32_t r[32];
+      tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c, r);
+      tmem_ld_wait();
+      float4* dst = reinterpret_cast<float4*>(yrow + c);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        dst[q] = make_float4(alpha * __uint_as_float(r[4 * q]), alpha * __uint_as_float(r[4 * q + 1]),
+                             alpha * __uint_as_float(r[4 * q + 2]), alpha * __uint_as_float(r[4 * q + 3]));
+    }
+  }
+  if (*abort_flag) {
+    // let loads and MMAs already issued by this CTA land before its shared memory
+    // and TMEM are released
+    const uint64_t until = globaltimer_ns() + 200000ull;
+    while (globaltimer_ns() < until) __nanosleep(1000);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn get_encode() {
+  static EncodeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(p);
+  });
+  return fn;
+}
+
+// 2D map over a [rows, row_bytes] uint8 matrix, box = box_rows x 128 bytes, 128-byte swizzle.
+bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t row_bytes, int box_rows) {
+  EncodeFn enc = get_encode();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBKBytes), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, bool NV>
+int launch(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const uint8_t* sfb, int64_t M, int64_t N,
+           int64_t K, float alpha, float* y, cudaStream_t st) {
+  using C = Cfg<BN, NV>;
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, a, M, K / 2, kBM) || !make_map(&mb, b, N, K / 2, BN)) return WUSH_ERR_CUDA;
+  auto kern = qgemm_kernel<BN, NV>;
+  static uint64_t attr_done = 0;  // one bit per device: dynamic shared memory opt-in done
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return WUSH_ERR_CUDA;
+  if (dev < 64 && !(attr_done >> dev & 1)) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+      return WUSH_ERR_CUDA;
+    attr_done |= uint64_t(1) << dev;
+  }
+  const int64_t polls = g_wait_limit_override > 0 ? g_wait_limit_override : kDefaultPolls;
+  const int debug_never = g_wait_limit_override > 0 ? 1 : 0;
+  const dim3 grid(static_cast<unsigned>(N / BN), static_cast<unsigned>(M / kBM));
+  kern<<<grid, kThreads, C::kSmemBytes, st>>>(ma, mb, sfa, sfb, y, static_cast<int>(M), static_cast<int>(N),
+                                              static_cast<int>(K), alpha, polls, debug_never);
+  return launch_status();
+}
+
+}  // namespace
+}  // namespace wush
+
+using namespace wush;
+
+extern "C" int wush_qgemm(const uint8_t* a_codes, const void* a_scales, const uint8_t* b_codes,
+                          const void* b_scales, int64_t M, int64_t N, int64_t K, int fmt, float alpha, float* y,
+                          void* stream) {
+  if (fmt != WUSH_FMT_MXFP4 && fmt != WUSH_FMT_NVFP4) return WUSH_ERR_UNSUPPORTED;
+  if (M <= 0 || N <= 0 || K <= 0 || M % 128 || N % 128 || K % 256) return WUSH_ERR_INVALID_ARG;
+  if (M > (int64_t(1) << 30) || N > (int64_t(1) << 30) || K > (int64_t(1) << 30) || N / 128 > 65535 * 128)
+    return WUSH_ERR_UNSUPPORTED;
+  if (!a_codes || !a_scales || !b_codes || !b_scales || !y) return WUSH_ERR_INVALID_ARG;
+  if (!aligned16(a_codes) || !aligned16(b_codes) || !aligned16(a_scales) || !aligned16(b_scales) || !aligned16(y))
+    return WUSH_ERR_INVALID_ARG;
+  if (M / 128 > 65535) return WUSH_ERR_UNSUPPORTED;
+  const auto* sa = static_cast<const uint8_t*>(a_scales);
+  const auto* sb = static_cast<const uint8_t*>(b_scales);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool nv = fmt == WUSH_FMT_NVFP4;
+  if (N % 256 == 0) {
+    return nv ? launch<256, true>(a_codes, sa, b_codes, sb, M, N, K, alpha, y, st)
+              : launch<256, false>(a_codes, sa, b_codes, sb, M, N, K, alpha, y, st);
+  }
+  return nv ? launch<128, true>(a_codes, sa, b_codes, sb, M, N, K, alpha, y, st)
+            : launch<128, false>(a_codes, sa, b_codes, sb, M, N, K, alpha, y, st);
+}

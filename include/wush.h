@@ -1,0 +1,237 @@
+/*
+ * wush.h -- C ABI of the B200 WUSH transform-then-quantize linear layer.
+ *
+ * The layer (AI Radio episode "WUSH: Near-Optimal Adaptive Transforms for LLM
+ * Quantization", "Problem Setup and Goal") computes
+ *     y = q(T_W W)^T q(T_X X)
+ * with per-block transforms T_X, T_W = T_X^{-T} built from second moments
+ * (WUSH news article, paragraphs on the construction and the deployment
+ * workflow), microscaled low-bit quantisation q (MXFP4, NVFP4, INT4; WUSH news
+ * article, experiments paragraph) and a block-scaled FP4 GEMM (AI Radio
+ * episode, "Conclusion").  An ITQ3_S-style 3-bit weight path with a 256-wide
+ * Walsh-Hadamard rotation (ITQ3_S article, "核心技术：FWHT预旋转与TurboQuant的完美融合")
+ * is a secondary variant.
+ *
+ * Storage conventions (PyTorch-native, K contiguous):
+ *   activations X^T : [rows = tokens, d_in] row-major
+ *   weights     W^T : [d_out, d_in]        row-major (the same row transform)
+ *   output      y^T : [tokens, d_out]      row-major, fp32
+ * A transform block is ``b`` consecutive d_in elements of one row; b is also the
+ * quantisation group: 32 for MXFP4 and INT4, 16 for NVFP4.  Block j of a row,
+ * x_j, is replaced by T[j] x_j with T stored as fp32 [d_in/b, b, b], T[j][i][k]
+ * at ((j*b)+i)*b+k.
+ *
+ * General rules for every entry point:
+ *   - The caller owns every buffer; no entry point allocates device memory and
+ *     none synchronises the stream unless it says so.
+ *   - "device" pointers are CUDA device (or managed) memory; "host" pointers are
+ *     ordinary host memory.
+ *   - Every argument is checked before any launch. A failed check returns
+ *     WUSH_ERR_INVALID_ARG / WUSH_ERR_UNSUPPORTED and launches nothing.
+ *   - A CUDA launch error returns WUSH_ERR_CUDA (cudaGetLastError after launch).
+ *   - Device pointers must be 16-byte aligned.
+ *   - ``stream`` is a cudaStream_t passed as void*; NULL is the legacy default
+ *     stream.  Work is enqueued in stream order.
+ *   - Inputs must be finite; non-finite values give unspecified codes.
+ *   - Waits inside kernels are bounded. A kernel that gives up sets a device
+ *     error word which wush_check_device_status() reports as WUSH_ERR_TIMEOUT.
+ */
+#ifndef WUSH_H
+#define WUSH_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  WUSH_OK = 0,
+  WUSH_ERR_INVALID_ARG = -1,
+  WUSH_ERR_UNSUPPORTED = -2,
+  WUSH_ERR_NOT_SPD = -3,
+  WUSH_ERR_CUDA = -4,
+  WUSH_ERR_TIMEOUT = -5,
+  WUSH_ERR_BUFFER_TOO_SMALL = -6
+} wush_status;
+
+typedef enum { WUSH_FMT_MXFP4 = 0, WUSH_FMT_NVFP4 = 1, WUSH_FMT_INT4 = 2 } wush_format;
+
+typedef enum {
+  WUSH_T_IDENTITY = 0,
+  WUSH_T_HADAMARD = 1,
+  WUSH_T_WUS = 2,
+  WUSH_T_WUSH = 3
+} wush_transform;
+
+typedef enum { WUSH_IN_BF16 = 0, WUSH_IN_FP32 = 1 } wush_input_dtype;
+
+/* Human-readable name of a status code (static storage). */
+const char* wush_status_string(int status);
+
+/* Block size (quantisation group) of a format: 32, 16, 32. 0 for an unknown format. */
+int wush_block_size(int fmt);
+
+/* ---------------------------------------------------------------------------
+ * Calibration (host, fp64 inside, not on the timed path)
+ *
+ * WUSH news article, paragraph 3 (W = Cholesky factor of the weights, U and S
+ * from an SVD, H = Hadamard; second-order statistics of weights and
+ * activations) and paragraph 6 (collect moments from calibration data, then
+ * Cholesky and SVD per block, in parallel).  Per block j:
+ *   Sigma_X = X_j X_j^T / n_calib,  Sigma_W = W_j W_j^T / d_out,
+ *   W' = chol(Sigma_W) (lower),  W'^T Sigma_X W' = U diag(lambda) U^T,
+ *   S = diag(sqrt(lambda)) (descending),  Hn = H_b / sqrt(b),
+ *   T_X = Hn S^{-1/2} U^T W'^T,   T_W = T_X^{-T} = Hn S^{1/2} U^T W'^{-1}.
+ * WUS drops Hn; HADAMARD gives T_X = T_W = Hn; IDENTITY gives I.
+ * Columns of U are signed so that their largest-magnitude entry is positive
+ * (ties: lowest index); eigenvalues are floored at 1e-12 * max.  A Cholesky
+ * failure is retried once with Sigma_W + 1e-8 * mean(diag) I; if that fails
+ * too, WUSH_ERR_NOT_SPD.
+ * ------------------------------------------------------------------------- */
+
+/* x_calib: host fp32 [n_calib, d_in]; w: host fp32 [d_out, d_in] (W^T);
+ * block in {16, 32} (any power of two 2..256 is accepted), d_in % block == 0;
+ * t_x, t_w: host fp32 outputs [d_in/block, block, block].  Uses the host's cores. */
+int wush_calibrate(const float* x_calib, int64_t n_calib, const float* w, int64_t d_out,
+                   int64_t d_in, int block, int kind, float* t_x, float* t_w);
+
+/* The same from precomputed per-block moments (host fp64 [d_in/block, block, block],
+ * e.g. from existing Hessians); t_x, t_w as above. */
+int wush_calibrate_from_moments(const double* sigma_x, const double* sigma_w, int64_t d_in,
+                                int block, int kind, float* t_x, float* t_w);
+
+/* ---------------------------------------------------------------------------
+ * Output buffer sizes for wush_transform_quant (bytes)
+ *
+ * codes:  two 4-bit codes per byte, K contiguous, lower d_in index in the low
+ *         nibble: rows * d_in / 2 bytes.
+ * scales: MXFP4 (UE8M0, one byte per 32) and NVFP4 (UE4M3, one byte per 16) are
+ *         written in the scale-factor tile layout of the block-scaled MMA: the
+ *         rows x (d_in/b) scale matrix is cut into 128-row x 4-column atoms of
+ *         512 contiguous bytes; scale (r, c) of an atom sits at byte
+ *         (r % 32) * 16 + (r / 32) * 4 + c; atoms are ordered row-block-major
+ *         (all column atoms of rows 0..127 first).  rows is padded up to 128 and
+ *         d_in/b up to 4; padding bytes are not written.
+ *         INT4 scales are fp16, plain row-major [rows, d_in/32].
+ * ------------------------------------------------------------------------- */
+size_t wush_codes_bytes(int64_t rows, int64_t d_in, int fmt);
+size_t wush_scales_bytes(int64_t rows, int64_t d_in, int fmt);
+
+/* ---------------------------------------------------------------------------
+ * Fused block transform + microscaled quantisation (device, one launch)
+ *
+ * WUSH news article, paragraph 6: at inference only the input activations are
+ * transformed (weights are transformed and quantised once, offline, with the
+ * same call and T_W); AI Radio episode, "The gist": the transform admits a fused
+ * GPU implementation.  Rules per format (the pages name the formats only):
+ *   MXFP4: amax = max|y| over 32; e = clamp(floor(log2 amax) - 2, -127, 127)
+ *          (e = -127 for amax 0); scale byte e + 127; code = E2M1 RNE-satfinite
+ *          of y / 2^e.
+ *   NVFP4: t = amax / fp32(6 * global_scale); s_b = UE4M3 RNE-satfinite(t);
+ *          d = fp32(s_b * global_scale); code = E2M1 RNE-satfinite(y / d);
+ *          codes 0 when s_b = 0.  global_scale is the per-tensor fp32 scale.
+ *   INT4:  s = fp16 RNE(amax / 7); q = clamp(rint(y / s), -7, 7) (0 if s = 0);
+ *          code = q & 0xF (two's complement nibble).
+ *   All decisions in fp32 with round-to-nearest-even. E2M1 codes carry the
+ *   sign of y even when the magnitude rounds to 0; an all-zero block gives +0.
+ *
+ * x:       device [rows, d_in], bf16 (x_dtype = WUSH_IN_BF16) or fp32.
+ * t:       device fp32 [d_in/b, b, b] for WUS/WUSH; ignored (may be NULL) for
+ *          IDENTITY and HADAMARD (computed with in-register butterflies, then
+ *          scaled by the fp32 constant 1/sqrt(b)).
+ * codes:   device, wush_codes_bytes(rows, d_in, fmt) bytes.
+ * scales:  device, wush_scales_bytes(rows, d_in, fmt) bytes.
+ * y_debug: optional device fp32 [rows, d_in] receiving the transformed values
+ *          before rounding (NULL to skip; costs 4 bytes/element of traffic).
+ * Requirements: rows >= 0 (0 is a no-op), d_in % b == 0, d_in > 0.
+ * ------------------------------------------------------------------------- */
+int wush_transform_quant(const void* x, int x_dtype, int64_t rows, int64_t d_in,
+                         const float* t, int kind, int fmt, float global_scale,
+                         uint8_t* codes, void* scales, float* y_debug, void* stream);
+
+/* max |T x| over a whole [rows, d_in] tensor, written as one fp32 to device
+ * *amax_out (the call zeroes it first, in stream order).  Used offline for the
+ * per-tensor NVFP4 scale global_scale = amax / (6 * 448) of a transformed
+ * weight or calibration tensor.  Arguments as in wush_transform_quant with the
+ * block size b given explicitly (16 or 32). */
+int wush_transform_amax(const void* x, int x_dtype, int64_t rows, int64_t d_in,
+                        const float* t, int kind, int block, float* amax_out, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Block-scaled FP4 GEMM on tcgen05 tensor cores (device)
+ *
+ * AI Radio episode, "Conclusion": the W4A4 layer runs an FP4 MatMul (up to
+ * 5.8x per layer over BF16).  y[m, n] = alpha * sum_k dq(a)[m, k] dq(b)[n, k]
+ * with dq the element code times its block scale, products exact and fp32
+ * accumulation.
+ *
+ * a_codes/a_scales: activation codes and scales from wush_transform_quant
+ *                   (rows = M, d_in = K).
+ * b_codes/b_scales: weight codes and scales from wush_transform_quant
+ *                   (rows = N, d_in = K).
+ * fmt:    WUSH_FMT_MXFP4 (UE8M0 per 32) or WUSH_FMT_NVFP4 (UE4M3 per 16).
+ * alpha:  fp32 epilogue scale (NVFP4: global_scale_x * global_scale_w; MXFP4: 1).
+ * y:      device fp32 [M, N] row-major, overwritten.
+ * Requirements: M % 128 == 0, N % 128 == 0, K % 256 == 0, all > 0.
+ * ------------------------------------------------------------------------- */
+int wush_qgemm(const uint8_t* a_codes, const void* a_scales, const uint8_t* b_codes,
+               const void* b_scales, int64_t M, int64_t N, int64_t K, int fmt, float alpha,
+               float* y, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * ITQ3_S-style 3-bit weights with a 256-wide Walsh-Hadamard rotation
+ *
+ * ITQ3_S article, "核心技术：FWHT预旋转与TurboQuant的完美融合": each 256-element
+ * weight vector (256 consecutive d_in weights of one output row) is rotated with
+ * the FWHT before a uniform 3-bit quantiser, and the exact inverse transform is
+ * applied when the weights are loaded for the matmul.
+ *   r = H_256 w / 16;  s = fp16 RNE(max|r| / 3.5);
+ *   c = clamp(rint(r / s + 3.5), 0, 7) (c = 0 when s = 0), all in fp64;
+ *   dequantised w_hat = H_256 ((c - 3.5) s) / 16.
+ * Packed code layout (our own; the article calls its layout "interleaved"
+ * without detail): per row and 256-block, 24 little-endian uint32 words; word
+ * p*8 + i holds bit p (p = 0, 1, 2) of the codes of elements 32*i .. 32*i + 31,
+ * element 32*i + l in bit l.  96 bytes per 256 weights, rows * d_in * 3 / 8 in all.
+ * ------------------------------------------------------------------------- */
+
+/* Host: w_fp16 host fp16 bits [d_out, d_in]; d_in % 256 == 0;
+ * codes: host, d_out * d_in * 3 / 8 bytes; scales_fp16: host fp16 bits [d_out, d_in/256]. */
+int itq3_quantize_weights(const uint16_t* w_fp16, int64_t d_out, int64_t d_in, uint8_t* codes,
+                          uint16_t* scales_fp16);
+
+/* y[t, o] = sum_k w_hat[o, k] x[t, k] on the device.
+ * codes, scales_fp16: device, as written by itq3_quantize_weights.
+ * x_fp16: device fp16 [tokens, d_in]; y: device fp32 [tokens, d_out], overwritten.
+ * mode 0: the inverse FWHT is applied to every weight block as it is loaded
+ *         (the article's fused design);
+ * mode 1: the algebraically identical activation-side form
+ *         sum_k ((c - 3.5) s)[o, k] (H_256 x / 16)[t, k]: x is rotated once per
+ *         call into ``workspace`` (device fp32 [tokens, d_in], caller-owned
+ *         scratch), then each weight is used without a transform.
+ * workspace may be NULL for mode 0.  Requirements: 1 <= tokens <= 16,
+ * d_in % 256 == 0, d_out % 8 == 0. */
+int itq3_dequant_gemv(const uint8_t* codes, const void* scales_fp16, const void* x_fp16,
+                      int64_t tokens, int64_t d_out, int64_t d_in, int mode, float* workspace,
+                      float* y, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Diagnostics
+ * ------------------------------------------------------------------------- */
+
+/* Synchronises ``stream``, then reports (and clears) the device error word set by
+ * a kernel whose bounded wait gave up: WUSH_ERR_TIMEOUT, else WUSH_OK, or
+ * WUSH_ERR_CUDA if the stream itself reports an error. */
+int wush_check_device_status(void* stream);
+
+/* Test hook: makes the next wush_qgemm launches give up their first barrier wait
+ * after ``max_polls`` polls (0 restores the default limit) so that the timeout
+ * path can be exercised without hanging anything. */
+int wush_debug_set_wait_limit(int64_t max_polls);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WUSH_H */

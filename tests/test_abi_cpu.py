@@ -1,0 +1,100 @@
+"""C-ABI library checks that need no GPU: exports, host calibration and ITQ3
+quantisation against the oracle, buffer sizes and argument validation."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import synth
+from oracle import calibrate as C
+from oracle import itq3 as I
+
+aq = pytest.importorskip("activation_quantization_b200")
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "wush.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:int|size_t|const char\*)\s+(\w+)\s*\(", src, flags=re.M)))
+
+
+def test_every_declared_symbol_is_exported():
+    lib = ctypes.CDLL(aq.LIB_PATH)
+    names = _declared()
+    assert len(names) >= 12
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(names) <= set(aq._SIGNATURES), "binding lacks a signature"
+
+
+@pytest.mark.parametrize("kind", ["identity", "hadamard", "wus", "wush"])
+def test_calibrate_matches_oracle(kind):
+    w = synth.WORKLOADS["tiny"]
+    xc, wt = synth.activations(w, calib=True), synth.weights(w)
+    for b in (16, 32):
+        tx, tw = aq.wush_calibrate(xc, wt, b, kind)
+        ox, ow = C.calibrate(xc, wt, b, kind)
+        for got, want in ((tx, ox), (tw, ow)):
+            scale = np.abs(want).max(axis=(1, 2), keepdims=True)
+            assert np.max(np.abs(got - want) / scale) < 1e-6
+
+
+def test_calibrate_from_moments_matches_calibrate():
+    w = synth.WORKLOADS["tiny"]
+    xc, wt = synth.activations(w, calib=True), synth.weights(w)
+    tx, tw = aq.wush_calibrate(xc, wt, 32, "wush")
+    mx, mw = C.block_moments(xc, 32), C.block_moments(wt, 32)
+    tx2, tw2 = aq.wush_calibrate_from_moments(mx, mw, "wush")
+    assert np.allclose(tx, tx2, rtol=1e-5, atol=1e-6 * np.abs(tx).max())
+
+
+def test_not_spd_status():
+    sx = np.broadcast_to(np.eye(4), (2, 4, 4)).copy()
+    with pytest.raises(aq.WushError) as e:
+        aq.wush_calibrate_from_moments(sx, -sx, "wush")
+    assert e.value.status == -3
+
+
+def _unpack_itq3(packed, d_out, d_in):
+    words = packed.view(np.uint32).reshape(d_out, d_in // 256, 3, 8)
+    bits = (words[..., None] >> np.arange(32, dtype=np.uint32)) & 1       # [o, blk, p, i, l]
+    c = bits[:, :, 0] | (bits[:, :, 1] << 1) | (bits[:, :, 2] << 2)        # [o, blk, i, l]
+    return c.reshape(d_out, d_in).astype(np.uint8)
+
+
+@pytest.mark.parametrize("shape", [(8, 256), (64, 1024)])
+def test_itq3_quantize_matches_oracle_bit_exact(shape):
+    w = synth.itq3_weights(*shape)
+    w[0, :256] = 0.0                                   # an all-zero block: s = 0, codes 0
+    codes, scales = aq.itq3_quantize_weights(w.astype(np.float16))
+    oc, os_ = I.quantize(w.astype(np.float16).astype(np.float64))
+    assert np.array_equal(scales.view(np.uint16), os_.view(np.uint16))
+    assert np.array_equal(_unpack_itq3(codes, *shape), oc)
+
+
+def test_buffer_sizes():
+    assert aq.wush_codes_bytes(4096, 4096, "mxfp4") == 8388608
+    assert aq.wush_scales_bytes(4096, 4096, "mxfp4") == 524288
+    assert aq.wush_scales_bytes(4096, 12288, "nvfp4") == 3145728
+    assert aq.wush_scales_bytes(8192, 5120, "int4") == 2621440
+    assert aq.wush_scales_bytes(130, 96, "mxfp4") == 2 * 1 * 512      # 2 row atoms x 1 col atom
+    assert aq.wush_block_size("nvfp4") == 16 and aq.wush_block_size(7) == 0
+
+
+def test_argument_validation_before_launch():
+    lib = aq._lib
+    # d_in not a multiple of the block, unknown format/kind, NULL pointers: no launch happens
+    assert lib.wush_transform_quant(16, 0, 4, 48, None, 0, 0, 0.0, 16, 16, None, None) == -1
+    assert lib.wush_transform_quant(16, 0, 4, 64, None, 0, 9, 0.0, 16, 16, None, None) == -2
+    assert lib.wush_transform_quant(16, 0, 4, 64, None, 7, 0, 0.0, 16, 16, None, None) == -2
+    assert lib.wush_transform_quant(None, 0, 4, 64, None, 0, 0, 0.0, 16, 16, None, None) == -1
+    assert lib.wush_transform_quant(16, 0, 4, 64, None, 3, 0, 0.0, 16, 16, None, None) == -1  # WUSH needs t
+    assert lib.wush_transform_quant(17, 0, 4, 64, None, 0, 0, 0.0, 16, 16, None, None) == -1  # misaligned
+    assert lib.wush_transform_quant(16, 0, 4, 64, None, 0, 1, 0.0, 16, 16, None, None) == -1  # NVFP4 s_g
+    assert lib.wush_transform_quant(16, 0, 0, 64, None, 0, 0, 0.0, 16, 16, None, None) == 0   # empty
+    assert lib.wush_calibrate(None, 0, None, 0, 64, 24, 3, 16, 16) == -1                      # block
+    assert lib.itq3_quantize_weights(16, 4, 100, 16, 16) == -1
+    assert lib.wush_status_string(-5) == b"a bounded device wait gave up"

@@ -1,0 +1,51 @@
+"""GPU parity: itq3_dequant_gemv (both modes) against the oracle's fp64 GEMV."""
+import numpy as np
+import pytest
+
+import synth
+from oracle import itq3 as I
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+def pack_codes(c):
+    """Test-side packer restating the header's bit-plane layout."""
+    d_out, d_in = c.shape
+    cb = c.reshape(d_out, d_in // 256, 8, 32).astype(np.uint32)        # [o, blk, i, l]
+    words = np.zeros((d_out, d_in // 256, 3, 8), np.uint32)
+    for p in range(3):
+        words[:, :, p, :] = np.sum(((cb >> p) & 1) << np.arange(32, dtype=np.uint32), axis=3).astype(np.uint32)
+    return words.reshape(-1).view(np.uint8)
+
+
+@pytest.mark.parametrize("shape", [(256, 1024), (4096, 4096)])
+@pytest.mark.parametrize("tokens", [1, 3, 4, 16])
+@pytest.mark.parametrize("mode", [0, 1])
+def test_itq3_gemv(lib, shape, tokens, mode):
+    d_out, d_in = shape
+    w = synth.itq3_weights(d_out, d_in)
+    x = synth.itq3_activations(tokens, d_in)
+    c, s = I.quantize(w)
+    want = I.gemv(c, s, x)
+    dev = "cuda"
+    y = torch.full((tokens, d_out), float("nan"), dtype=torch.float32, device=dev)
+    ws = torch.empty((tokens, d_in), dtype=torch.float32, device=dev) if mode == 1 else None
+    lib.itq3_dequant_gemv(torch.from_numpy(pack_codes(c)).to(dev), torch.from_numpy(s).to(dev),
+                          torch.from_numpy(x.astype(np.float16)).to(dev), d_out, mode, y, ws)
+    got = y.cpu().numpy().astype(np.float64)
+    err = np.linalg.norm(got - want) / np.linalg.norm(want)
+    assert err <= 1e-5, err
+
+
+def test_itq3_library_quantiser_feeds_gemv(lib):
+    w = synth.itq3_weights(512, 2048)
+    codes, scales = lib.itq3_quantize_weights(w.astype(np.float16))
+    x = synth.itq3_activations(4, 2048)
+    c, s = I.quantize(w)
+    want = I.gemv(c, s, x)
+    y = torch.empty((4, 512), dtype=torch.float32, device="cuda")
+    lib.itq3_dequant_gemv(torch.from_numpy(codes).cuda(), torch.from_numpy(scales).cuda(),
+                          torch.from_numpy(x.astype(np.float16)).cuda(), 512, 0, y)
+    err = np.linalg.norm(y.cpu().numpy() - want) / np.linalg.norm(want)
+    assert err <= 1e-5

@@ -1,0 +1,158 @@
+"""GPU parity: wush_transform_quant against the oracle, element by element.
+
+Codes and scales are bit-exact except where the oracle's pre-rounding value sits
+within 1e-6 (relative to the magnitude of the terms that form it) of a rounding
+boundary; those are counted and bounded (tests/parity.py).  Transformed values
+agree within 1e-5 of that magnitude.
+"""
+import functools
+
+import numpy as np
+import pytest
+
+import synth
+from oracle import calibrate as C
+from oracle import transforms as T
+from tests import parity as P
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+FMT_WORKLOAD = {"mxfp4": "up_proj", "nvfp4": "down_proj", "int4": "int4"}
+
+
+@functools.lru_cache(maxsize=None)
+def _calib_inputs(name, n_calib):
+    w = synth.WORKLOADS[name]
+    return synth.activations(w, tokens=n_calib, calib=True), synth.weights(w)[:2048]
+
+
+@functools.lru_cache(maxsize=None)
+def _transform_cached(kind, fmt, name, n_calib):
+    w = synth.WORKLOADS[name]
+    b = P.Q.BLOCK[fmt]
+    if kind in ("identity", "hadamard"):
+        return (T.identity_blocks(w.d_in, b) if kind == "identity" else T.hadamard_blocks(w.d_in, b)).astype(np.float32)
+    xc, wt = _calib_inputs(name, n_calib)
+    tx, _ = C.calibrate(xc, wt, b, kind)
+    return tx.astype(np.float32)
+
+
+def _transform(kind, fmt, w, n_calib=1024):
+    return _transform_cached(kind, fmt, w.name, n_calib)
+
+
+def _global_scale(x, t, fmt):
+    if fmt != "nvfp4":
+        return 0.0
+    return float(C.nvfp4_global_scale(T.apply_block_transform(x, t).astype(np.float32)))
+
+
+def _as_input(x, bf16):
+    if bf16:
+        return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32))
+
+
+def run_gpu_t(lib, xt_cpu, t, kind, fmt, gs):
+    rows, d_in = xt_cpu.shape
+    xt = xt_cpu.cuda()
+    tt = None if kind in ("identity", "hadamard") else torch.from_numpy(t).cuda()
+    codes, scales = lib.alloc_quant_outputs(rows, d_in, fmt)
+    y = torch.empty((rows, d_in), dtype=torch.float32, device="cuda")
+    lib.wush_transform_quant(xt, tt, kind, fmt, codes, scales, gs, y)
+    torch.cuda.synchronize()
+    return (P.unpack_nibbles(codes.cpu().numpy(), rows, d_in),
+            P.decode_scales(scales.cpu().numpy(), rows, d_in, fmt), y.cpu().numpy())
+
+
+@pytest.mark.parametrize("kind", ["identity", "hadamard", "wus", "wush"])
+def test_tiny_fp32_mxfp4(lib, kind):
+    w = synth.WORKLOADS["tiny"]
+    x = synth.activations(w)
+    t = _transform(kind, "mxfp4", w, n_calib=512)
+    c, s, y = run_gpu_t(lib, _as_input(x, False), t, kind, "mxfp4", 0.0)
+    out = P.compare_transform_quant(x, t, "mxfp4", None, c, s, y)
+    assert out["elements"] == x.size
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4", "int4"])
+@pytest.mark.parametrize("kind", ["identity", "hadamard", "wus", "wush"])
+def test_ragged_rows_bf16(lib, fmt, kind):
+    # 300 rows: two full 128-row tiles and a ragged tail; the full d_in of the workload
+    w = synth.WORKLOADS[FMT_WORKLOAD[fmt]]
+    x = synth.activations(w, tokens=300)
+    t = _transform(kind, fmt, w)
+    gs = _global_scale(x, t, fmt)
+    c, s, y = run_gpu_t(lib, _as_input(x, True), t, kind, fmt, gs)
+    P.compare_transform_quant(x, t, fmt, gs, c, s, y)
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4", "int4"])
+def test_partial_scale_atom_and_special_values(lib, fmt):
+    # d_in = 3 blocks (a partial 4-column scale atom), 5 rows; zero blocks, tiny and
+    # huge values, negative values that round to -0, exact grid values
+    b = P.Q.BLOCK[fmt]
+    d_in = 3 * b
+    x = synth.small_random(11, (5, d_in)).astype(np.float32)
+    x[0, :b] = 0.0
+    x[1, :b] = -1e-30
+    x[1, 3] = 1.0
+    x[2, b:2 * b] *= 1e4 if fmt == "int4" else 1e20
+    x[3, :] = np.array([0.0, 0.5, 1, 1.5, 2, 3, 4, 6] * (d_in // 8), np.float32)
+    x[4, 2 * b:] = -x[4, 2 * b:] * 1e-12
+    t = T.identity_blocks(d_in, b).astype(np.float32)
+    gs = 1e-3 if fmt == "nvfp4" else 0.0
+    c, s, y = run_gpu_t(lib, _as_input(x, False), t, "identity", fmt, gs)
+    P.compare_transform_quant(x, t, fmt, gs if fmt == "nvfp4" else None, c, s, y)
+    if fmt == "mxfp4":
+        assert s[0, 0] == 0 and np.all(c[0, :b] == 0)
+
+
+def test_dense_path_matches_hadamard_path(lib):
+    # the WUS code path fed H/sqrt(b) must agree with the butterfly path
+    w = synth.WORKLOADS["up_proj"]
+    x = synth.activations(w, tokens=256)
+    t = T.hadamard_blocks(w.d_in, 32).astype(np.float32)
+    c1, s1, y1 = run_gpu_t(lib, _as_input(x, True), t, "wus", "mxfp4", 0.0)
+    P.compare_transform_quant(x, t, "mxfp4", None, c1, s1, y1)
+    c2, s2, y2 = run_gpu_t(lib, _as_input(x, True), t, "hadamard", "mxfp4", 0.0)
+    mag = P.magnitude(x, t)
+    assert np.all(np.abs(y1 - y2) <= 2e-6 * mag)
+
+
+def test_empty_rows_is_noop(lib):
+    x = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
+    codes = torch.zeros(16, dtype=torch.uint8, device="cuda")
+    lib.wush_transform_quant(x, None, "identity", "mxfp4", codes, codes)
+    torch.cuda.synchronize()
+    assert int(codes.sum()) == 0
+
+
+def test_amax_matches_oracle(lib):
+    w = synth.WORKLOADS["down_proj"]
+    x = synth.activations(w, tokens=200)
+    t = _transform("wush", "nvfp4", w)
+    out = torch.empty(1, dtype=torch.float32, device="cuda")
+    lib.wush_transform_amax(_as_input(x, True).cuda(), torch.from_numpy(t).cuda(), "wush", 16, out)
+    want = np.max(np.abs(T.apply_block_transform(x, t)))
+    assert abs(float(out.item()) - want) <= 1e-5 * want
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4", "int4"])
+def test_full_size_sampled_rows(lib, fmt):
+    # the bench's launch configuration (full workload, WUSH), oracle on sampled rows
+    w = synth.WORKLOADS[FMT_WORKLOAD[fmt]]
+    x = synth.activations(w)
+    t = _transform("wush", fmt, w)
+    gs = _global_scale(x[:512], t, fmt) * 1.5
+    c, s, y = run_gpu_t(lib, _as_input(x, True), t, "wush", fmt, gs)
+    rng = np.random.default_rng(5)
+    sel = np.unique(np.concatenate([rng.integers(0, w.tokens, 96), [0, w.tokens - 1]]))
+    P.compare_transform_quant(x, t, fmt, gs if fmt == "nvfp4" else None, c, s, y, rows_sel=sel)
+    # properties over every block: MXFP4 scale rule amax / 2^e in [4, 8)
+    if fmt == "mxfp4":
+        yb = np.abs(y.reshape(w.tokens, -1, 32)).max(axis=2)
+        e = s.astype(np.int64) - 127
+        r = yb / np.ldexp(1.0, e)
+        assert np.all((r >= 4) & (r < 8) | (yb == 0))
