@@ -1,0 +1,446 @@
+"""Benchmark of the W4A4 WUSH linear layer hot path on B200.
+
+One step = the whole hot path on one batch: wush_transform_quant of the
+activations (WUSH block transform + MXFP4 quantisation) followed by wush_qgemm
+(tcgen05 block-scaled FP4 GEMM) into fp32 y.  Weights are transformed and
+quantised once, offline, outside the timed region.
+
+Default workload (up_proj): X bf16 [4096 tokens, 4096] Student-t(3) with 41
+outlier channels x50, W [12288, 4096] N(0, 0.02^2), per-block (b = 32) WUSH
+transforms from 8192 seeded calibration tokens, MXFP4.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {wush,reference}]
+
+N > 1 is launched by torchrun (one process per GPU); every rank runs its own
+batch (weak scaling, no collective on the data path); timing is the max over
+ranks of the device-timed region.  ``--impl reference`` times the CPU oracle on
+the host cores instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+L2_BYTES = 126 * 2 ** 20
+ROTATIONS = 3
+FP4_OVER_BF16 = 4.0          # nominal dense FP4 : BF16 tensor ratio (9 : 2.25 PFLOP/s)
+
+
+# --------------------------------------------------------------------------- helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return dict(hbm_gbs=float(p["hbm_gbs"]), bf16_tflops=float(p["bf16_tflops"]),
+                    bf16_tflops_sustained=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def traffic_from_profiles(kernel: str, workload: str, source_file: str):
+    """DRAM bytes per launch recorded by an ncu capture, if the kernel source is unchanged."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    sha = hashlib.sha1(open(source_file, "rb").read()).hexdigest()[:12]
+    for line in open(path):
+        f = dict(kv.split("=", 1) for kv in line.split() if "=" in kv)
+        if f.get("kernel") == kernel and f.get("workload") == workload and f.get("src_sha") == sha:
+            return float(f["dram_bytes_per_launch"])
+    return None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the GPU is loaded."""
+
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "hw_power_brake_slowdown": 0x80, "sw_power_cap": 0x4}
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.samples, self.reasons = [], set()
+        self.period = period_s
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # no NVML: report no samples
+            self.nv = None
+            self.max_mhz = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                get = getattr(self.nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    self.nv.nvmlDeviceGetCurrentClocksThrottleReasons
+                r = get(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.nv is not None:
+            self._t.join()
+
+    def summary(self):
+        med = statistics.median(self.samples) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+    def rejected(self):
+        bad = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"} & self.reasons
+        stuck = (self.samples and self.max_mhz and statistics.median(self.samples) < 0.6 * self.max_mhz
+                 and not self.reasons)
+        return bool(bad) or bool(stuck)
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("num_threads")]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+# --------------------------------------------------------------------------- workload
+
+WORKLOADS = {
+    "up_proj": dict(fmt="mxfp4", kind="wush"),
+    "down_proj": dict(fmt="nvfp4", kind="wush"),
+}
+
+
+def build_inputs(name: str):
+    w = synth.WORKLOADS[name]
+    x = synth.activations(w)
+    wt = synth.weights(w)
+    xc = synth.activations(w, calib=True)
+    return w, x, wt, xc
+
+
+def describe(w, fmt, kind):
+    return {"workload": (f"{w.name}: X bf16 [{w.tokens} tok, {w.d_in}] {w.x_dist} with {w.n_outlier} outlier "
+                         f"channels x{w.outlier_factor:g}; W bf16 [{w.d_out}, {w.d_in}] N(0,0.02^2); "
+                         f"{kind.upper()} b={w.block} from {w.n_calib} calib tokens; {fmt.upper()} W4A4, y fp32"),
+            "M": w.tokens, "N": w.d_out, "K": w.d_in, "format": fmt, "transform": kind,
+            "l2": f"inputs > L2: y is {w.tokens * w.d_out * 4 / 2**20:.0f} MiB per step; "
+                  f"{ROTATIONS} rotating copies of X and of the weight codes"}
+
+
+# --------------------------------------------------------------------------- CPU oracle leg
+
+class OracleLeg:
+    """The oracle on a sample of token rows of the step (T_X X -> quantise -> fp64 GEMM).
+
+    Calibration and the weights' transform + quantisation are prepared once (offline
+    work, as on the GPU side); ``step(rows)`` is the timed part.
+    """
+
+    def __init__(self, w, x, wt, xc, fmt, kind):
+        from oracle import calibrate as C
+        from oracle import quant as Q
+        from oracle import transforms as T
+        self.w, self.x, self.fmt = w, x, fmt
+        tx, tw = C.calibrate(xc, wt, w.block, kind)
+        self.tx, tw = tx.astype(np.float32), tw.astype(np.float32)
+        self.gx = gw = None
+        if fmt == "nvfp4":
+            self.gx = C.nvfp4_global_scale(T.apply_block_transform(xc, self.tx).astype(np.float32))
+            gw = C.nvfp4_global_scale(T.apply_block_transform(wt, tw).astype(np.float32))
+        self.w_dq = Q.transform_quantize(wt, tw, fmt, gw)["dq"]
+
+    def step(self, rows):
+        from oracle import gemm as G
+        from oracle import quant as Q
+        a = Q.transform_quantize(self.x[:rows], self.tx, self.fmt, self.gx)["dq"]
+        return G.gemm_dequantized(a, self.w_dq)
+
+    def rows_for(self, seconds):
+        t0 = time.perf_counter()
+        self.step(16)
+        dt = time.perf_counter() - t0
+        return int(min(self.w.tokens, max(16, 16 * seconds / max(dt, 1e-3))))
+
+
+def time_oracle(w, x, wt, xc, fmt, kind, target_s=12.0):
+    leg = OracleLeg(w, x, wt, xc, fmt, kind)
+    rows = leg.rows_for(target_s / 3)
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        leg.step(rows)
+        reps += 1
+        if time.perf_counter() - t0 > target_s / 2 or reps >= 8:
+            break
+    dt = (time.perf_counter() - t0) / reps
+    flops = 2.0 * rows * w.d_out * w.d_in
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"{rows} of {w.tokens} token rows through the whole step (transform, quantise, fp64 "
+                      f"GEMM against the offline-quantised {w.d_out}x{w.d_in} weights), {reps} reps, "
+                      f"{dt:.2f} s each"}
+
+
+# --------------------------------------------------------------------------- GPU leg
+
+def run_gpu(args, rank, world):
+    import torch
+    import activation_quantization_b200 as aq
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    spec = WORKLOADS[args.workload]
+    fmt, kind = spec["fmt"], spec["kind"]
+    w, x, wt, xc = build_inputs(args.workload)
+    M, N, K = w.tokens, w.d_out, w.d_in
+    b = w.block
+
+    # offline: calibration (host C++), weight transform + quantisation (GPU), NVFP4 scales
+    tx, tw = aq.wush_calibrate(xc, wt, b, kind)
+    t_x, t_w = torch.from_numpy(tx).to(dev), torch.from_numpy(tw).to(dev)
+    gx = gw = 0.0
+    if fmt == "nvfp4":
+        amax = torch.empty(1, dtype=torch.float32, device=dev)
+        aq.wush_transform_amax(torch.from_numpy(xc).to(torch.bfloat16).to(dev), t_x, kind, b, amax)
+        gx = float(np.float32(amax.item() / (6 * 448)))
+        wt_dev = torch.from_numpy(wt).to(torch.bfloat16).to(dev)
+        aq.wush_transform_amax(wt_dev, t_w, kind, b, amax)
+        gw = float(np.float32(amax.item() / (6 * 448)))
+    alpha = float(np.float32(gx) * np.float32(gw)) if fmt == "nvfp4" else 1.0
+    xs = [torch.from_numpy(x).to(torch.bfloat16).to(dev) for _ in range(ROTATIONS)]
+    wcodes = []
+    for _ in range(ROTATIONS):
+        bc, bs = aq.alloc_quant_outputs(N, K, fmt, dev)
+        aq.wush_transform_quant(torch.from_numpy(wt).to(torch.bfloat16).to(dev), t_w, kind, fmt, bc, bs, gw)
+        wcodes.append((bc, bs))
+    acodes = [aq.alloc_quant_outputs(M, K, fmt, dev) for _ in range(ROTATIONS)]
+    y = torch.empty((M, N), dtype=torch.float32, device=dev)
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.Stream(device=dev)
+
+    def tq(r):
+        aq.wush_transform_quant(xs[r], t_x, kind, fmt, acodes[r][0], acodes[r][1], gx, stream=stream)
+
+    def gemm(r):
+        aq.wush_qgemm(acodes[r][0], acodes[r][1], wcodes[r][0], wcodes[r][1], M, N, K, fmt, alpha, y,
+                      stream=stream)
+
+    # capture each kernel of each rotation as its own CUDA graph
+    with torch.cuda.stream(stream):
+        for r in range(ROTATIONS):
+            tq(r)
+            gemm(r)
+    stream.synchronize()
+    graphs_tq, graphs_gemm = [], []
+    for r in range(ROTATIONS):
+        g1, g2 = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g1, stream=stream):
+            tq(r)
+        with torch.cuda.graph(g2, stream=stream):
+            gemm(r)
+        graphs_tq.append(g1)
+        graphs_gemm.append(g2)
+    if aq.wush_check_device_status(stream) != 0:
+        raise RuntimeError("device status after capture")
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def timed(steps):
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        barrier()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            for i in range(steps):
+                r = i % ROTATIONS
+                ev[i][0].record(stream)
+                graphs_tq[r].replay()
+                ev[i][1].record(stream)
+                graphs_gemm[r].replay()
+                ev[i][2].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        total_ms = ev[0][0].elapsed_time(ev[-1][2])
+        tq_ms = [e[0].elapsed_time(e[1]) for e in ev]
+        gm_ms = [e[1].elapsed_time(e[2]) for e in ev]
+        return total_ms, tq_ms, gm_ms
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            graphs_tq[i % ROTATIONS].replay()
+            graphs_gemm[i % ROTATIONS].replay()
+    stream.synchronize()
+
+    for attempt in range(2):
+        sampler = ClockSampler(dev.index)
+        with sampler:
+            total_ms, tq_ms, gm_ms = timed(args.steps)
+        if not sampler.rejected():
+            break
+    status = aq.wush_check_device_status(stream)
+    if status != 0:
+        raise RuntimeError(f"device status {status}")
+
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    flops_step = 2.0 * M * N * K
+    value = flops_step * args.steps * world / (total_ms * 1e-3) / 1e12
+    tq_us = 1e3 * float(np.mean(tq_ms))
+    gm_us = 1e3 * float(np.mean(gm_ms))
+    peaks = load_peaks()
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    tq_bytes = (M * K * 2 + aq.wush_codes_bytes(M, K, fmt) + aq.wush_scales_bytes(M, K, fmt)
+                + (K // b) * b * b * 4)
+    gemm_tflops = flops_step / (gm_us * 1e-6) / 1e12
+    tq_gbs = tq_bytes / (tq_us * 1e-6) / 1e9
+    qgemm_src = os.path.join(ROOT, "activation_quantization_b200", "csrc", "qgemm.cu")
+    tq_src = os.path.join(ROOT, "activation_quantization_b200", "csrc", "transform_quant.cu")
+
+    # end to end through the public API: pinned host X -> device, step, y -> pinned host
+    if True:
+        x_host = torch.from_numpy(x).to(torch.bfloat16).pin_memory()
+        y_host = torch.empty((M, N), dtype=torch.float32).pin_memory()
+        e_steps = max(3, min(args.steps, 10))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            for i in range(e_steps + 1):
+                if i == 1:
+                    e0.record(stream)
+                xs[0].copy_(x_host, non_blocking=True)
+                tq(0)
+                gemm(0)
+                y_host.copy_(y, non_blocking=True)
+            e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = e0.elapsed_time(e1) / e_steps
+        if world > 1:
+            import torch.distributed as dist
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": flops_step * world / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int(x_host.numel() * 2), "d2h_bytes_per_step": int(y_host.numel() * 4),
+               "ms_per_step": e_ms}
+
+    result = None
+    if rank == 0:
+        traffic = traffic_from_profiles("qgemm_kernel", args.workload, qgemm_src)
+        tq_traffic = traffic_from_profiles("transform_quant_kernel", args.workload, tq_src)
+        result = {
+            "metric": "transform+quant HBM GB/s; W4A4 block-scaled GEMM TFLOP/s (% of peak)",
+            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "e2m1 x e2m1 -> fp32 (transform in fp32)", "data": "synthetic",
+            "config": describe(w, fmt, kind),
+            "transform_quant": {"us": tq_us, "GB_s": tq_gbs, "bytes_per_launch": tq_bytes,
+                                "frac_of_hbm": tq_gbs / peaks["hbm_gbs"], "dram_bytes_per_launch": tq_traffic},
+            "qgemm": {"us": gm_us, "TFLOP_s": gemm_tflops, "frac_of_fp4_peak": gemm_tflops / fp4_peak},
+            "roofline": {"kernel": "qgemm_kernel", "bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak,
+                         "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak, "traffic": traffic,
+                         "peak_source": (f"{peaks['source']} bf16 burst {peaks['bf16_tflops']:.1f} TFLOP/s x "
+                                         f"{FP4_OVER_BF16:g} (nominal dense FP4:BF16)")},
+            "e2e": e2e, "gpu_launches": 2 * args.steps,
+            "clocks": sampler.summary(),
+        }
+    return result, (w, x, wt, xc, fmt, kind)
+
+
+# --------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="wush", choices=["wush", "reference"])
+    ap.add_argument("--workload", default="up_proj", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    spec = WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        w, x, wt, xc = build_inputs(args.workload)
+        leg = OracleLeg(w, x, wt, xc, spec["fmt"], spec["kind"])
+        step_rows = leg.rows_for(1.5)
+        times = []
+        for i in range(args.warmup + args.steps):
+            t0 = time.perf_counter()
+            leg.step(step_rows)
+            if i >= args.warmup:
+                times.append(time.perf_counter() - t0)
+        dt = sum(times) / len(times)
+        val = 2.0 * step_rows * w.d_out * w.d_in / dt / 1e12
+        cb = {"value": val, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+              "sample": f"{step_rows} of {w.tokens} token rows per step through the whole step"}
+        print(json.dumps({"impl": "reference", "metric": "transform+quant HBM GB/s; W4A4 block-scaled GEMM "
+                          "TFLOP/s (% of peak)", "value": val, "unit": "TFLOP/s", "n_gpus": world,
+                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+                          "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                          "data": "synthetic", "config": describe(w, spec["fmt"], spec["kind"]),
+                          "cpu_baseline": cb,
+                          "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                                  "d2h_bytes_per_step": 0}}))
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    result, ctx = run_gpu(args, rank, world)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            w, x, wt, xc, fmt, kind = ctx
+            result["cpu_baseline"] = time_oracle(w, x, wt, xc, fmt, kind)
+        print(json.dumps(result))
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
