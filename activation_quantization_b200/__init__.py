@@ -39,6 +39,7 @@ _SIGNATURES = {
     "wush_qgemm": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _f32, _vp, _vp]),
     "itq3_quantize_weights": (_i32, [_vp, _i64, _i64, _vp, _vp]),
     "itq3_dequant_gemv": (_i32, [_vp, _vp, _vp, _i64, _i64, _i64, _i32, _vp, _vp, _vp]),
+    "itq3_dequant_gemv_noalloc": (_i32, [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp]),
     "wush_check_device_status": (_i32, [_vp]),
     "wush_debug_set_wait_limit": (_i32, [_i64]),
 }
@@ -187,6 +188,14 @@ def itq3_dequant_gemv(codes, scales, x, d_out: int, mode: int, y, workspace=None
     _check("itq3_dequant_gemv",
            _lib.itq3_dequant_gemv(_ptr(codes), _ptr(scales), _ptr(x), tokens, d_out, d_in, int(mode),
                                   _ptr(workspace), _ptr(y), _stream(stream)))
+
+
+def itq3_dequant_gemv_noalloc(codes, scales, x, d_out: int, y, stream=None):
+    """Mode-1 ITQ3 GEMV with the library's fixed scratch instead of a workspace."""
+    tokens, d_in = x.shape
+    _check("itq3_dequant_gemv_noalloc",
+           _lib.itq3_dequant_gemv_noalloc(_ptr(codes), _ptr(scales), _ptr(x), tokens, d_out, d_in, _ptr(y),
+                                          _stream(stream)))
 
 
 def wush_check_device_status(stream=None) -> int:

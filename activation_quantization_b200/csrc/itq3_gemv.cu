@@ -18,6 +18,8 @@
 //   workspace; the GEMV then uses the levels (c - 3.5) s with no transform.
 #include <cuda_fp16.h>
 
+#include <mutex>
+
 #include "common.cuh"
 
 namespace wush {
@@ -182,5 +184,75 @@ extern "C" int itq3_dequant_gemv(const uint8_t* codes, const void* scales_fp16, 
   if (t == 1) itq3_rotated_kernel<1><<<grid, block, 0, st>>>(c32, sc, workspace, t, n, k, y);
   else if (t <= 4) itq3_rotated_kernel<4><<<grid, block, 0, st>>>(c32, sc, workspace, t, n, k, y);
   else itq3_rotated_kernel<16><<<grid, block, 0, st>>>(c32, sc, workspace, t, n, k, y);
+  return launch_status();
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of mode 1.
+//
+// Some callers cannot call cudaMalloc at the point where they run this GEMV: an
+// inference engine that carves all device memory out of its own pool at start-up
+// and forbids further allocations, a real-time loop that cannot afford the
+// latency or the possible failure of an allocation, or a plugin whose host owns
+// the device memory.  For them the rotated activations live in one fixed array
+// inside this library instead of a caller-provided workspace.
+namespace wush {
+namespace {
+
+// Capacity of the fixed scratch: tokens * d_in fp32 values (1 MiB).  Every device
+// that loads the library holds this array until the process exits.
+constexpr int64_t kNoAllocScratchFloats = int64_t(1) << 18;
+
+}  // namespace
+
+static __device__ __align__(256) float g_itq3_noalloc_scratch[kNoAllocScratchFloats];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+float* g_scratch_addr[kMaxDevices] = {};
+std::mutex g_scratch_mutex;
+
+// Device address of the scratch array on the current device, looked up once per
+// device.  (In host code the array's name is only a host-side stand-in, so the
+// kernels must be handed this address, never the name.)
+int scratch_for_current_device(float** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return WUSH_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_itq3_noalloc_scratch) != cudaSuccess || !p) return WUSH_ERR_CUDA;
+    g_scratch_addr[dev] = static_cast<float*>(p);
+  }
+  *out = g_scratch_addr[dev];
+  return WUSH_OK;
+}
+
+}  // namespace
+}  // namespace wush
+
+extern "C" int itq3_dequant_gemv_noalloc(const uint8_t* codes, const void* scales_fp16, const void* x_fp16,
+                                         int64_t tokens, int64_t d_out, int64_t d_in, float* y, void* stream) {
+  if (tokens < 1 || tokens > 16 || d_out <= 0 || d_in <= 0 || d_in % 256 || d_out % 8) return WUSH_ERR_INVALID_ARG;
+  if (tokens * d_in > kNoAllocScratchFloats) return WUSH_ERR_BUFFER_TOO_SMALL;
+  if (d_out > (int64_t(1) << 30)) return WUSH_ERR_UNSUPPORTED;
+  if (!codes || !scales_fp16 || !x_fp16 || !y || !aligned16(codes)) return WUSH_ERR_INVALID_ARG;
+  float* scratch = nullptr;
+  const int st = scratch_for_current_device(&scratch);
+  if (st != WUSH_OK) return st;
+  // The rotation kernel writes every scratch element the GEMV then reads, so
+  // nothing left there by an earlier call needs clearing.
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const auto* c32 = reinterpret_cast<const uint32_t*>(codes);
+  const auto* sc = static_cast<const __half*>(scales_fp16);
+  const auto* xh = static_cast<const __half*>(x_fp16);
+  const int t = static_cast<int>(tokens), n = static_cast<int>(d_out), k = static_cast<int>(d_in);
+  const dim3 grid(static_cast<unsigned>((d_out + kWarps - 1) / kWarps)), block(kWarps * 32);
+  const int items = t * (k / 256);
+  itq3_rotate_x_kernel<<<(items + kWarps - 1) / kWarps, block, 0, s>>>(xh, t, k, scratch);
+  if (t == 1) itq3_rotated_kernel<1><<<grid, block, 0, s>>>(c32, sc, scratch, t, n, k, y);
+  else if (t <= 4) itq3_rotated_kernel<4><<<grid, block, 0, s>>>(c32, sc, scratch, t, n, k, y);
+  else itq3_rotated_kernel<16><<<grid, block, 0, s>>>(c32, sc, scratch, t, n, k, y);
   return launch_status();
 }

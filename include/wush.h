@@ -216,6 +216,24 @@ int itq3_dequant_gemv(const uint8_t* codes, const void* scales_fp16, const void*
                       int64_t tokens, int64_t d_out, int64_t d_in, int mode, float* workspace,
                       float* y, void* stream);
 
+/* Allocation-free form of itq3_dequant_gemv mode 1.  The pages have no
+ * counterpart: it exists for callers that cannot call cudaMalloc where they run
+ * the GEMV (an engine that reserves all device memory in its own pool at start-up
+ * and allows no later allocation, a real-time loop that cannot take an
+ * allocation's latency or failure, a plugin whose host owns device memory).
+ * Instead of a caller workspace, the rotated activations go to one fixed array
+ * inside the library, 262,144 fp32 values (1 MiB) per device, held by every GPU
+ * that loads the library until the process exits.
+ * Arguments as in itq3_dequant_gemv; tokens * d_in must be <= 262,144, else
+ * WUSH_ERR_BUFFER_TOO_SMALL and nothing is launched.  Calls no allocating
+ * routine.  The first call on a device looks up the array's device address (with
+ * that device current); make that first call before any stream capture.  All
+ * calls on a device share the array: calls whose kernels overlap on the GPU
+ * (different streams, no ordering between them) race on it.  Nothing needs to
+ * start at zero: every call overwrites the part of the array it reads. */
+int itq3_dequant_gemv_noalloc(const uint8_t* codes, const void* scales_fp16, const void* x_fp16,
+                              int64_t tokens, int64_t d_out, int64_t d_in, float* y, void* stream);
+
 /* ---------------------------------------------------------------------------
  * Diagnostics
  * ------------------------------------------------------------------------- */
