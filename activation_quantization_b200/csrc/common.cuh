@@ -16,6 +16,14 @@ enum : int { kErrTimeoutBarrier = 1, kErrTimeoutTmem = 2 };
 // it; returns a cudaError_t as int.
 int read_and_clear_error_word(int* word);
 
+// The same for the tensor-core transform+quant kernel's error word.
+int read_and_clear_tq_error(int* word);
+
+// Tensor-core form of wush_transform_quant (bf16 inputs); WUSH_ERR_UNSUPPORTED
+// for shapes it does not take.
+int transform_quant_tc(const void* x, int64_t rows, int64_t d_in, const float* t, int kind, int fmt,
+                       float gscale, uint8_t* codes, void* scales, float* ydbg, cudaStream_t st);
+
 // Poll limit for bounded mbarrier waits (0 = the built-in default).
 extern int64_t g_wait_limit_override;
 

@@ -186,16 +186,19 @@ __global__ void __launch_bounds__(kRowsPerCta) transform_quant_kernel(
         const float den = 6.0f * gscale;
         const uint32_t sb = ue4m3_rne(__fdiv_rn(amax, den));
         const float d = __fmul_rn(ue4m3_value(sb), gscale);
+        const bool live = sb != 0u && amax > 0.f;
+        const float rd = live ? __fdiv_rn(1.0f, d) : 0.f;
 #pragma unroll
-        for (int i = 0; i < B; ++i) c[i] = (sb != 0u && amax > 0.f) ? e2m1_rne(__fdiv_rn(y[i], d)) : 0u;
+        for (int i = 0; i < B; ++i) c[i] = live ? e2m1_rne(y[i] * rd) : 0u;
         s_sf[(tid & 31) * 16 + (tid >> 5) * 4 + jj] = static_cast<uint8_t>(sb);
       } else {  // INT4
         const float pre = fminf(__fdiv_rn(amax, 7.0f), 65504.0f);
         const __half s16 = __float2half_rn(pre);
         const float s = __half2float(s16);
+        const float rs = s > 0.f ? __fdiv_rn(1.0f, s) : 0.f;
 #pragma unroll
         for (int i = 0; i < B; ++i) {
-          float q = s > 0.f ? rintf(__fdiv_rn(y[i], s)) : 0.f;
+          float q = s > 0.f ? rintf(y[i] * rs) : 0.f;
           q = fminf(fmaxf(q, -7.0f), 7.0f);
           c[i] = static_cast<uint32_t>(static_cast<int>(q)) & 0xFu;
         }
@@ -312,9 +315,13 @@ extern "C" int wush_transform_quant(const void* x, int x_dtype, int64_t rows, in
   if (rows == 0) return WUSH_OK;
   if (!codes || !scales || !aligned16(codes) || !aligned16(scales)) return WUSH_ERR_INVALID_ARG;
   if (y_debug && !aligned16(y_debug)) return WUSH_ERR_INVALID_ARG;
-  if (fmt == WUSH_FMT_NVFP4 && !(global_scale > 0.0f && global_scale < 3.0e38f)) return WUSH_ERR_INVALID_ARG;
+  if (fmt == WUSH_FMT_NVFP4 && !(global_scale >= 1e-30f && global_scale < 1e30f)) return WUSH_ERR_INVALID_ARG;
   const bool xf32 = x_dtype == WUSH_IN_FP32;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!xf32) {
+    const int tc = transform_quant_tc(x, rows, d_in, t, kind, fmt, global_scale, codes, scales, y_debug, s);
+    if (tc != WUSH_ERR_UNSUPPORTED) return tc;
+  }
   if (fmt == WUSH_FMT_MXFP4)
     return launch_fmt<32, kMx>(x, xf32, rows, d_in, t, kind, 0.f, codes, scales, y_debug, nullptr, s);
   if (fmt == WUSH_FMT_NVFP4)

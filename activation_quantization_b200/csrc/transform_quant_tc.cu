@@ -1,0 +1,566 @@
+// Fused per-block transform + microscaled quantisation on tcgen05 tensor cores
+// (bf16 activations).
+//
+// WUSH news article, paragraph 6 (only the activations are transformed at
+// inference; blocks are independent) and AI Radio episode, "The gist" (a fused
+// GPU implementation).  The format rules are stated in wush.h.
+//
+// A persistent CTA walks a contiguous range of 128-row x 128-column tiles of X in
+// column-major order, with three roles:
+//   warp 0     TMA producer: each tile is two 128-byte-swizzled boxes of 64 bf16
+//              columns, landing in a 4-stage shared-memory ring;
+//   warp 1     MMA issuer (WUS/WUSH): for every b-block of the tile, y = x T^T
+//              as kind::f16 MMAs, M = 128 rows, N = b, K = 16 per instruction,
+//              with T split exactly into three bf16 parts (hi + mid + lo = the
+//              fp32 T) and the three products accumulated in fp32 in TMEM; two
+//              accumulators (one per epilogue warpgroup) let the MMAs of later tiles
+//              overlap the epilogues of earlier ones;
+//   warps 2-17 epilogue, four warpgroups each owning every fourth tile: one thread per row reads its b transformed values
+//              straight out of TMEM (tcgen05.ld 32x32b) -- or, for identity and
+//              Hadamard, out of the swizzled shared-memory tile -- and computes
+//              absmax, scale and codes in registers (hardware cvt.rn.satfinite
+//              e2m1x2), storing packed codes and scale words.  The same warps
+//              convert each new column's fp32 T into the bf16 split operand
+//              layout in shared memory, double-buffered.
+// Every mbarrier wait is bounded (see sm100.cuh).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace wush {
+namespace {
+
+using namespace sm100;
+
+constexpr int kTileRows = 128;
+constexpr int kTileCols = 128;                       // bf16 elements
+constexpr int kBoxCols = 64;                         // 128 bytes
+constexpr int kStages = 4;
+constexpr int kEpiWarps = 16;
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kEpiGroups = 4;                        // epilogue warpgroups, one tile each
+constexpr int kAccs = 4;                             // TMEM accumulators (128 columns each)
+constexpr int kThreads = 64 + kEpiThreads;
+constexpr int kStageBytes = kTileRows * kTileCols * 2;  // 32 KB
+constexpr int kBoxBytes = kTileRows * kBoxCols * 2;     // 16 KB
+constexpr int kTBufBytes = 24 * 1024;
+constexpr uint32_t kTmemCols = 512;
+constexpr int64_t kDefaultPolls = int64_t(1) << 40;
+constexpr uint64_t kDeadlineNs = 4000000000ull;
+constexpr int kSmemBytes = kStages * kStageBytes + 2 * kTBufBytes + 1024 + 256;
+
+enum Kind : int { kIdentity = 0, kHadamard = 1, kDense = 2 };
+enum Fmt : int { kMx = 0, kNv = 1, kI4 = 2 };
+
+__device__ int g_tq_error = 0;
+
+__device__ __forceinline__ float exp2i(int k) {
+  return k >= -126 ? __uint_as_float(static_cast<uint32_t>(k + 127) << 23) : __uint_as_float(1u << (k + 149));
+}
+
+__device__ __forceinline__ int floor_log2(float a) {
+  const uint32_t b = __float_as_uint(a);
+  const int e = (b >> 23) & 0xFF;
+  return e ? e - 127 : (31 - __clz(b & 0x7FFFFFu)) - 149;
+}
+
+__device__ __forceinline__ uint32_t ue4m3_rne(float t) {
+  if (!(t < 448.0f)) return 126u;
+  if (t == 0.0f) return 0u;
+  int e = floor_log2(t);
+  if (e < -6) return static_cast<uint32_t>(rintf(t * 512.0f));
+  float q = rintf(t * exp2i(3 - e));
+  if (q >= 16.0f) { q = 8.0f; ++e; }
+  return (static_cast<uint32_t>(e + 7) << 3) | (static_cast<uint32_t>(q) - 8u);
+}
+
+__device__ __forceinline__ float ue4m3_value(uint32_t c) {
+  const uint32_t e = c >> 3, m = c & 7u;
+  return e == 0 ? static_cast<float>(m) * 0.001953125f : static_cast<float>(8u + m) * exp2i(static_cast<int>(e) - 10);
+}
+
+// Eight values -> eight E2M1 codes, element 0 in the low nibble (RNE, satfinite).
+__device__ __forceinline__ uint32_t e2m1x8(float v0, float v1, float v2, float v3, float v4, float v5, float v6,
+                                           float v7) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(out)
+      : "f"(v0), "f"(v1), "f"(v2), "f"(v3), "f"(v4), "f"(v5), "f"(v6), "f"(v7));
+  return out;
+}
+
+__device__ __forceinline__ uint32_t int4_nibble(float v) {
+  int q = __float2int_rn(v);
+  q = q < -7 ? -7 : (q > 7 ? 7 : q);
+  return static_cast<uint32_t>(q) & 0xFu;
+}
+
+// Quantise one block of B fp32 values held by this thread.  Writes B/8 code
+// words and returns the scale (byte for MXFP4/NVFP4, fp16 bits for INT4).
+template <int B, int FMT>
+__device__ __forceinline__ uint32_t quantize_block(const float (&y)[B], float gscale, float den, uint32_t (&w)[B / 8]) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < B; ++i) amax = fmaxf(amax, fabsf(y[i]));
+  if constexpr (FMT == kMx) {
+    int e = amax > 0.f ? floor_log2(amax) - 2 : -127;
+    e = e < -127 ? -127 : (e > 127 ? 127 : e);
+    const float inv = exp2i(-e);
+#pragma unroll
+    for (int q = 0; q < B / 8; ++q)
+      w[q] = amax > 0.f ? e2m1x8(y[8 * q] * inv, y[8 * q + 1] * inv, y[8 * q + 2] * inv, y[8 * q + 3] * inv,
+                                 y[8 * q + 4] * inv, y[8 * q + 5] * inv, y[8 * q + 6] * inv, y[8 * q + 7] * inv)
+                        : 0u;
+    return static_cast<uint32_t>(e + 127);
+  } else if constexpr (FMT == kNv) {
+    const uint32_t sb = ue4m3_rne(__fdiv_rn(amax, den));
+    const float d = __fmul_rn(ue4m3_value(sb), gscale);
+    const bool live = sb != 0u && amax > 0.f;
+    const float r = live ? __fdiv_rn(1.0f, d) : 0.f;
+#pragma unroll
+    for (int q = 0; q < B / 8; ++q)
+      w[q] = live ? e2m1x8(y[8 * q] * r, y[8 * q + 1] * r, y[8 * q + 2] * r, y[8 * q + 3] * r, y[8 * q + 4] * r,
+                           y[8 * q + 5] * r, y[8 * q + 6] * r, y[8 * q + 7] * r)
+                  : 0u;
+    return sb;
+  } else {
+    const float pre = fminf(__fdiv_rn(amax, 7.0f), 65504.0f);
+    const __half s16 = __float2half_rn(pre);
+    const float s = __half2float(s16);
+    const float r = s > 0.f ? __fdiv_rn(1.0f, s) : 0.f;
+#pragma unroll
+    for (int q = 0; q < B / 8; ++q) {
+      uint32_t acc = 0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) acc |= int4_nibble(y[8 * q + k] * r) << (4 * k);
+      w[q] = s > 0.f ? acc : 0u;
+    }
+    return static_cast<uint32_t>(__half_as_ushort(s16));
+  }
+}
+
+template <int B>
+__device__ __forceinline__ void fwht_normalized(float (&y)[B]) {
+#pragma unroll
+  for (int h = 1; h < B; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < B; i += 2 * h) {
+#pragma unroll
+      for (int k = i; k < i + h; ++k) {
+        const float a = y[k], b = y[k + h];
+        y[k] = a + b;
+        y[k + h] = a - b;
+      }
+    }
+  }
+  const float s = B == 32 ? 0.17677669529663688f : 0.25f;
+#pragma unroll
+  for (int i = 0; i < B; ++i) y[i] *= s;
+}
+
+template <int B>
+__device__ __forceinline__ void tmem_ld_block(uint32_t taddr, float (&y)[B]) {
+  uint32_t r[B];
+  if constexpr (B == 32) tmem_ld_32x32b_x32(taddr, r);
+  else tmem_ld_32x32b_x16(taddr, r);
+  tmem_ld_wait();
+#pragma unroll
+  for (int i = 0; i < B; ++i) y[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ uint32_t bf16_bits_rn(float v) {
+  return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(v)));
+}
+
+// Instruction descriptor, kind::f16: bf16 A and B (K-major), fp32 D, M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t m, uint32_t n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((n >> 3) << 17) | ((m >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+template <int B, int FMT, int KIND, bool DBG>
+__global__ void __launch_bounds__(kThreads, 1)
+    tq_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* __restrict__ t, float gscale,
+                 uint8_t* __restrict__ codes, void* __restrict__ scales, float* __restrict__ ydbg, int rows,
+                 int d_in, int n_row_tiles, int n_tiles, int64_t max_polls) {
+  constexpr int kBlocks = kTileCols / B;           // b-blocks per tile: 4 or 8
+  constexpr int kKSteps = B / 16;                  // K = 16 per MMA
+  constexpr int kChunk = B * 32;                   // bytes of one [B n x 16 k] bf16 operand chunk
+  constexpr bool kMma = KIND == kDense;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* tbuf = smem + kStages * kStageBytes;
+  uint64_t* x_full = reinterpret_cast<uint64_t*>(tbuf + 2 * kTBufBytes);
+  uint64_t* x_empty = x_full + kStages;
+  uint64_t* acc_full = x_empty + kStages;
+  uint64_t* acc_empty = acc_full + kAccs;
+  uint64_t* t_full = acc_empty + kAccs;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(t_full + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int nb = d_in / B;
+  const int tile_lo = static_cast<int>(static_cast<int64_t>(blockIdx.x) * n_tiles / gridDim.x);
+  const int tile_hi = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * n_tiles / gridDim.x);
+  const int col_lo = tile_lo / n_row_tiles;
+  const uint64_t deadline = globaltimer_ns() + kDeadlineNs;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&x_full[s], 1);
+      mbar_init(&x_empty[s], kMma ? 1 : 128);
+    }
+    for (int a = 0; a < kAccs; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 128);
+    }
+    for (int b = 0; b < 2; ++b) mbar_init(&t_full[b], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tmap_x);
+  }
+  if (warp == 1 && kMma) tmem_alloc(tmem_slot, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = kMma ? *tmem_slot : 0u;
+
+  auto give_up = [&]() {
+    if (!*abort_flag) {
+      *abort_flag = 1;
+      atomicOr(&g_tq_error, 1 << kErrTimeoutBarrier);
+    }
+  };
+
+  if (warp == 0) {
+    if (elect_one()) {
+      for (int i = tile_lo; i < tile_hi; ++i) {
+        const int n = i - tile_lo, s = n % kStages;
+        if (!mbar_wait_bounded(&x_empty[s], ((n / kStages) & 1) ^ 1, max_polls, deadline, abort_flag)) {
+          give_up();
+          break;
+        }
+        const int row0 = (i % n_row_tiles) * kTileRows, col0 = (i / n_row_tiles) * kTileCols;
+        uint8_t* st = smem + s * kStageBytes;
+        mbar_arrive_expect_tx(&x_full[s], kStageBytes);
+        tma_load_2d(st, &tmap_x, col0, row0, &x_full[s]);
+        tma_load_2d(st + kBoxBytes, &tmap_x, col0 + kBoxCols, row0, &x_full[s]);
+      }
+    }
+  } else if (warp == 1) {
+    if (kMma && elect_one()) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kTileRows, B);
+      for (int i = tile_lo; i < tile_hi; ++i) {
+        const int n = i - tile_lo, s = n % kStages, a = n % kAccs;
+        const int k = i / n_row_tiles - col_lo;     // column ordinal within this CTA
+        if (!mbar_wait_bounded(&t_full[k & 1], (k >> 1) & 1, max_polls, deadline, abort_flag) ||
+            !mbar_wait_bounded(&acc_empty[a], ((n / kAccs) & 1) ^ 1, max_polls, deadline, abort_flag) ||
+            !mbar_wait_bounded(&x_full[s], (n / kStages) & 1, max_polls, deadline, abort_flag)) {
+          give_up();
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sx = smem_u32(smem + s * kStageBytes);
+        const uint32_t st_ = smem_u32(tbuf + (k & 1) * kTBufBytes);
+        const uint32_t d0 = tmem + a * kTileCols;
+#pragma unroll
+        for (int jj = 0; jj < kBlocks; ++jj) {
+          const int col_bytes = jj * B * 2;                      // byte column of the block in the tile
+          const uint32_t abase = sx + (col_bytes / 128) * kBoxBytes + (col_bytes % 128);
+#pragma unroll
+          for (int sp = 0; sp < 3; ++sp) {
+#pragma unroll
+            for (int kk = 0; kk < kKSteps; ++kk) {
+              const uint64_t ad = desc_kmajor_sw128(abase + kk * 32);
+              const uint64_t bd = smem_desc(st_ + ((jj * 3 + sp) * kKSteps + kk) * kChunk, 128, 256, kLayoutNone);
+              mma_bf16(d0 + jj * B, ad, bd, idesc, (sp | kk) ? 1u : 0u);
+            }
+          }
+        }
+        tc_commit(&x_empty[s]);
+        tc_commit(&acc_full[a]);
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    // Four warpgroups of 4 warps.  Warpgroup g takes tiles n = g, g+4, ... of the
+    // CTA's range, so four tiles are in flight at once; inside a warpgroup, warp w
+    // may read only TMEM lane quarter w % 4, i.e. rows 32*(w % 4) .. +31, and each
+    // thread handles all b-blocks of one row of the tile.
+    const int et = threadIdx.x - 64;            // 0..511
+    const int g = et / 128;                     // warpgroup
+    const int q = warp & 3;
+    const int rloc = q * 32 + lane;             // row within the tile
+    const float den = 6.0f * gscale;
+    const int n_cols = tile_hi > tile_lo ? (tile_hi - 1) / n_row_tiles - col_lo + 1 : 0;
+
+    // fp32 T of column col_lo + k -> the three bf16 split operands in buffer k & 1,
+    // by nthr threads (id tid); all float4 loads of a thread are issued first.
+    auto convert_t = [&](int k, int tid, int nthr, int bar_id) {
+      constexpr int kGroups = kBlocks * B * B / 4;
+      uint8_t* dst = tbuf + (k & 1) * kTBufBytes;
+      const int j0 = (col_lo + k) * kBlocks;
+      for (int base = 0; base < kGroups; base += 8 * nthr) {
+        float4 v[8];
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+          const int gi = base + tid + p * nthr;
+          const int e0 = 4 * gi;
+          v[p] = (gi < kGroups && j0 + e0 / (B * B) < nb)
+                     ? __ldg(reinterpret_cast<const float4*>(t + static_cast<int64_t>(j0) * B * B + e0))
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+          const int gi = base + tid + p * nthr;
+          if (gi >= kGroups) continue;
+          const int e0 = 4 * gi;
+          const int jj = e0 / (B * B), nrow = (e0 / B) % B, kcol = e0 % B;
+          const int kk = kcol / 16, kin = kcol % 16;
+          const int off = (nrow / 8) * 256 + (kin / 8) * 128 + (nrow % 8) * 16 + (kin % 8) * 2;
+          const float x4[4] = {v[p].x, v[p].y, v[p].z, v[p].w};
+          uint32_t h[3][4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            h[0][c] = bf16_bits_rn(x4[c]);
+            const float r1 = x4[c] - __uint_as_float(h[0][c] << 16);
+            h[1][c] = bf16_bits_rn(r1);
+            const float r2 = r1 - __uint_as_float(h[1][c] << 16);
+            h[2][c] = bf16_bits_rn(r2);
+          }
+#pragma unroll
+          for (int sp = 0; sp < 3; ++sp)
+            *reinterpret_cast<uint2*>(dst + ((jj * 3 + sp) * kKSteps + kk) * kChunk + off) =
+                make_uint2(h[sp][0] | (h[sp][1] << 16), h[sp][2] | (h[sp][3] << 16));
+        }
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(nthr) : "memory");
+      if (tid == 0) mbar_arrive(&t_full[k & 1]);
+    };
+    if constexpr (kMma) {
+      if (n_cols > 0) convert_t(0, et, kEpiThreads, 1);
+      if (n_cols > 1) convert_t(1, et, kEpiThreads, 1);
+    }
+
+    for (int i = tile_lo + g; i < tile_hi; i += kEpiGroups) {
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+      const int n = i - tile_lo, s = n % kStages, a = n % kAccs;
+      const int row0 = (i % n_row_tiles) * kTileRows, col0 = (i / n_row_tiles) * kTileCols;
+      const int r = row0 + rloc;
+      const bool row_ok = r < rows;
+      bool ok;
+      if constexpr (kMma) ok = mbar_wait_bounded(&acc_full[a], (n / kAccs) & 1, max_polls, deadline, abort_flag);
+      else ok = mbar_wait_bounded(&x_full[s], (n / kStages) & 1, max_polls, deadline, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) { give_up(); break; }
+      if constexpr (kMma) tc_fence_after();
+      const uint8_t* sx = smem + s * kStageBytes;
+      uint32_t sc_words[kBlocks / 4];
+#pragma unroll
+      for (int w4 = 0; w4 < kBlocks / 4; ++w4) sc_words[w4] = 0u;
+#pragma unroll
+      for (int jj = 0; jj < kBlocks; ++jj) {
+        float y[B];
+        if constexpr (kMma) {
+          tmem_ld_block<B>(tmem + (static_cast<uint32_t>(q * 32) << 16) + a * kTileCols + jj * B, y);
+        } else {
+          const int col_bytes = jj * B * 2;
+          const uint8_t* rowp = sx + (col_bytes / 128) * kBoxBytes + rloc * 128;
+#pragma unroll
+          for (int c = 0; c < B / 8; ++c) {
+            const int chunk = (col_bytes % 128) / 16 + c;
+            const uint4 v = *reinterpret_cast<const uint4*>(rowp + ((chunk ^ (rloc & 7)) * 16));
+            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              y[8 * c + 2 * h] = bf16_lo(u[h]);
+              y[8 * c + 2 * h + 1] = bf16_hi(u[h]);
+            }
+          }
+          if constexpr (KIND == kHadamard) fwht_normalized<B>(y);
+        }
+        if (jj == kBlocks - 1) {                  // the tile's values are all out of TMEM / smem
+          if constexpr (kMma) {
+            tc_fence_before();
+            mbar_arrive(&acc_empty[a]);
+          } else {
+            mbar_arrive(&x_empty[s]);
+          }
+        }
+        const int j = col0 / B + jj;
+        const bool blk_ok = row_ok && j < nb;
+        if constexpr (DBG) {
+          if (blk_ok) {
+            float4* dp = reinterpret_cast<float4*>(ydbg + static_cast<int64_t>(r) * d_in + static_cast<int64_t>(j) * B);
+#pragma unroll
+            for (int w = 0; w < B / 4; ++w) dp[w] = make_float4(y[4 * w], y[4 * w + 1], y[4 * w + 2], y[4 * w + 3]);
+          }
+        }
+        uint32_t cw[B / 8];
+        const uint32_t sc = quantize_block<B, FMT>(y, gscale, den, cw);
+        if (blk_ok) {
+          uint8_t* cp = codes + static_cast<int64_t>(r) * (d_in / 2) + static_cast<int64_t>(j) * (B / 2);
+          if constexpr (B == 32) *reinterpret_cast<uint4*>(cp) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+          else *reinterpret_cast<uint2*>(cp) = make_uint2(cw[0], cw[1]);
+        }
+        if constexpr (FMT == kI4) {
+          if (blk_ok) reinterpret_cast<uint16_t*>(scales)[static_cast<int64_t>(r) * nb + j] = static_cast<uint16_t>(sc);
+        } else {
+          sc_words[jj / 4] |= (blk_ok ? sc : 0u) << (8 * (jj % 4));
+        }
+      }
+      if constexpr (FMT != kI4) {
+        // this thread's 4 scale bytes of each 4-column atom form one aligned word
+        const int n_atom_cols = (nb + 3) / 4;
+#pragma unroll
+        for (int w4 = 0; w4 < kBlocks / 4; ++w4) {
+          const int atom_col = col0 / B / 4 + w4;
+          if (atom_col < n_atom_cols) {
+            const int64_t off = (static_cast<int64_t>(row0 / 128) * n_atom_cols + atom_col) * 512 +
+                                (rloc & 31) * 16 + (rloc >> 5) * 4;
+            *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(scales) + off) = sc_words[w4];
+          }
+        }
+      }
+      if constexpr (kMma) {
+        // The warpgroup that finishes the last tile of column k refills that
+        // column's T buffer with column k + 2: every MMA reading it has completed.
+        const int k = i / n_row_tiles - col_lo;
+        const bool last_of_col = (i + 1 == tile_hi) || ((i + 1) / n_row_tiles != i / n_row_tiles);
+        if (last_of_col && k + 2 < n_cols) convert_t(k + 2, et - g * 128, 128, 2 + g);
+      }
+    }
+  }
+
+  __syncwarp();
+  if (*abort_flag) {
+    const uint64_t until = globaltimer_ns() + 200000ull;
+    while (globaltimer_ns() < until) __nanosleep(1000);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1 && kMma) tmem_dealloc(tmem, kTmemCols);
+}
+
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn get_encode() {
+  static EncodeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(p);
+  });
+  return fn;
+}
+
+int num_sms() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev < 64 && cached[dev]) return cached[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev < 64) cached[dev] = n;
+  return n;
+}
+
+template <int B, int FMT, int KIND, bool DBG>
+int launch_tc(const void* x, int64_t rows, int64_t d_in, const float* t, float gscale, uint8_t* codes,
+              void* scales, float* ydbg, cudaStream_t st) {
+  EncodeFn enc = get_encode();
+  if (!enc) return WUSH_ERR_CUDA;
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d_in), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(d_in) * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBoxCols), static_cast<cuuint32_t>(kTileRows)};
+  const cuuint32_t estr[2] = {1, 1};
+  if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return WUSH_ERR_CUDA;
+  auto kern = tq_tc_kernel<B, FMT, KIND, DBG>;
+  static uint64_t attr_done = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return WUSH_ERR_CUDA;
+  if (dev < 64 && !(attr_done >> dev & 1)) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
+      return WUSH_ERR_CUDA;
+    attr_done |= uint64_t(1) << dev;
+  }
+  const int n_row_tiles = static_cast<int>((rows + kTileRows - 1) / kTileRows);
+  const int n_col_tiles = static_cast<int>((d_in + kTileCols - 1) / kTileCols);
+  const int n_tiles = n_row_tiles * n_col_tiles;
+  const int sms = num_sms();
+  if (sms <= 0) return WUSH_ERR_CUDA;
+  const int grid = n_tiles < sms ? n_tiles : sms;
+  const int64_t polls = g_wait_limit_override > 0 ? g_wait_limit_override : kDefaultPolls;
+  kern<<<grid, kThreads, kSmemBytes, st>>>(map, t, gscale, codes, scales, ydbg, static_cast<int>(rows),
+                                           static_cast<int>(d_in), n_row_tiles, n_tiles, polls);
+  return launch_status();
+}
+
+template <int B, int FMT>
+int dispatch_kind(int kind, const void* x, int64_t rows, int64_t d_in, const float* t, float gscale,
+                  uint8_t* codes, void* scales, float* ydbg, cudaStream_t st) {
+  const int k = kind == WUSH_T_IDENTITY ? kIdentity : (kind == WUSH_T_HADAMARD ? kHadamard : kDense);
+#define WUSH_TC(KK)                                                                                     \
+  return ydbg ? launch_tc<B, FMT, KK, true>(x, rows, d_in, t, gscale, codes, scales, ydbg, st)          \
+              : launch_tc<B, FMT, KK, false>(x, rows, d_in, t, gscale, codes, scales, ydbg, st)
+  if (k == kIdentity) { WUSH_TC(kIdentity); }
+  if (k == kHadamard) { WUSH_TC(kHadamard); }
+  WUSH_TC(kDense);
+#undef WUSH_TC
+}
+
+}  // namespace
+
+int read_and_clear_tq_error(int* word) {
+  cudaError_t e = cudaMemcpyFromSymbol(word, g_tq_error, sizeof(int));
+  if (e != cudaSuccess) return e;
+  if (*word) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_tq_error, &zero, sizeof(int));
+  }
+  return e;
+}
+
+// Tensor-core form of wush_transform_quant for bf16 inputs whose rows are 16-byte
+// aligned and whose sizes fit int32 indexing.  Returns WUSH_ERR_UNSUPPORTED when the
+// shape is outside that, so the caller can use the one-row-per-thread kernel.
+int transform_quant_tc(const void* x, int64_t rows, int64_t d_in, const float* t, int kind, int fmt,
+                       float gscale, uint8_t* codes, void* scales, float* ydbg, cudaStream_t st) {
+  if (d_in % 8 || rows > (int64_t(1) << 30) || d_in > (int64_t(1) << 30) || rows * (d_in / 2) > (int64_t(1) << 62))
+    return WUSH_ERR_UNSUPPORTED;
+  if (fmt == WUSH_FMT_MXFP4) return dispatch_kind<32, kMx>(kind, x, rows, d_in, t, gscale, codes, scales, ydbg, st);
+  if (fmt == WUSH_FMT_NVFP4) return dispatch_kind<16, kNv>(kind, x, rows, d_in, t, gscale, codes, scales, ydbg, st);
+  return dispatch_kind<32, kI4>(kind, x, rows, d_in, t, gscale, codes, scales, ydbg, st);
+}
+
+}  // namespace wush

@@ -113,7 +113,7 @@ int wush_calibrate_from_moments(const double* sigma_x, const double* sigma_w, in
  *         512 contiguous bytes; scale (r, c) of an atom sits at byte
  *         (r % 32) * 16 + (r / 32) * 4 + c; atoms are ordered row-block-major
  *         (all column atoms of rows 0..127 first).  rows is padded up to 128 and
- *         d_in/b up to 4; padding bytes are not written.
+ *         d_in/b up to 4; padding bytes are written as zero.
  *         INT4 scales are fp16, plain row-major [rows, d_in/32].
  * ------------------------------------------------------------------------- */
 size_t wush_codes_bytes(int64_t rows, int64_t d_in, int fmt);
@@ -130,9 +130,11 @@ size_t wush_scales_bytes(int64_t rows, int64_t d_in, int fmt);
  *          (e = -127 for amax 0); scale byte e + 127; code = E2M1 RNE-satfinite
  *          of y / 2^e.
  *   NVFP4: t = amax / fp32(6 * global_scale); s_b = UE4M3 RNE-satfinite(t);
- *          d = fp32(s_b * global_scale); code = E2M1 RNE-satfinite(y / d);
- *          codes 0 when s_b = 0.  global_scale is the per-tensor fp32 scale.
- *   INT4:  s = fp16 RNE(amax / 7); q = clamp(rint(y / s), -7, 7) (0 if s = 0);
+ *          d = fp32(s_b * global_scale); r = fp32(1 / d);
+ *          code = E2M1 RNE-satfinite(fp32(y * r)); codes 0 when s_b = 0.
+ *          global_scale is the per-tensor fp32 scale, in [1e-30, 1e30).
+ *   INT4:  s = fp16 RNE(amax / 7); r = fp32(1 / s);
+ *          q = clamp(rint(fp32(y * r)), -7, 7) (0 if s = 0);
  *          code = q & 0xF (two's complement nibble).
  *   All decisions in fp32 with round-to-nearest-even. E2M1 codes carry the
  *   sign of y even when the magnitude rounds to 0; an all-zero block gives +0.

@@ -16,10 +16,13 @@ MXFP4 (b = 32): amax = max |y|; e = floor(log2 amax) - 2, clamped to
   minus the element format's largest exponent, 2 for E2M1.)
 NVFP4 (b = 16): with the per-tensor fp32 scale s_g:
   t = fp32(amax) / fp32(6 * s_g);  s_b = UE4M3_RNE_sat(t);
-  d = fp32(s_b * s_g);  code = E2M1_RNE_sat(fp32(y / d)); code 0 when s_b = 0.
-  Dequantised value = E2M1(code) * s_b * s_g.
-INT4 (b = 32), symmetric: s = fp16_RNE(fp32(amax) / 7);
-  q = clamp(rint(fp32(y / s)), -7, 7); q = 0 when s = 0.  Dequantised q * s.
+  d = fp32(s_b * s_g);  r = fp32(1 / d);  code = E2M1_RNE_sat(fp32(y * r));
+  code 0 when s_b = 0.  Dequantised value = E2M1(code) * s_b * s_g.
+INT4 (b = 32), symmetric: s = fp16_RNE(fp32(amax) / 7); r = fp32(1 / s);
+  q = clamp(rint(fp32(y * r)), -7, 7); q = 0 when s = 0.  Dequantised q * s.
+  (Each element is multiplied by the block's fp32 reciprocal scale rather than
+  divided by the scale: the pages leave the order of operations open, and one
+  division per block instead of per element is the kernel's choice.)
 
 A block whose amax is 0 gets codes +0.  Otherwise the E2M1 sign bit is the sign
 bit of y, also when the magnitude rounds to 0.
@@ -78,14 +81,16 @@ def quantize_nvfp4(y32: np.ndarray, s_g) -> dict:
     sb = e4m3_code_unsigned(t.astype(np.float64))
     sbv = e4m3_value(sb).astype(F32)             # every UE4M3 value is exact in fp32
     d = (sbv * s_g).astype(F32)
-    safe_d = np.where(d == 0, F32(1.0), d)
-    v = (yb / safe_d[..., None]).astype(F32)
+    live = (sb != 0) & (amax > 0)
+    rcp = np.where(live, (F32(1.0) / np.where(d == 0, F32(1.0), d)).astype(F32), F32(0.0)).astype(F32)
+    v = (yb * rcp[..., None]).astype(F32)
     codes = e2m1_code(v.astype(np.float64))
-    zero_blk = (sb == 0) | (amax == 0)
-    codes = np.where(zero_blk[..., None], 0, codes).astype(np.uint8)
+    codes = np.where(live[..., None], codes, 0).astype(np.uint8)
     dq = e2m1_value(codes) * (e4m3_value(sb) * np.float64(s_g))[..., None]
-    elem_margin = (distance_to_boundary(np.abs(v.astype(np.float64)), E2M1_BOUNDARIES)
-                   * d.astype(np.float64)[..., None])
+    with np.errstate(divide="ignore"):
+        elem_margin = np.where(live[..., None],
+                               distance_to_boundary(np.abs(v.astype(np.float64)), E2M1_BOUNDARIES)
+                               / rcp.astype(np.float64)[..., None], np.inf)
     block_margin = distance_to_boundary(t.astype(np.float64), E4M3_MIDPOINTS) * np.float64(den)
     rows = yb.shape[0]
     return dict(codes=codes.reshape(rows, -1), scale_bytes=sb, scale=e4m3_value(sb),
@@ -108,13 +113,15 @@ def quantize_int4(y32: np.ndarray) -> dict:
     pre = (amax / F32(7.0)).astype(F32)
     s16 = fp16_rne_sat(pre)
     s = s16.astype(F32)
-    safe_s = np.where(s == 0, F32(1.0), s)
-    v = (yb / safe_s[..., None]).astype(F32)
+    rcp = np.where(s > 0, (F32(1.0) / np.where(s > 0, s, F32(1.0))).astype(F32), F32(0.0)).astype(F32)
+    v = (yb * rcp[..., None]).astype(F32)
     q = np.clip(np.rint(v), -7, 7).astype(np.int64)
     q = np.where((s == 0)[..., None], 0, q)
     dq = q * s.astype(np.float64)[..., None]
-    elem_margin = (distance_to_boundary(np.abs(v.astype(np.float64)), INT4_MIDPOINTS)
-                   * s.astype(np.float64)[..., None])
+    with np.errstate(divide="ignore"):
+        elem_margin = np.where((s > 0)[..., None],
+                               distance_to_boundary(np.abs(v.astype(np.float64)), INT4_MIDPOINTS)
+                               / rcp.astype(np.float64)[..., None], np.inf)
     block_margin = _fp16_midpoint_distance(pre) * 7.0
     rows = yb.shape[0]
     return dict(codes=(q & 0xF).astype(np.uint8).reshape(rows, -1), q=q.reshape(rows, -1),

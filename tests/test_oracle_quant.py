@@ -78,7 +78,7 @@ def test_nvfp4_brute_force():
             sb = 126 if t > 448 else min(cands, key=lambda c: (c & 1, c))
             assert q["scale_bytes"][r, j] == sb
             d = F32(F32(grid[sb]) * s_g)
-            want = _nearest_code_brute((yb[r, j] / d).astype(F32))
+            want = _nearest_code_brute((yb[r, j] * F32(F32(1) / d)).astype(F32))
             assert np.array_equal(q["codes"][r, 16 * j:16 * j + 16], want)
 
 
@@ -89,7 +89,7 @@ def test_int4_brute_force():
     for r in range(6):
         for j in range(4):
             s = np.float16(F32(np.max(np.abs(yb[r, j]))) / F32(7))
-            v = (yb[r, j] / F32(s)).astype(F32)
+            v = (yb[r, j] * F32(F32(1) / F32(s))).astype(F32)
             want = []
             for x in v.astype(np.float64):
                 cands = np.arange(-7, 8)
