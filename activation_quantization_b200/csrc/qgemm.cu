@@ -9,17 +9,20 @@
 // (NVFP4, kind::mxf4nvf4, block16).  Products of codes and scales are exact;
 // accumulation is fp32 in TMEM.
 //
-// One CTA computes one 128 x BN output tile (BN = 256, or 128 when N % 256 != 0)
-// with 4 warps:
-//   warp 0  TMA producer: per 256-wide k-tile, one 2D TMA load of the A tile
-//           (128 rows x 128 bytes, 128-byte swizzle), one of the B tile, and
-//           untiled bulk copies of the matching 512-byte scale atoms, all
-//           completing on the stage's "full" mbarrier;
-//   warp 1  allocates TMEM; one elected thread copies the stage's scale atoms
-//           into TMEM (tcgen05.cp 32x128b.warpx4) and issues the four K=64
-//           block-scaled MMAs, then commits the stage back to the producer;
-//   warps 0-3  epilogue: tcgen05.ld of the fp32 accumulator rows, times alpha,
-//           stored to y.
+// A persistent CTA per SM walks 128 x BN output tiles (BN = 256, or 128 when
+// N % 256 != 0) round-robin, with three roles:
+//   warp 0     TMA producer: per 256-wide k-tile, one 2D TMA load of the A tile
+//              (128 rows x 128 bytes, 128-byte swizzle), one of the B tile, and
+//              untiled bulk copies of the matching 512-byte scale atoms, all
+//              completing on the stage's "full" mbarrier; the 4-stage ring runs
+//              on across tile boundaries;
+//   warp 1     allocates TMEM; one elected thread copies the stage's scale atoms
+//              into TMEM (tcgen05.cp 32x128b.warpx4) and issues the four K=64
+//              block-scaled MMAs, then commits the stage back to the producer;
+//   warps 2-9  epilogue: tcgen05.ld of the fp32 accumulator (two warps per TMEM
+//              lane quarter, half the columns each), release of the accumulator
+//              as soon as it is in registers, then times alpha and stored to y
+//              while the next tile's MMAs already run.
 // Every mbarrier wait is bounded (poll count, wall time, and a shared abort
 // flag); a wait that gives up records a device error word and the CTA drains
 // and frees its TMEM before returning.
@@ -53,12 +56,14 @@ constexpr int kBM = 128;
 constexpr int kBK = 256;             // fp4 elements per k-tile = 128 bytes per row
 constexpr int kBKBytes = kBK / 2;
 constexpr int kStages = 4;
-constexpr int kThreads = 128;
+constexpr int kEpiWarps = 8;                      // two per TMEM lane quarter
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kThreads = 64 + kEpiThreads;         // producer warp, MMA warp, epilogue
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSfaCol = 256;    // TMEM column of the A scale factors
 constexpr uint32_t kSfbCol = 288;    // TMEM column of the B scale factors
 constexpr int64_t kDefaultPolls = int64_t(1) << 40;
-constexpr uint64_t kDeadlineNs = 4000000000ull;  // 4 s of wall time per wait
+constexpr uint64_t kDeadlineNs = 4000000000ull;  // 4 s of wall time per wait, from its start
 
 template <int BN, bool NV>
 struct Cfg {
@@ -84,17 +89,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * C::kStageBytes);
   uint64_t* empty = full + kStages;
   uint64_t* acc_full = empty + kStages;
-  uint64_t* never = acc_full + 1;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* never = acc_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const int n_blk = blockIdx.x;
-  const int m_blk = blockIdx.y;
+  const int n_tiles_n = N / BN;
+  const int n_tiles = (M / kBM) * n_tiles_n;
   const int k_tiles = K / kBK;
   const int n_acols = (K / (NV ? 16 : 32) + 3) / 4;     // scale atoms per 128-row block
-  const uint64_t deadline = globaltimer_ns() + kDeadlineNs;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -102,6 +107,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&empty[s], 1);
     }
     mbar_init(acc_full, 1);
+    mbar_init(acc_empty, kEpiThreads);
     mbar_init(never, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -114,30 +120,44 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  auto give_up = [&]() {
+    if (!*abort_flag) {
+      *abort_flag = 1;
+      atomicOr(&g_error_word, 1 << kErrTimeoutBarrier);
+    }
+  };
+
+  // Tiles are taken round-robin, walking down M inside each BN-wide column of
+  // output so that concurrently running CTAs share their B (weight) tiles in L2.
   if (warp == 0) {
     if (elect_one()) {
-      for (int kt = 0; kt < k_tiles; ++kt) {
-        const int s = kt % kStages;
-        const uint32_t ph = (kt / kStages) & 1;
-        if (!mbar_wait_bounded(&empty[s], ph ^ 1, max_polls, deadline, abort_flag)) {
-          if (!*abort_flag) { *abort_flag = 1; atomicOr(&g_error_word, 1 << kErrTimeoutBarrier); }
-          break;
-        }
-        uint8_t* st = smem + s * C::kStageBytes;
-        uint8_t* sa = st;
-        uint8_t* sb = sa + C::kABytes;
-        uint8_t* ssfa = sb + C::kBBytes;
-        uint8_t* ssfb = ssfa + C::kSfaBytes;
-        mbar_arrive_expect_tx(&full[s], C::kTxBytes);
-        tma_load_2d(sa, &tmap_a, kt * kBKBytes, m_blk * kBM, &full[s]);
-        tma_load_2d(sb, &tmap_b, kt * kBKBytes, n_blk * BN, &full[s]);
-        bulk_load(ssfa, sfa + (static_cast<int64_t>(m_blk) * n_acols + kt * C::kAtomsK) * 512, C::kSfaBytes,
-                  &full[s]);
+      int it = 0;  // k-tile counter over all of this CTA's tiles: drives the ring
+      for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+        const int m_blk = tile % (M / kBM), n_blk = tile / (M / kBM);
+        bool ok = true;
+        for (int kt = 0; kt < k_tiles; ++kt, ++it) {
+          const int s = it % kStages;
+          if (!mbar_wait_bounded(&empty[s], ((it / kStages) & 1) ^ 1, max_polls, kDeadlineNs, abort_flag)) {
+            give_up();
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + s * C::kStageBytes;
+          uint8_t* sb = sa + C::kABytes;
+          uint8_t* ssfa = sb + C::kBBytes;
+          uint8_t* ssfb = ssfa + C::kSfaBytes;
+          mbar_arrive_expect_tx(&full[s], C::kTxBytes);
+          tma_load_2d(sa, &tmap_a, kt * kBKBytes, m_blk * kBM, &full[s]);
+          tma_load_2d(sb, &tmap_b, kt * kBKBytes, n_blk * BN, &full[s]);
+          bulk_load(ssfa, sfa + (static_cast<int64_t>(m_blk) * n_acols + kt * C::kAtomsK) * 512, C::kSfaBytes,
+                    &full[s]);
 #pragma unroll
-        for (int h = 0; h < C::kRowAtomsB; ++h)
-          bulk_load(ssfb + h * C::kAtomsK * 512,
-                    sfb + (static_cast<int64_t>(n_blk * C::kRowAtomsB + h) * n_acols + kt * C::kAtomsK) * 512,
-                    C::kAtomsK * 512, &full[s]);
+          for (int h = 0; h < C::kRowAtomsB; ++h)
+            bulk_load(ssfb + h * C::kAtomsK * 512,
+                      sfb + (static_cast<int64_t>(n_blk * C::kRowAtomsB + h) * n_acols + kt * C::kAtomsK) * 512,
+                      C::kAtomsK * 512, &full[s]);
+        }
+        if (!ok) break;
       }
     }
   } else if (warp == 1) {
@@ -145,73 +165,84 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       if (debug_never) {
         // test hook: wait on a barrier nothing arrives on, to exercise the give-up path
-        ok = mbar_wait_bounded(never, 0, max_polls, deadline, abort_flag);
+        ok = mbar_wait_bounded(never, 0, max_polls, kDeadlineNs, abort_flag);
       }
       const uint32_t tsfa = tmem + kSfaCol;
       const uint32_t tsfb = tmem + kSfbCol;
-      for (int kt = 0; ok && kt < k_tiles; ++kt) {
-        const int s = kt % kStages;
-        const uint32_t ph = (kt / kStages) & 1;
-        if (!mbar_wait_bounded(&full[s], ph, max_polls, deadline, abort_flag)) { ok = false; break; }
+      int it = 0, tcount = 0;
+      for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x, ++tcount) {
+        // the epilogue must have drained the accumulator of the previous tile
+        if (!mbar_wait_bounded(acc_empty, (tcount & 1) ^ 1, max_polls, kDeadlineNs, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        uint8_t* st = smem + s * C::kStageBytes;
-        const uint32_t sa = smem_u32(st);
-        const uint32_t sb = sa + C::kABytes;
-        const uint32_t ssfa = sb + C::kBBytes;
-        const uint32_t ssfb = ssfa + C::kSfaBytes;
+        for (int kt = 0; kt < k_tiles; ++kt, ++it) {
+          const int s = it % kStages;
+          if (!mbar_wait_bounded(&full[s], (it / kStages) & 1, max_polls, kDeadlineNs, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + s * C::kStageBytes);
+          const uint32_t sb = sa + C::kABytes;
+          const uint32_t ssfa = sb + C::kBBytes;
+          const uint32_t ssfb = ssfa + C::kSfaBytes;
 #pragma unroll
-        for (int a = 0; a < C::kAtomsK; ++a) {
-          tc_cp_32x128b_warpx4(tsfa + 4 * a, desc_sf_atom(ssfa + a * 512));
+          for (int a = 0; a < C::kAtomsK; ++a) {
+            tc_cp_32x128b_warpx4(tsfa + 4 * a, desc_sf_atom(ssfa + a * 512));
 #pragma unroll
-          for (int h = 0; h < C::kRowAtomsB; ++h)
-            tc_cp_32x128b_warpx4(tsfb + 4 * (C::kRowAtomsB * a + h), desc_sf_atom(ssfb + (h * C::kAtomsK + a) * 512));
+            for (int h = 0; h < C::kRowAtomsB; ++h)
+              tc_cp_32x128b_warpx4(tsfb + 4 * (C::kRowAtomsB * a + h), desc_sf_atom(ssfb + (h * C::kAtomsK + a) * 512));
+          }
+#pragma unroll
+          for (int kk = 0; kk < kBK / 64; ++kk) {
+            const int atom = NV ? kk : kk / 2;
+            const uint32_t sf_id = NV ? 0u : 2u * (kk & 1);
+            const uint32_t idesc = idesc_block_scaled_e2m1(kBM, BN, NV ? 0u : 1u, sf_id, sf_id);
+            const uint64_t ad = desc_kmajor_sw128(sa + kk * 32);
+            const uint64_t bd = desc_kmajor_sw128(sb + kk * 32);
+            mma_block_scaled<NV>(tmem, ad, bd, idesc, (kt | kk) ? 1u : 0u, (tsfa + 4 * atom) | (sf_id << 30),
+                                 (tsfb + 4 * C::kRowAtomsB * atom) | (sf_id << 30));
+          }
+          tc_commit(&empty[s]);
         }
-#pragma unroll
-        for (int kk = 0; kk < kBK / 64; ++kk) {
-          const int atom = NV ? kk : kk / 2;
-          const uint32_t sf_id = NV ? 0u : 2u * (kk & 1);
-          const uint32_t idesc = idesc_block_scaled_e2m1(kBM, BN, NV ? 0u : 1u, sf_id, sf_id);
-          const uint64_t ad = desc_kmajor_sw128(sa + kk * 32);
-          const uint64_t bd = desc_kmajor_sw128(sb + kk * 32);
-          mma_block_scaled<NV>(tmem, ad, bd, idesc, (kt | kk) ? 1u : 0u,
-                               (tsfa + 4 * atom) | (sf_id << 30),
-                               (tsfb + 4 * C::kRowAtomsB * atom) | (sf_id << 30));
-        }
-        tc_commit(&empty[s]);
-      }
-      if (ok) {
+        if (!ok) break;
         tc_commit(acc_full);
-      } else if (!*abort_flag) {
-        *abort_flag = 1;
-        atomicOr(&g_error_word, 1 << kErrTimeoutBarrier);
+      }
+      if (!ok) give_up();
+    }
+  } else {
+    // epilogue: warp w drains TMEM lane quarter w % 4 (rows 32*(w%4) ..), columns
+    // [half * BN/2, (half + 1) * BN/2); the accumulator is released as soon as its
+    // values are in registers, so the next tile's MMAs overlap these stores.
+    const int ew = warp - 2;
+    const int q = warp & 3;
+    const int half = ew / 4;
+    int tcount = 0;
+    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++tcount) {
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+      const int m_blk = tile % (M / kBM), n_blk = tile / (M / kBM);
+      bool ok = mbar_wait_bounded(acc_full, tcount & 1, max_polls, kDeadlineNs, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) { give_up(); break; }
+      tc_fence_after();
+      const int row = m_blk * kBM + q * 32 + lane;
+      float* yrow = y + static_cast<int64_t>(row) * N + static_cast<int64_t>(n_blk) * BN + half * (BN / 2);
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + half * (BN / 2);
+#pragma unroll 1
+      for (int c = 0; c < BN / 2; c += 32) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tbase + c, r);
+        tmem_ld_wait();
+        if (c + 32 == BN / 2) {
+          tc_fence_before();
+          mbar_arrive(acc_empty);
+        }
+        float4* dst = reinterpret_cast<float4*>(yrow + c);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          dst[j] = make_float4(alpha * __uint_as_float(r[4 * j]), alpha * __uint_as_float(r[4 * j + 1]),
+                               alpha * __uint_as_float(r[4 * j + 2]), alpha * __uint_as_float(r[4 * j + 3]));
       }
     }
   }
   __syncwarp();
 
-  // epilogue: every warp drains its 32 TMEM lanes (rows 32*warp .. 32*warp + 31)
-  bool have_acc = mbar_wait_bounded(acc_full, 0, max_polls, deadline, abort_flag);
-  if (!have_acc && !*abort_flag) {
-    *abort_flag = 1;
-    atomicOr(&g_error_word, 1 << kErrTimeoutBarrier);
-  }
-  have_acc = __all_sync(0xffffffffu, have_acc);
-  if (have_acc) {
-    tc_fence_after();
-    const int row = m_blk * kBM + warp * 32 + lane;
-    float* yrow = y + static_cast<int64_t>(row) * N + static_cast<int64_t>(n_blk) * BN;
-#pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
-      uint32_t r[32];
-      tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c, r);
-      tmem_ld_wait();
-      float4* dst = reinterpret_cast<float4*>(yrow + c);
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        dst[q] = make_float4(alpha * __uint_as_float(r[4 * q]), alpha * __uint_as_float(r[4 * q + 1]),
-                             alpha * __uint_as_float(r[4 * q + 2]), alpha * __uint_as_float(r[4 * q + 3]));
-    }
-  }
   if (*abort_flag) {
     // let loads and MMAs already issued by this CTA land before its shared memory
     // and TMEM are released
@@ -222,6 +253,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+int num_sms() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev < 64 && cached[dev]) return cached[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev < 64) cached[dev] = n;
+  return n;
 }
 
 using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -271,7 +313,10 @@ int launch(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const uint8_t
   }
   const int64_t polls = g_wait_limit_override > 0 ? g_wait_limit_override : kDefaultPolls;
   const int debug_never = g_wait_limit_override > 0 ? 1 : 0;
-  const dim3 grid(static_cast<unsigned>(N / BN), static_cast<unsigned>(M / kBM));
+  const int n_tiles = static_cast<int>((M / kBM) * (N / BN));
+  const int sms = num_sms();
+  if (sms <= 0) return WUSH_ERR_CUDA;
+  const dim3 grid(static_cast<unsigned>(n_tiles < sms ? n_tiles : sms));
   kern<<<grid, kThreads, C::kSmemBytes, st>>>(ma, mb, sfa, sfb, y, static_cast<int>(M), static_cast<int>(N),
                                               static_cast<int>(K), alpha, polls, debug_never);
   return launch_status();

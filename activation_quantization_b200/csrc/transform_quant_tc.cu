@@ -222,7 +222,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tile_lo = static_cast<int>(static_cast<int64_t>(blockIdx.x) * n_tiles / gridDim.x);
   const int tile_hi = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * n_tiles / gridDim.x);
   const int col_lo = tile_lo / n_row_tiles;
-  const uint64_t deadline = globaltimer_ns() + kDeadlineNs;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -255,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (elect_one()) {
       for (int i = tile_lo; i < tile_hi; ++i) {
         const int n = i - tile_lo, s = n % kStages;
-        if (!mbar_wait_bounded(&x_empty[s], ((n / kStages) & 1) ^ 1, max_polls, deadline, abort_flag)) {
+        if (!mbar_wait_bounded(&x_empty[s], ((n / kStages) & 1) ^ 1, max_polls, kDeadlineNs, abort_flag)) {
           give_up();
           break;
         }
@@ -272,9 +271,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = tile_lo; i < tile_hi; ++i) {
         const int n = i - tile_lo, s = n % kStages, a = n % kAccs;
         const int k = i / n_row_tiles - col_lo;     // column ordinal within this CTA
-        if (!mbar_wait_bounded(&t_full[k & 1], (k >> 1) & 1, max_polls, deadline, abort_flag) ||
-            !mbar_wait_bounded(&acc_empty[a], ((n / kAccs) & 1) ^ 1, max_polls, deadline, abort_flag) ||
-            !mbar_wait_bounded(&x_full[s], (n / kStages) & 1, max_polls, deadline, abort_flag)) {
+        if (!mbar_wait_bounded(&t_full[k & 1], (k >> 1) & 1, max_polls, kDeadlineNs, abort_flag) ||
+            !mbar_wait_bounded(&acc_empty[a], ((n / kAccs) & 1) ^ 1, max_polls, kDeadlineNs, abort_flag) ||
+            !mbar_wait_bounded(&x_full[s], (n / kStages) & 1, max_polls, kDeadlineNs, abort_flag)) {
           give_up();
           break;
         }
@@ -369,8 +368,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int r = row0 + rloc;
       const bool row_ok = r < rows;
       bool ok;
-      if constexpr (kMma) ok = mbar_wait_bounded(&acc_full[a], (n / kAccs) & 1, max_polls, deadline, abort_flag);
-      else ok = mbar_wait_bounded(&x_full[s], (n / kStages) & 1, max_polls, deadline, abort_flag);
+      if constexpr (kMma) ok = mbar_wait_bounded(&acc_full[a], (n / kAccs) & 1, max_polls, kDeadlineNs, abort_flag);
+      else ok = mbar_wait_bounded(&x_full[s], (n / kStages) & 1, max_polls, kDeadlineNs, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) { give_up(); break; }
       if constexpr (kMma) tc_fence_after();
