@@ -42,6 +42,7 @@ _SIGNATURES = {
     "itq3_dequant_gemv_noalloc": (_i32, [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp]),
     "wush_check_device_status": (_i32, [_vp]),
     "wush_debug_set_wait_limit": (_i32, [_i64]),
+    "wush_debug_set_gemm_variant": (_i32, [_i32]),
 }
 
 EXPORTED = []
@@ -200,6 +201,10 @@ def itq3_dequant_gemv_noalloc(codes, scales, x, d_out: int, y, stream=None):
 
 def wush_check_device_status(stream=None) -> int:
     return _lib.wush_check_device_status(_stream(stream))
+
+
+def wush_debug_set_gemm_variant(variant: int):
+    _check("wush_debug_set_gemm_variant", _lib.wush_debug_set_gemm_variant(int(variant)))
 
 
 def wush_debug_set_wait_limit(max_polls: int):

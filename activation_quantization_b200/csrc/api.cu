@@ -27,6 +27,12 @@ extern "C" int wush_check_device_status(void* stream) {
   return (word | word_tq) == 0 ? WUSH_OK : WUSH_ERR_TIMEOUT;
 }
 
+extern "C" int wush_debug_set_gemm_variant(int variant) {
+  if (variant < 0 || variant > 2) return WUSH_ERR_INVALID_ARG;
+  wush::g_gemm_variant = variant;
+  return WUSH_OK;
+}
+
 extern "C" int wush_debug_set_wait_limit(int64_t max_polls) {
   if (max_polls < 0) return WUSH_ERR_INVALID_ARG;
   wush::g_wait_limit_override = max_polls;

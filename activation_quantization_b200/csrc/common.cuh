@@ -24,6 +24,9 @@ int read_and_clear_tq_error(int* word);
 int transform_quant_tc(const void* x, int64_t rows, int64_t d_in, const float* t, int kind, int fmt,
                        float gscale, uint8_t* codes, void* scales, float* ydbg, cudaStream_t st);
 
+// GEMM kernel choice (see wush_debug_set_gemm_variant).
+extern int g_gemm_variant;
+
 // Poll limit for bounded mbarrier waits (0 = the built-in default).
 extern int64_t g_wait_limit_override;
 

@@ -250,6 +250,12 @@ int wush_check_device_status(void* stream);
  * path can be exercised without hanging anything. */
 int wush_debug_set_wait_limit(int64_t max_polls);
 
+/* Test hook: 0 (default) lets wush_qgemm use CTA-pair (cta_group::2) 256 x 256
+ * tiles when M % 256 == 0 and N % 256 == 0; 1 uses single-CTA 128 x 256 tiles
+ * (when N % 256 == 0), 2 single-CTA 128 x 128 tiles, so that the forms can be
+ * checked against each other. */
+int wush_debug_set_gemm_variant(int variant);
+
 #ifdef __cplusplus
 }
 #endif

@@ -42,18 +42,32 @@ def _rel_fro(got, want):
     return float(np.linalg.norm(got - want) / np.linalg.norm(want))
 
 
+SHAPES = [(128, 256, 256), (256, 512, 2048), (384, 384, 1280), (128, 128, 4096),
+          (256, 256, 256), (512, 768, 1536), (1024, 1024, 4096)]
+
+
 @pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
-@pytest.mark.parametrize("mnk", [(128, 256, 256), (256, 512, 2048), (384, 384, 1280), (128, 128, 4096)])
-def test_gemm_random_codes(lib, fmt, mnk):
+@pytest.mark.parametrize("mnk", SHAPES)
+@pytest.mark.parametrize("variant", [0, 1, 2])
+def test_gemm_random_codes(lib, fmt, mnk, variant):
+    # variant 0: CTA-pair 256x256 tiles when M, N % 256 == 0; 1: single-CTA 128x256; 2: single-CTA 128x128
     m, n, k = mnk
+    if variant == 1 and (m % 256 or n % 256):
+        pytest.skip("same kernel as variant 0")
+    if variant == 2 and n % 256:
+        pytest.skip("same kernel as variant 0")
+    lib.wush_debug_set_gemm_variant(variant)
     a_c, a_s, a_dq = _random_operand(101 + m + k, m, k, fmt)
     b_c, b_s, b_dq = _random_operand(202 + n + k, n, k, fmt)
     alpha = 0.37 if fmt == "nvfp4" else 1.0
     dev = "cuda"
     y = torch.full((m, n), float("nan"), dtype=torch.float32, device=dev)
-    lib.wush_qgemm(torch.from_numpy(a_c).to(dev), torch.from_numpy(a_s).to(dev), torch.from_numpy(b_c).to(dev),
-                   torch.from_numpy(b_s).to(dev), m, n, k, fmt, alpha, y)
-    assert lib.wush_check_device_status() == 0
+    try:
+        lib.wush_qgemm(torch.from_numpy(a_c).to(dev), torch.from_numpy(a_s).to(dev), torch.from_numpy(b_c).to(dev),
+                       torch.from_numpy(b_s).to(dev), m, n, k, fmt, alpha, y)
+        assert lib.wush_check_device_status() == 0
+    finally:
+        lib.wush_debug_set_gemm_variant(0)
     got = y.cpu().numpy().astype(np.float64)
     want = G.gemm_dequantized(a_dq, b_dq, alpha)
     assert np.isfinite(got).all()
@@ -131,8 +145,9 @@ def test_full_size_up_proj_sampled(lib):
     assert _rel_fro(got, want) <= P.GEMM_REL_FRO
 
 
-def test_bounded_wait_gives_up_and_context_survives(lib):
-    m, n, k = 128, 256, 512
+@pytest.mark.parametrize("m", [128, 256])     # single-CTA kernel, CTA-pair kernel
+def test_bounded_wait_gives_up_and_context_survives(lib, m):
+    n, k = 256, 512
     a_c, a_s, a_dq = _random_operand(7, m, k, "mxfp4")
     b_c, b_s, b_dq = _random_operand(8, n, k, "mxfp4")
     dev = "cuda"
