@@ -37,6 +37,7 @@ _SIGNATURES = {
     "wush_transform_quant": (_i32, [_vp, _i32, _i64, _i64, _vp, _i32, _i32, _f32, _vp, _vp, _vp, _vp]),
     "wush_transform_amax": (_i32, [_vp, _i32, _i64, _i64, _vp, _i32, _i32, _vp, _vp]),
     "wush_qgemm": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _f32, _vp, _vp]),
+    "wush_qgemm_int4": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp]),
     "itq3_quantize_weights": (_i32, [_vp, _i64, _i64, _vp, _vp]),
     "itq3_dequant_gemv": (_i32, [_vp, _vp, _vp, _i64, _i64, _i64, _i32, _vp, _vp, _vp]),
     "itq3_dequant_gemv_noalloc": (_i32, [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp]),
@@ -182,6 +183,12 @@ def wush_qgemm(a_codes, a_scales, b_codes, b_scales, M: int, N: int, K: int, fmt
     _check("wush_qgemm",
            _lib.wush_qgemm(_ptr(a_codes), _ptr(a_scales), _ptr(b_codes), _ptr(b_scales), M, N, K,
                            _enum(FORMATS, fmt), float(alpha), _ptr(y), _stream(stream)))
+
+
+def wush_qgemm_int4(a_codes, a_scales, b_codes, b_scales, M: int, N: int, K: int, y, stream=None):
+    _check("wush_qgemm_int4",
+           _lib.wush_qgemm_int4(_ptr(a_codes), _ptr(a_scales), _ptr(b_codes), _ptr(b_scales), M, N, K, _ptr(y),
+                                _stream(stream)))
 
 
 def itq3_dequant_gemv(codes, scales, x, d_out: int, mode: int, y, workspace=None, stream=None):

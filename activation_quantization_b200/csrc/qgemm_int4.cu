@@ -1,0 +1,325 @@
+// INT4 x INT4 GEMM with per-32-group fp16 scales on tcgen05 tensor cores.
+//
+// WUSH news article, experiments paragraph: INT4 is the format where WUSH cuts
+// the layer loss most.  y[m, n] = sum_g s_a[m, g] s_b[n, g] sum_{k in g} q_a q_b,
+// with q in [-7, 7] (two's-complement nibbles, low nibble = lower k) and fp16 s.
+// sm_100 tensor cores have no 4-bit integer kind and no per-group integer
+// scaling, so each operand element is dequantised to fp16(q * s) -- one rounding,
+// relative error <= 2^-11 -- and multiplied with kind::f16 MMAs (fp16 x fp16,
+// fp32 accumulation in TMEM).
+//
+// A persistent CTA per SM walks 128 x 256 output tiles round-robin (M fastest):
+//   warps 0-7   dequantisers: per 64-wide k-step, thread t turns row t of the B
+//               tile (and, for t < 128, row t of the A tile) from 32 code bytes
+//               and two fp16 scales into 128 bytes of fp16 written in the 128-byte
+//               swizzled K-major operand layout of a 4-stage shared ring;
+//   warp 8      allocates TMEM; one thread issues four M=128 N=256 K=16 MMAs per
+//               k-step and commits the stage back to the dequantisers;
+//   warps 9-16  epilogue: TMEM -> registers -> 128-byte-swizzled shared chunk ->
+//               TMA store of y (fp32), releasing the accumulator once it is read.
+// Every wait is bounded; a wait that gives up sets the device error word.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace wush {
+
+static __device__ int g_int4_error = 0;
+
+int read_and_clear_int4_error(int* word) {
+  cudaError_t e = cudaMemcpyFromSymbol(word, g_int4_error, sizeof(int));
+  if (e != cudaSuccess) return e;
+  if (*word) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_int4_error, &zero, sizeof(int));
+  }
+  return e;
+}
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kBM = 128, kBN = 256, kBK = 64;          // fp16 elements: 128-byte operand rows
+constexpr int kStages = 4;
+constexpr int kDqWarps = 8, kDqThreads = kDqWarps * 32;
+constexpr int kMmaWarp = kDqWarps;
+constexpr int kEpiWarp0 = kDqWarps + 1, kEpiWarps = 8, kEpiThreads = kEpiWarps * 32;
+constexpr int kThreads = (kEpiWarp0 + kEpiWarps) * 32;  // 544
+constexpr int kABytes = kBM * kBK * 2;                   // 16 KB
+constexpr int kBBytes = kBN * kBK * 2;                   // 32 KB
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kEpiChunkBytes = 32 * 32 * 4;
+constexpr int kSmemBytes = kStages * kStageBytes + kEpiWarps * kEpiChunkBytes + 1024 + 256;
+constexpr uint32_t kTmemCols = 256;
+constexpr int64_t kDefaultPolls = int64_t(1) << 40;
+constexpr uint64_t kDeadlineNs = 4000000000ull;
+
+// Instruction descriptor, kind::f16: fp16 A and B (K-major), fp32 D, M x N.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(uint32_t m, uint32_t n) {
+  return (1u << 4) | ((n >> 3) << 17) | ((m >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// Eight two's-complement nibbles (element 2i in the low nibble of byte i) times the
+// fp16 scale s2 = (s, s): four half2 words holding elements (0,1) (2,3) (4,5) (6,7).
+// Each nibble is biased to q + 8, placed in the mantissa of 1024.0 (0x6400 | n =
+// 1024 + n exactly), 1032 is subtracted (exact), then one fp16 multiply by s.
+__device__ __forceinline__ void dequant8(uint32_t w, __half2 s2, uint32_t (&out)[4]) {
+  const uint32_t b = w ^ 0x88888888u;
+  const uint32_t kMagic = 0x64006400u;
+  const __half2 bias = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));  // 1032
+  uint32_t h[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = ((b >> (4 * i)) & 0x000F000Fu) | kMagic;  // (e_i, e_{i+4})
+  __half2 v[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __half2 x = *reinterpret_cast<const __half2*>(&h[i]);
+    v[i] = __hmul2(__hsub2(x, bias), s2);
+  }
+  const uint32_t* u = reinterpret_cast<const uint32_t*>(v);
+  out[0] = prmt(u[0], u[1], 0x5410);   // e0, e1
+  out[1] = prmt(u[2], u[3], 0x5410);   // e2, e3
+  out[2] = prmt(u[0], u[1], 0x7632);   // e4, e5
+  out[3] = prmt(u[2], u[3], 0x7632);   // e6, e7
+}
+
+// One operand row of a 64-wide k-step: 32 code bytes + the two group scales ->
+// 128 bytes of fp16 at row ``r`` of a 128-byte-swizzled tile.
+__device__ __forceinline__ void dequant_row(const uint8_t* __restrict__ codes, const __half* __restrict__ scales,
+                                            uint8_t* tile, int r) {
+  const uint4 c0 = __ldg(reinterpret_cast<const uint4*>(codes));
+  const uint4 c1 = __ldg(reinterpret_cast<const uint4*>(codes + 16));
+  const __half2 sc = __ldg(reinterpret_cast<const __half2*>(scales));
+  const __half2 s0 = __low2half2(sc), s1 = __high2half2(sc);
+  const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {           // j: 8 elements = one 16-byte chunk of the fp16 row
+    uint32_t o[4];
+    dequant8(w[j], j < 4 ? s0 : s1, o);
+    *reinterpret_cast<uint4*>(tile + r * 128 + ((j ^ (r & 7)) * 16)) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    qgemm_int4_kernel(const uint8_t* __restrict__ a_codes, const __half* __restrict__ a_scales,
+                      const uint8_t* __restrict__ b_codes, const __half* __restrict__ b_scales,
+                      const __grid_constant__ CUtensorMap tmap_y, int M, int N, int K, int64_t max_polls) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* epi_smem = smem + kStages * kStageBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(epi_smem + kEpiWarps * kEpiChunkBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* acc_full = empty + kStages;
+  uint64_t* acc_empty = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int mt = M / kBM, n_tiles = mt * (N / kBN), k_steps = K / kBK;
+  const int64_t row_bytes = K / 2, n_groups = K / 32;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], kDqThreads);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, kEpiThreads);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tmap_y);
+  }
+  if (warp == kMmaWarp) tmem_alloc(tmem_slot, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto give_up = [&]() {
+    if (!*abort_flag) {
+      *abort_flag = 1;
+      atomicOr(&g_int4_error, 1 << kErrTimeoutBarrier);
+    }
+  };
+
+  if (warp < kDqWarps) {
+    const int t = threadIdx.x;                       // B row t of the tile; A row t for t < 128
+    int it = 0;
+    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+      const int m0 = (tile % mt) * kBM, n0 = (tile / mt) * kBN;
+      const uint8_t* brow = b_codes + static_cast<int64_t>(n0 + t) * row_bytes;
+      const __half* bsc = b_scales + static_cast<int64_t>(n0 + t) * n_groups;
+      const uint8_t* arow = a_codes + static_cast<int64_t>(m0 + (t & 127)) * row_bytes;
+      const __half* asc = a_scales + static_cast<int64_t>(m0 + (t & 127)) * n_groups;
+      bool ok = true;
+      for (int ks = 0; ks < k_steps; ++ks, ++it) {
+        const int s = it % kStages;
+        ok = mbar_wait_bounded(&empty[s], ((it / kStages) & 1) ^ 1, max_polls, kDeadlineNs, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) { give_up(); ok = false; break; }
+        uint8_t* sa = smem + s * kStageBytes;
+        uint8_t* sb = sa + kABytes;
+        dequant_row(brow + ks * 32, bsc + ks * 2, sb, t);
+        if (t < kBM) dequant_row(arow + ks * 32, asc + ks * 2, sa, t);
+        fence_proxy_async_smem();                    // generic writes -> tensor-core reads
+        mbar_arrive(&full[s]);
+      }
+      if (!ok) break;
+    }
+  } else if (warp == kMmaWarp) {
+    if (elect_one()) {
+      constexpr uint32_t idesc = idesc_f16_f32(kBM, kBN);
+      bool ok = true;
+      int it = 0, tcount = 0;
+      for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x, ++tcount) {
+        if (!mbar_wait_bounded(acc_empty, (tcount & 1) ^ 1, max_polls, kDeadlineNs, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        for (int ks = 0; ks < k_steps; ++ks, ++it) {
+          const int s = it % kStages;
+          if (!mbar_wait_bounded(&full[s], (it / kStages) & 1, max_polls, kDeadlineNs, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + s * kStageBytes);
+          const uint32_t sb = sa + kABytes;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            mma_f16(tmem, desc_kmajor_sw128(sa + kk * 32), desc_kmajor_sw128(sb + kk * 32), idesc, (ks | kk) ? 1u : 0u);
+          tc_commit(&empty[s]);
+        }
+        if (!ok) break;
+        tc_commit(acc_full);
+      }
+      if (!ok) give_up();
+    }
+  } else {
+    const int ew = warp - kEpiWarp0, q = warp & 3, half = ew / 4;
+    uint8_t* sbuf = epi_smem + ew * kEpiChunkBytes;
+    int tcount = 0;
+    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++tcount) {
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+      const int m0 = (tile % mt) * kBM, n0 = (tile / mt) * kBN;
+      bool ok = mbar_wait_bounded(acc_full, tcount & 1, max_polls, kDeadlineNs, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) { give_up(); break; }
+      tc_fence_after();
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + half * 128;
+#pragma unroll
+      for (int p = 0; p < 2; ++p) {              // two rounds of 64 columns keep the registers in budget
+        uint32_t r[2][32];
+        tmem_ld_32x32b_x32(tbase + 64 * p, r[0]);
+        tmem_ld_32x32b_x32(tbase + 64 * p + 32, r[1]);
+        tmem_ld_wait();
+        if (p == 1) {
+          tc_fence_before();
+          mbar_arrive(acc_empty);
+        }
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          if (lane == 0) bulk_wait_group_read<0>();
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(sbuf + lane * 128 + ((j ^ (lane & 7)) * 16)) =
+                make_uint4(r[c][4 * j], r[c][4 * j + 1], r[c][4 * j + 2], r[c][4 * j + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmap_y, sbuf, n0 + half * 128 + 64 * p + 32 * c, m0 + q * 32);
+            bulk_commit_group();
+          }
+        }
+      }
+    }
+    if (lane == 0) bulk_wait_group_all();
+  }
+  __syncwarp();
+  if (*abort_flag) {
+    const uint64_t until = globaltimer_ns() + 200000ull;
+    while (globaltimer_ns() < until) __nanosleep(1000);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+}
+
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn get_encode() {
+  static EncodeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(p);
+  });
+  return fn;
+}
+
+}  // namespace
+}  // namespace wush
+
+using namespace wush;
+
+extern "C" int wush_qgemm_int4(const uint8_t* a_codes, const void* a_scales, const uint8_t* b_codes,
+                               const void* b_scales, int64_t M, int64_t N, int64_t K, float* y, void* stream) {
+  if (M <= 0 || N <= 0 || K <= 0 || M % 128 || N % 256 || K % 64) return WUSH_ERR_INVALID_ARG;
+  if (M > (int64_t(1) << 30) || N > (int64_t(1) << 30) || K > (int64_t(1) << 30)) return WUSH_ERR_UNSUPPORTED;
+  if (!a_codes || !a_scales || !b_codes || !b_scales || !y) return WUSH_ERR_INVALID_ARG;
+  if (!aligned16(a_codes) || !aligned16(b_codes) || !aligned16(y) ||
+      (reinterpret_cast<uintptr_t>(a_scales) & 3u) || (reinterpret_cast<uintptr_t>(b_scales) & 3u))
+    return WUSH_ERR_INVALID_ARG;
+  EncodeFn enc = get_encode();
+  if (!enc) return WUSH_ERR_CUDA;
+  CUtensorMap my;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * 4};
+  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  if (enc(&my, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+      CUDA_SUCCESS)
+    return WUSH_ERR_CUDA;
+  static uint64_t attr_done = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return WUSH_ERR_CUDA;
+  if (dev < 64 && !(attr_done >> dev & 1)) {
+    if (cudaFuncSetAttribute(qgemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+        cudaSuccess)
+      return WUSH_ERR_CUDA;
+    attr_done |= uint64_t(1) << dev;
+  }
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+    return WUSH_ERR_CUDA;
+  const int64_t n_tiles = (M / kBM) * (N / kBN);
+  const int grid = static_cast<int>(n_tiles < sms ? n_tiles : sms);
+  const int64_t polls = g_wait_limit_override > 0 ? g_wait_limit_override : kDefaultPolls;
+  qgemm_int4_kernel<<<grid, kThreads, kSmemBytes, static_cast<cudaStream_t>(stream)>>>(
+      a_codes, static_cast<const __half*>(a_scales), b_codes, static_cast<const __half*>(b_scales), my,
+      static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), polls);
+  return launch_status();
+}

@@ -183,6 +183,25 @@ int wush_qgemm(const uint8_t* a_codes, const void* a_scales, const uint8_t* b_co
                float* y, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * INT4 GEMM with per-32-group fp16 scales (device)
+ *
+ * WUSH news article, experiments paragraph (INT4 is the format with the largest
+ * loss reduction).  y[m, n] = sum_g s_a[m, g] s_b[n, g] sum_{k in g} q_a q_b.
+ * B200 tensor cores have no 4-bit integer or per-group-scaled integer MMA, so each
+ * element is dequantised to fp16(q * s) (one rounding, relative error <= 2^-11)
+ * and multiplied with fp16 MMAs accumulating in fp32.
+ *
+ * a_codes/a_scales: INT4 codes and fp16 scales of the activations from
+ *                   wush_transform_quant (rows = M, d_in = K).
+ * b_codes/b_scales: the same for the weights (rows = N).
+ * y:      device fp32 [M, N] row-major, overwritten.
+ * Requirements: M % 128 == 0, N % 256 == 0, K % 64 == 0, all > 0; scales 4-byte
+ * aligned.
+ * ------------------------------------------------------------------------- */
+int wush_qgemm_int4(const uint8_t* a_codes, const void* a_scales, const uint8_t* b_codes,
+                    const void* b_scales, int64_t M, int64_t N, int64_t K, float* y, void* stream);
+
+/* ---------------------------------------------------------------------------
  * ITQ3_S-style 3-bit weights with a 256-wide Walsh-Hadamard rotation
  *
  * ITQ3_S article, "核心技术：FWHT预旋转与TurboQuant的完美融合": each 256-element
