@@ -104,15 +104,25 @@ __device__ __forceinline__ void dequant8(uint32_t w, __half2 s2, uint32_t (&out)
   out[3] = prmt(u[2], u[3], 0x7632);   // e6, e7
 }
 
-// One operand row of a 64-wide k-step: 32 code bytes + the two group scales ->
+// Raw inputs of one operand row for one 64-wide k-step: 32 code bytes and the two
+// group scales.
+struct RawRow {
+  uint4 c0, c1;
+  __half2 sc;
+};
+
+__device__ __forceinline__ RawRow load_row(const uint8_t* __restrict__ codes, const __half* __restrict__ scales) {
+  RawRow r;
+  r.c0 = __ldg(reinterpret_cast<const uint4*>(codes));
+  r.c1 = __ldg(reinterpret_cast<const uint4*>(codes + 16));
+  r.sc = __ldg(reinterpret_cast<const __half2*>(scales));
+  return r;
+}
+
 // 128 bytes of fp16 at row ``r`` of a 128-byte-swizzled tile.
-__device__ __forceinline__ void dequant_row(const uint8_t* __restrict__ codes, const __half* __restrict__ scales,
-                                            uint8_t* tile, int r) {
-  const uint4 c0 = __ldg(reinterpret_cast<const uint4*>(codes));
-  const uint4 c1 = __ldg(reinterpret_cast<const uint4*>(codes + 16));
-  const __half2 sc = __ldg(reinterpret_cast<const __half2*>(scales));
-  const __half2 s0 = __low2half2(sc), s1 = __high2half2(sc);
-  const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+__device__ __forceinline__ void dequant_row(const RawRow& raw, uint8_t* tile, int r) {
+  const __half2 s0 = __low2half2(raw.sc), s1 = __high2half2(raw.sc);
+  const uint32_t w[8] = {raw.c0.x, raw.c0.y, raw.c0.z, raw.c0.w, raw.c1.x, raw.c1.y, raw.c1.z, raw.c1.w};
 #pragma unroll
   for (int j = 0; j < 8; ++j) {           // j: 8 elements = one 16-byte chunk of the fp16 row
     uint32_t o[4];
@@ -164,23 +174,47 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
 
   if (warp < kDqWarps) {
+    // The raw codes and scales of the next k-step are loaded before waiting for
+    // a free stage, so their L2 latency overlaps the wait and the current step.
     const int t = threadIdx.x;                       // B row t of the tile; A row t for t < 128
+    const bool has_a = t < kBM;
     int it = 0;
-    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+    const int first = blockIdx.x;
+    auto row_ptrs = [&](int tile, const uint8_t*& br, const __half*& bs, const uint8_t*& ar, const __half*& as) {
       const int m0 = (tile % mt) * kBM, n0 = (tile / mt) * kBN;
-      const uint8_t* brow = b_codes + static_cast<int64_t>(n0 + t) * row_bytes;
-      const __half* bsc = b_scales + static_cast<int64_t>(n0 + t) * n_groups;
-      const uint8_t* arow = a_codes + static_cast<int64_t>(m0 + (t & 127)) * row_bytes;
-      const __half* asc = a_scales + static_cast<int64_t>(m0 + (t & 127)) * n_groups;
+      br = b_codes + static_cast<int64_t>(n0 + t) * row_bytes;
+      bs = b_scales + static_cast<int64_t>(n0 + t) * n_groups;
+      ar = a_codes + static_cast<int64_t>(m0 + (t & (kBM - 1))) * row_bytes;
+      as = a_scales + static_cast<int64_t>(m0 + (t & (kBM - 1))) * n_groups;
+    };
+    const uint8_t *br, *ar;
+    const __half *bs, *as;
+    RawRow nb{}, na{};
+    if (first < n_tiles) {
+      row_ptrs(first, br, bs, ar, as);
+      nb = load_row(br, bs);
+      if (has_a) na = load_row(ar, as);
+    }
+    for (int tile = first; tile < n_tiles; tile += gridDim.x) {
       bool ok = true;
       for (int ks = 0; ks < k_steps; ++ks, ++it) {
+        const RawRow cb = nb, ca = na;
+        // prefetch the next k-step (of this tile, or the first of the next tile)
+        if (ks + 1 < k_steps) {
+          nb = load_row(br + (ks + 1) * 32, bs + (ks + 1) * 2);
+          if (has_a) na = load_row(ar + (ks + 1) * 32, as + (ks + 1) * 2);
+        } else if (tile + static_cast<int>(gridDim.x) < n_tiles) {
+          row_ptrs(tile + gridDim.x, br, bs, ar, as);
+          nb = load_row(br, bs);
+          if (has_a) na = load_row(ar, as);
+        }
         const int s = it % kStages;
         ok = mbar_wait_bounded(&empty[s], ((it / kStages) & 1) ^ 1, max_polls, kDeadlineNs, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) { give_up(); ok = false; break; }
         uint8_t* sa = smem + s * kStageBytes;
         uint8_t* sb = sa + kABytes;
-        dequant_row(brow + ks * 32, bsc + ks * 2, sb, t);
-        if (t < kBM) dequant_row(arow + ks * 32, asc + ks * 2, sa, t);
+        dequant_row(cb, sb, t);
+        if (has_a) dequant_row(ca, sa, t);
         fence_proxy_async_smem();                    // generic writes -> tensor-core reads
         mbar_arrive(&full[s]);
       }
