@@ -21,11 +21,12 @@ extern "C" const char* wush_status_string(int status) {
 
 extern "C" int wush_check_device_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return WUSH_ERR_CUDA;
-  int word = 0, word_tq = 0, word_i4 = 0;
+  int word = 0, word_tq = 0, word_i4 = 0, word_it = 0;
   if (wush::read_and_clear_error_word(&word) != cudaSuccess) return WUSH_ERR_CUDA;
   if (wush::read_and_clear_tq_error(&word_tq) != cudaSuccess) return WUSH_ERR_CUDA;
   if (wush::read_and_clear_int4_error(&word_i4) != cudaSuccess) return WUSH_ERR_CUDA;
-  return (word | word_tq | word_i4) == 0 ? WUSH_OK : WUSH_ERR_TIMEOUT;
+  if (wush::read_and_clear_itq3_error(&word_it) != cudaSuccess) return WUSH_ERR_CUDA;
+  return (word | word_tq | word_i4 | word_it) == 0 ? WUSH_OK : WUSH_ERR_TIMEOUT;
 }
 
 extern "C" int wush_debug_set_gemm_variant(int variant) {

@@ -19,6 +19,7 @@ int read_and_clear_error_word(int* word);
 // The same for the tensor-core transform+quant kernel's and the INT4 GEMM's words.
 int read_and_clear_tq_error(int* word);
 int read_and_clear_int4_error(int* word);
+int read_and_clear_itq3_error(int* word);
 
 // Tensor-core form of wush_transform_quant (bf16 inputs); WUSH_ERR_UNSUPPORTED
 // for shapes it does not take.

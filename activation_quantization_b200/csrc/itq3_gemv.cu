@@ -21,19 +21,34 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace wush {
+
+static __device__ int g_itq3_error = 0;
+
+int read_and_clear_itq3_error(int* word) {
+  cudaError_t e = cudaMemcpyFromSymbol(word, g_itq3_error, sizeof(int));
+  if (e != cudaSuccess) return e;
+  if (*word) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_itq3_error, &zero, sizeof(int));
+  }
+  return e;
+}
+
 namespace {
 
 constexpr int kWarps = 8;
 
-__device__ __forceinline__ void unpack_levels(const uint32_t* __restrict__ words, int lane, float s,
-                                              float (&v)[8]) {
+// Levels (c - 3.5) s of the eight elements 32 i + lane of one 256-block, from the
+// CTA's shared copy of its 24 code words (all lanes read the same words).
+__device__ __forceinline__ void unpack_levels_smem(const uint32_t* words, int lane, float s, float (&v)[8]) {
   const uint4* w4 = reinterpret_cast<const uint4*>(words);
   uint32_t w[24];
 #pragma unroll
   for (int q = 0; q < 6; ++q) {
-    const uint4 t = __ldg(w4 + q);
+    const uint4 t = w4[q];
     w[4 * q] = t.x; w[4 * q + 1] = t.y; w[4 * q + 2] = t.z; w[4 * q + 3] = t.w;
   }
 #pragma unroll
@@ -67,38 +82,86 @@ __device__ __forceinline__ void warp_fwht256(float (&v)[8], int lane) {
   }
 }
 
-template <int T>
-__global__ void __launch_bounds__(kWarps * 32) itq3_fused_kernel(const uint32_t* __restrict__ codes,
-                                                                  const __half* __restrict__ scales,
-                                                                  const __half* __restrict__ x, int tokens,
-                                                                  int d_out, int d_in, float* __restrict__ y) {
-  const int lane = threadIdx.x & 31;
-  const int o = blockIdx.x * kWarps + (threadIdx.x >> 5);
-  if (o >= d_out) return;
+// One CTA owns kWarps consecutive output rows (one per warp).  Thread 0 fetches
+// the CTA's packed codes and scales (contiguous, kWarps * nb * 96 and
+// kWarps * nb * 2 bytes) with two bulk async copies; meanwhile all threads stage
+// the activations of the current 256-block for every token as fp32 in a double
+// buffer, so each warp reads its x values from shared memory (lane l reads
+// element 32 i + l: no bank conflicts) and its code words as broadcasts.
+// MODE 0: x is fp16 and the inverse FWHT runs on every weight block (the
+// article's fused design).  MODE 1: x is the fp32 rotated activation (H x / 16)
+// and the weights are used as their levels (c - 3.5) s.
+template <int T, int MODE>
+__global__ void __launch_bounds__(kWarps * 32) itq3_gemv_kernel(const uint8_t* __restrict__ codes,
+                                                                const __half* __restrict__ scales,
+                                                                const void* __restrict__ xin, int tokens,
+                                                                int d_out, int d_in, float* __restrict__ y) {
+  extern __shared__ __align__(16) uint8_t itq3_smem[];
   const int nb = d_in / 256;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int o0 = blockIdx.x * kWarps;
+  const int codes_bytes = kWarps * nb * 96;
+  const int scale_bytes = ((kWarps * nb * 2 + 15) / 16) * 16;
+  uint8_t* scodes = itq3_smem;
+  const __half* sscales = reinterpret_cast<const __half*>(itq3_smem + codes_bytes);
+  float* sx = reinterpret_cast<float*>(itq3_smem + codes_bytes + scale_bytes);   // [2][T][256]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sx + 2 * T * 256);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 1);
+
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(bar, 1);
+    *abort_flag = 0;
+    sm100::fence_barrier_init();
+    sm100::mbar_arrive_expect_tx(bar, static_cast<uint32_t>(codes_bytes + kWarps * nb * 2));
+    sm100::bulk_load(scodes, codes + static_cast<int64_t>(o0) * nb * 96, static_cast<uint32_t>(codes_bytes), bar);
+    sm100::bulk_load(itq3_smem + codes_bytes, scales + static_cast<int64_t>(o0) * nb,
+                     static_cast<uint32_t>(kWarps * nb * 2), bar);
+  }
+  auto stage_x = [&](int blk, int buf) {
+    float* dst = sx + buf * T * 256;
+    for (int i = threadIdx.x; i < tokens * 256; i += kWarps * 32) {
+      const int tt = i >> 8, e = i & 255;
+      const int64_t src = static_cast<int64_t>(tt) * d_in + blk * 256 + e;
+      dst[tt * 256 + e] = MODE == 0 ? __half2float(static_cast<const __half*>(xin)[src])
+                                    : static_cast<const float*>(xin)[src];
+    }
+  };
+  stage_x(0, 0);
+  __syncthreads();                                   // barrier initialised, block 0 of x staged
+  const bool have_codes = sm100::mbar_wait_bounded(bar, 0, int64_t(1) << 40, 4000000000ull, abort_flag);
+  if (!have_codes && threadIdx.x == 0) atomicOr(&g_itq3_error, 1 << kErrTimeoutBarrier);
+
   float acc[T];
 #pragma unroll
   for (int t = 0; t < T; ++t) acc[t] = 0.f;
+  const int row = warp;
   for (int blk = 0; blk < nb; ++blk) {
+    if (blk + 1 < nb) stage_x(blk + 1, (blk + 1) & 1);
     float v[8];
-    unpack_levels(codes + (static_cast<int64_t>(o) * nb + blk) * 24, lane,
-                  __half2float(scales[static_cast<int64_t>(o) * nb + blk]), v);
-    warp_fwht256(v, lane);
+    unpack_levels_smem(reinterpret_cast<const uint32_t*>(scodes + (row * nb + blk) * 96), lane,
+                       __half2float(sscales[row * nb + blk]), v);
+    if constexpr (MODE == 0) {
+      warp_fwht256(v, lane);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] *= 0.0625f;
+    }
+    const float* xb = sx + (blk & 1) * T * 256 + lane;
 #pragma unroll
     for (int t = 0; t < T; ++t) {
       if (t >= tokens) break;
-      const __half* xr = x + static_cast<int64_t>(t) * d_in + blk * 256 + lane;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[t] = fmaf(v[i] * 0.0625f, __half2float(xr[32 * i]), acc[t]);
+      for (int i = 0; i < 8; ++i) acc[t] = fmaf(v[i], xb[t * 256 + 32 * i], acc[t]);
     }
+    __syncthreads();                                 // x block blk + 1 staged; block blk no longer read
   }
+  if (!have_codes) return;
 #pragma unroll
   for (int t = 0; t < T; ++t) {
     if (t >= tokens) break;
     float a = acc[t];
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
-    if (lane == 0) y[static_cast<int64_t>(t) * d_out + o] = a;
+    if (lane == 0) y[static_cast<int64_t>(t) * d_out + o0 + row] = a;
   }
 }
 
@@ -120,38 +183,32 @@ __global__ void __launch_bounds__(kWarps * 32) itq3_rotate_x_kernel(const __half
   for (int i = 0; i < 8; ++i) out[32 * i] = v[i] * 0.0625f;
 }
 
-template <int T>
-__global__ void __launch_bounds__(kWarps * 32) itq3_rotated_kernel(const uint32_t* __restrict__ codes,
-                                                                    const __half* __restrict__ scales,
-                                                                    const float* __restrict__ x_rot, int tokens,
-                                                                    int d_out, int d_in, float* __restrict__ y) {
-  const int lane = threadIdx.x & 31;
-  const int o = blockIdx.x * kWarps + (threadIdx.x >> 5);
-  if (o >= d_out) return;
-  const int nb = d_in / 256;
-  float acc[T];
-#pragma unroll
-  for (int t = 0; t < T; ++t) acc[t] = 0.f;
-  for (int blk = 0; blk < nb; ++blk) {
-    float v[8];
-    unpack_levels(codes + (static_cast<int64_t>(o) * nb + blk) * 24, lane,
-                  __half2float(scales[static_cast<int64_t>(o) * nb + blk]), v);
-#pragma unroll
-    for (int t = 0; t < T; ++t) {
-      if (t >= tokens) break;
-      const float* xr = x_rot + static_cast<int64_t>(t) * d_in + blk * 256 + lane;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[t] = fmaf(v[i], __ldg(xr + 32 * i), acc[t]);
-    }
-  }
-#pragma unroll
-  for (int t = 0; t < T; ++t) {
-    if (t >= tokens) break;
-    float a = acc[t];
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
-    if (lane == 0) y[static_cast<int64_t>(t) * d_out + o] = a;
-  }
+size_t itq3_smem_bytes(int tmax, int64_t d_in) {
+  const int64_t nb = d_in / 256;
+  return static_cast<size_t>(kWarps * nb * 96 + ((kWarps * nb * 2 + 15) / 16) * 16 + 2 * tmax * 256 * 4 + 16);
+}
+
+template <int MODE>
+int launch_gemv(const uint32_t* c32, const __half* sc, const void* x, int t, int n, int k, float* y,
+                cudaStream_t st) {
+  const int tmax = t == 1 ? 1 : (t <= 4 ? 4 : 16);
+  const size_t smem = itq3_smem_bytes(tmax, k);
+  if (smem > 200 * 1024) return WUSH_ERR_UNSUPPORTED;
+  const dim3 grid(static_cast<unsigned>(n / kWarps)), block(kWarps * 32);
+  const uint8_t* cb = reinterpret_cast<const uint8_t*>(c32);
+#define WUSH_ITQ3(TT)                                                                                          \
+  do {                                                                                                         \
+    if (smem > 48 * 1024 &&                                                                                    \
+        cudaFuncSetAttribute(itq3_gemv_kernel<TT, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,          \
+                             static_cast<int>(smem)) != cudaSuccess)                                           \
+      return WUSH_ERR_CUDA;                                                                                    \
+    itq3_gemv_kernel<TT, MODE><<<grid, block, smem, st>>>(cb, sc, x, t, n, k, y);                              \
+  } while (0)
+  if (tmax == 1) WUSH_ITQ3(1);
+  else if (tmax == 4) WUSH_ITQ3(4);
+  else WUSH_ITQ3(16);
+#undef WUSH_ITQ3
+  return launch_status();
 }
 
 }  // namespace
@@ -165,26 +222,20 @@ extern "C" int itq3_dequant_gemv(const uint8_t* codes, const void* scales_fp16, 
   if (tokens < 1 || tokens > 16 || d_out <= 0 || d_in <= 0 || d_in % 256 || d_out % 8) return WUSH_ERR_INVALID_ARG;
   if (d_out > (int64_t(1) << 30) || d_in > (int64_t(1) << 30)) return WUSH_ERR_UNSUPPORTED;
   if (mode != 0 && mode != 1) return WUSH_ERR_UNSUPPORTED;
-  if (!codes || !scales_fp16 || !x_fp16 || !y || !aligned16(codes)) return WUSH_ERR_INVALID_ARG;
+  if (!codes || !scales_fp16 || !x_fp16 || !y || !aligned16(codes) || !aligned16(scales_fp16))
+    return WUSH_ERR_INVALID_ARG;
   if (mode == 1 && (!workspace || !aligned16(workspace))) return WUSH_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const auto* c32 = reinterpret_cast<const uint32_t*>(codes);
   const auto* sc = static_cast<const __half*>(scales_fp16);
   const auto* xh = static_cast<const __half*>(x_fp16);
   const int t = static_cast<int>(tokens), n = static_cast<int>(d_out), k = static_cast<int>(d_in);
-  const dim3 grid(static_cast<unsigned>((d_out + kWarps - 1) / kWarps)), block(kWarps * 32);
-  if (mode == 0) {
-    if (t == 1) itq3_fused_kernel<1><<<grid, block, 0, st>>>(c32, sc, xh, t, n, k, y);
-    else if (t <= 4) itq3_fused_kernel<4><<<grid, block, 0, st>>>(c32, sc, xh, t, n, k, y);
-    else itq3_fused_kernel<16><<<grid, block, 0, st>>>(c32, sc, xh, t, n, k, y);
-    return launch_status();
-  }
+  if (mode == 0) return launch_gemv<0>(c32, sc, xh, t, n, k, y, st);
+  const dim3 block(kWarps * 32);
   const int items = t * (k / 256);
   itq3_rotate_x_kernel<<<(items + kWarps - 1) / kWarps, block, 0, st>>>(xh, t, k, workspace);
-  if (t == 1) itq3_rotated_kernel<1><<<grid, block, 0, st>>>(c32, sc, workspace, t, n, k, y);
-  else if (t <= 4) itq3_rotated_kernel<4><<<grid, block, 0, st>>>(c32, sc, workspace, t, n, k, y);
-  else itq3_rotated_kernel<16><<<grid, block, 0, st>>>(c32, sc, workspace, t, n, k, y);
-  return launch_status();
+  if (launch_status() != WUSH_OK) return WUSH_ERR_CUDA;
+  return launch_gemv<1>(c32, sc, workspace, t, n, k, y, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -237,7 +288,8 @@ extern "C" int itq3_dequant_gemv_noalloc(const uint8_t* codes, const void* scale
   if (tokens < 1 || tokens > 16 || d_out <= 0 || d_in <= 0 || d_in % 256 || d_out % 8) return WUSH_ERR_INVALID_ARG;
   if (tokens * d_in > kNoAllocScratchFloats) return WUSH_ERR_BUFFER_TOO_SMALL;
   if (d_out > (int64_t(1) << 30)) return WUSH_ERR_UNSUPPORTED;
-  if (!codes || !scales_fp16 || !x_fp16 || !y || !aligned16(codes)) return WUSH_ERR_INVALID_ARG;
+  if (!codes || !scales_fp16 || !x_fp16 || !y || !aligned16(codes) || !aligned16(scales_fp16))
+    return WUSH_ERR_INVALID_ARG;
   float* scratch = nullptr;
   const int st = scratch_for_current_device(&scratch);
   if (st != WUSH_OK) return st;
@@ -248,11 +300,9 @@ extern "C" int itq3_dequant_gemv_noalloc(const uint8_t* codes, const void* scale
   const auto* sc = static_cast<const __half*>(scales_fp16);
   const auto* xh = static_cast<const __half*>(x_fp16);
   const int t = static_cast<int>(tokens), n = static_cast<int>(d_out), k = static_cast<int>(d_in);
-  const dim3 grid(static_cast<unsigned>((d_out + kWarps - 1) / kWarps)), block(kWarps * 32);
+  const dim3 block(kWarps * 32);
   const int items = t * (k / 256);
   itq3_rotate_x_kernel<<<(items + kWarps - 1) / kWarps, block, 0, s>>>(xh, t, k, scratch);
-  if (t == 1) itq3_rotated_kernel<1><<<grid, block, 0, s>>>(c32, sc, scratch, t, n, k, y);
-  else if (t <= 4) itq3_rotated_kernel<4><<<grid, block, 0, s>>>(c32, sc, scratch, t, n, k, y);
-  else itq3_rotated_kernel<16><<<grid, block, 0, s>>>(c32, sc, scratch, t, n, k, y);
-  return launch_status();
+  if (launch_status() != WUSH_OK) return WUSH_ERR_CUDA;
+  return launch_gemv<1>(c32, sc, scratch, t, n, k, y, s);
 }

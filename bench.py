@@ -137,11 +137,15 @@ def cpu_threads():
 WORKLOADS = {
     "up_proj": dict(fmt="mxfp4", kind="wush"),
     "down_proj": dict(fmt="nvfp4", kind="wush"),
+    "int4": dict(fmt="int4", kind="wush"),
 }
 
 
-def build_inputs(name: str):
+def build_inputs(name: str, tokens=None):
     w = synth.WORKLOADS[name]
+    if tokens:
+        import dataclasses
+        w = dataclasses.replace(w, tokens=tokens)
     x = synth.activations(w)
     wt = synth.weights(w)
     xc = synth.activations(w, calib=True)
@@ -220,7 +224,7 @@ def run_gpu(args, rank, world):
     torch.cuda.set_device(dev)
     spec = WORKLOADS[args.workload]
     fmt, kind = spec["fmt"], spec["kind"]
-    w, x, wt, xc = build_inputs(args.workload)
+    w, x, wt, xc = build_inputs(args.workload, args.tokens)
     M, N, K = w.tokens, w.d_out, w.d_in
     b = w.block
 
@@ -252,8 +256,11 @@ def run_gpu(args, rank, world):
         aq.wush_transform_quant(xs[r], t_x, kind, fmt, acodes[r][0], acodes[r][1], gx, stream=stream)
 
     def gemm(r):
-        aq.wush_qgemm(acodes[r][0], acodes[r][1], wcodes[r][0], wcodes[r][1], M, N, K, fmt, alpha, y,
-                      stream=stream)
+        if fmt == "int4":
+            aq.wush_qgemm_int4(acodes[r][0], acodes[r][1], wcodes[r][0], wcodes[r][1], M, N, K, y, stream=stream)
+        else:
+            aq.wush_qgemm(acodes[r][0], acodes[r][1], wcodes[r][0], wcodes[r][1], M, N, K, fmt, alpha, y,
+                          stream=stream)
 
     # capture each kernel of each rotation as its own CUDA graph
     with torch.cuda.stream(stream):
@@ -324,12 +331,17 @@ def run_gpu(args, rank, world):
     tq_us = 1e3 * float(np.mean(tq_ms))
     gm_us = 1e3 * float(np.mean(gm_ms))
     peaks = load_peaks()
-    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    # the GEMM's own dtype: FP4 for MXFP4/NVFP4, fp16 for the dequantised INT4 path
+    fp4_peak = peaks["bf16_tflops"] * (FP4_OVER_BF16 if fmt != "int4" else 1.0)
     tq_bytes = (M * K * 2 + aq.wush_codes_bytes(M, K, fmt) + aq.wush_scales_bytes(M, K, fmt)
                 + (K // b) * b * b * 4)
+    gemm_kernel = "qgemm_int4_kernel" if fmt == "int4" else "qgemm_kernel"
+    gemm_peak_src = ("bf16 burst x 1 (the INT4 path multiplies fp16)" if fmt == "int4"
+                     else f"bf16 burst x {FP4_OVER_BF16:g} (nominal dense FP4:BF16)")
     gemm_tflops = flops_step / (gm_us * 1e-6) / 1e12
     tq_gbs = tq_bytes / (tq_us * 1e-6) / 1e9
-    qgemm_src = os.path.join(ROOT, "activation_quantization_b200", "csrc", "qgemm.cu")
+    qgemm_src = os.path.join(ROOT, "activation_quantization_b200", "csrc",
+                             "qgemm_int4.cu" if fmt == "int4" else "qgemm.cu")
     tq_src = os.path.join(ROOT, "activation_quantization_b200", "csrc", "transform_quant.cu")
 
     # end to end through the public API: pinned host X -> device, step, y -> pinned host
@@ -360,7 +372,7 @@ def run_gpu(args, rank, world):
 
     result = None
     if rank == 0:
-        traffic = traffic_from_profiles("qgemm_kernel", args.workload, qgemm_src)
+        traffic = traffic_from_profiles(gemm_kernel, args.workload, qgemm_src)
         tq_traffic = traffic_from_profiles("transform_quant_kernel", args.workload, tq_src)
         result = {
             "metric": "transform+quant HBM GB/s; W4A4 block-scaled GEMM TFLOP/s (% of peak)",
@@ -370,15 +382,65 @@ def run_gpu(args, rank, world):
             "config": describe(w, fmt, kind),
             "transform_quant": {"us": tq_us, "GB_s": tq_gbs, "bytes_per_launch": tq_bytes,
                                 "frac_of_hbm": tq_gbs / peaks["hbm_gbs"], "dram_bytes_per_launch": tq_traffic},
-            "qgemm": {"us": gm_us, "TFLOP_s": gemm_tflops, "frac_of_fp4_peak": gemm_tflops / fp4_peak},
-            "roofline": {"kernel": "qgemm_kernel", "bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak,
+            "qgemm": {"us": gm_us, "TFLOP_s": gemm_tflops, "frac_of_peak": gemm_tflops / fp4_peak},
+            "roofline": {"kernel": gemm_kernel, "bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak,
                          "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak, "traffic": traffic,
-                         "peak_source": (f"{peaks['source']} bf16 burst {peaks['bf16_tflops']:.1f} TFLOP/s x "
-                                         f"{FP4_OVER_BF16:g} (nominal dense FP4:BF16)")},
+                         "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']:.1f} TFLOP/s, {gemm_peak_src}"},
             "e2e": e2e, "gpu_launches": 2 * args.steps,
             "clocks": sampler.summary(),
         }
     return result, (w, x, wt, xc, fmt, kind)
+
+
+# --------------------------------------------------------------------------- ITQ3 GEMV
+
+def run_itq3(args):
+    """Times itq3_dequant_gemv (both modes) at 1, 4 and 16 tokens; one JSON line each."""
+    import torch
+    import activation_quantization_b200 as aq
+    dev = torch.device("cuda", 0)
+    w = synth.itq3_weights()
+    d_out, d_in = w.shape
+    codes, scales = aq.itq3_quantize_weights(w.astype(np.float16))
+    copies = 24                                    # 24 x 6.4 MB of weights rotate: more than L2
+    cs = [torch.from_numpy(codes).to(dev) for _ in range(copies)]
+    ss = [torch.from_numpy(scales).to(dev) for _ in range(copies)]
+    peaks = load_peaks()
+    for t in synth.ITQ3_TOKENS:
+        x = torch.from_numpy(synth.itq3_activations(t).astype(np.float16)).to(dev)
+        y = torch.empty((t, d_out), dtype=torch.float32, device=dev)
+        ws = torch.empty((t, d_in), dtype=torch.float32, device=dev)
+        for mode in (0, 1):
+            # one CUDA graph holds a burst of calls over the rotating weight copies,
+            # so the device time is not bounded by the host's launch rate
+            burst = 2 * copies
+            stream = torch.cuda.Stream(device=dev)
+            with torch.cuda.stream(stream):
+                for i in range(3):
+                    aq.itq3_dequant_gemv(cs[i], ss[i], x, d_out, mode, y, ws, stream=stream)
+            stream.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(burst):
+                    aq.itq3_dequant_gemv(cs[i % copies], ss[i % copies], x, d_out, mode, y, ws, stream=stream)
+            reps = max(1, args.steps // burst)
+            with torch.cuda.stream(stream):
+                for _ in range(max(1, args.warmup // burst)):
+                    g.replay()
+            stream.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                for _ in range(reps):
+                    g.replay()
+                e1.record(stream)
+            stream.synchronize()
+            us = e0.elapsed_time(e1) / (reps * burst) * 1e3
+            byts = codes.nbytes + scales.nbytes + t * d_in * 2 + t * d_out * 4
+            print(json.dumps({"workload": f"itq3 W fp16 [{d_out}, {d_in}] 3-bit, {t} tokens",
+                              "mode": "fused inverse FWHT" if mode == 0 else "activation-side rotation",
+                              "us": us, "GB_s": byts / us / 1e3, "frac_of_hbm": byts / us / 1e3 / peaks["hbm_gbs"],
+                              "bytes_per_call": byts}))
 
 
 # --------------------------------------------------------------------------- main
@@ -389,18 +451,22 @@ def main():
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="wush", choices=["wush", "reference"])
-    ap.add_argument("--workload", default="up_proj", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="up_proj", choices=sorted(WORKLOADS) + ["itq3"])
+    ap.add_argument("--tokens", type=int, default=None, help="override the workload's token count")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
+    if args.workload == "itq3":
+        run_itq3(args)
+        return
     spec = WORKLOADS[args.workload]
 
     if args.impl == "reference":
         if rank != 0:
             return
-        w, x, wt, xc = build_inputs(args.workload)
+        w, x, wt, xc = build_inputs(args.workload, args.tokens)
         leg = OracleLeg(w, x, wt, xc, spec["fmt"], spec["kind"])
         step_rows = leg.rows_for(1.5)
         times = []
