@@ -4,13 +4,14 @@
 // ITQ3_S article, section "核心技术：FWHT预旋转与TurboQuant的完美融合": weights are
 // stored as uniform 3-bit codes of their FWHT-rotated 256-element blocks, and
 // the exact inverse transform is applied as the weights are loaded for the
-// matmul.  Here one warp owns one output row; lane l holds elements 32*i + l
-// (i = 0..7) of each 256-block, which is exactly the bit-plane word layout of
-// the packed codes (word p*8 + i, bit l), so every lane unpacks its own eight
-// codes from six broadcast 16-byte loads.
+// matmul.  Here one warp owns one output row; lane l holds elements 8*l .. 8*l + 7
+// of each 256-block, whose codes are the 24 contiguous bits at bit 24*l of the
+// block's packed 96 bytes, so a lane decodes its eight weights with one funnel
+// shift and one bit-field extract and one FMA each, and reads its x values with
+// 16-byte shared loads.
 //
 // mode 0 (the article's design): the 256-point inverse FWHT of each weight
-//   block runs in registers -- index bits 5..7 inside the lane, bits 0..4 across
+//   block runs in registers -- index bits 0..2 inside the lane, bits 3..7 across
 //   lanes with xor-shuffles -- and the restored weights meet x.
 // mode 1 (algebraically identical, cheaper per weight on B200): H/16 is
 //   symmetric and orthogonal, so w_hat . x = ((c - 3.5) s) . (H x / 16).  A
@@ -41,25 +42,23 @@ namespace {
 
 constexpr int kWarps = 8;
 
-// Levels (c - 3.5) s of the eight elements 32 i + lane of one 256-block, from the
-// CTA's shared copy of its 24 code words (all lanes read the same words).
+// Levels (c - 3.5) s of the eight elements 8 lane .. 8 lane + 7 of one 256-block,
+// from the CTA's shared copy of its 24 code words: 3-bit codes packed
+// little-endian, element e at bits 3e .. 3e + 2 of the block.
 __device__ __forceinline__ void unpack_levels_smem(const uint32_t* words, int lane, float s, float (&v)[8]) {
-  const uint4* w4 = reinterpret_cast<const uint4*>(words);
-  uint32_t w[24];
+  const int bit = 24 * lane;
+  const int w0 = bit >> 5;
+  const uint32_t lo = words[w0], hi = words[w0 + 1 < 24 ? w0 + 1 : 23];
+  const uint32_t bits = __funnelshift_r(lo, hi, bit & 31);
+  const float m = -3.5f * s;
 #pragma unroll
-  for (int q = 0; q < 6; ++q) {
-    const uint4 t = w4[q];
-    w[4 * q] = t.x; w[4 * q + 1] = t.y; w[4 * q + 2] = t.z; w[4 * q + 3] = t.w;
-  }
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t c = ((w[i] >> lane) & 1u) | (((w[8 + i] >> lane) & 1u) << 1) | (((w[16 + i] >> lane) & 1u) << 2);
-    v[i] = (static_cast<float>(c) - 3.5f) * s;
-  }
+  for (int i = 0; i < 8; ++i) v[i] = fmaf(static_cast<float>((bits >> (3 * i)) & 7u), s, m);
 }
 
-// In-place unnormalised 256-point FWHT of the warp-distributed vector (element
-// 32*i + lane in v[i]).
+// In-place unnormalised 256-point FWHT of a warp-distributed vector whose index
+// bits are split between the lane (five bits) and the register index (three
+// bits); the butterflies run over all eight bits, so either split gives the
+// Sylvester-ordered H_256 times the vector.
 __device__ __forceinline__ void warp_fwht256(float (&v)[8], int lane) {
 #pragma unroll
   for (int b = 0; b < 5; ++b) {
@@ -86,8 +85,7 @@ __device__ __forceinline__ void warp_fwht256(float (&v)[8], int lane) {
 // the CTA's packed codes and scales (contiguous, kWarps * nb * 96 and
 // kWarps * nb * 2 bytes) with two bulk async copies; meanwhile all threads stage
 // the activations of the current 256-block for every token as fp32 in a double
-// buffer, so each warp reads its x values from shared memory (lane l reads
-// element 32 i + l: no bank conflicts) and its code words as broadcasts.
+// buffer, so each warp reads its x values and code words from shared memory.
 // MODE 0: x is fp16 and the inverse FWHT runs on every weight block (the
 // article's fused design).  MODE 1: x is the fp32 rotated activation (H x / 16)
 // and the weights are used as their levels (c - 3.5) s.
@@ -145,12 +143,16 @@ __global__ void __launch_bounds__(kWarps * 32) itq3_gemv_kernel(const uint8_t* _
 #pragma unroll
       for (int i = 0; i < 8; ++i) v[i] *= 0.0625f;
     }
-    const float* xb = sx + (blk & 1) * T * 256 + lane;
+    const float* xb = sx + (blk & 1) * T * 256 + 8 * lane;
 #pragma unroll
     for (int t = 0; t < T; ++t) {
       if (t >= tokens) break;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[t] = fmaf(v[i], xb[t * 256 + 32 * i], acc[t]);
+      const float4 xa = *reinterpret_cast<const float4*>(xb + t * 256);
+      const float4 xc = *reinterpret_cast<const float4*>(xb + t * 256 + 4);
+      acc[t] = fmaf(v[0], xa.x, acc[t]); acc[t] = fmaf(v[1], xa.y, acc[t]);
+      acc[t] = fmaf(v[2], xa.z, acc[t]); acc[t] = fmaf(v[3], xa.w, acc[t]);
+      acc[t] = fmaf(v[4], xc.x, acc[t]); acc[t] = fmaf(v[5], xc.y, acc[t]);
+      acc[t] = fmaf(v[6], xc.z, acc[t]); acc[t] = fmaf(v[7], xc.w, acc[t]);
     }
     __syncthreads();                                 // x block blk + 1 staged; block blk no longer read
   }

@@ -7,8 +7,8 @@
 // the vector.  Per block (256 consecutive d_in weights of one row), in fp64:
 //   r = H_256 w / 16 (butterflies, exact for fp16 inputs),
 //   s = fp16 RNE(max|r| / 3.5),  c = clamp(rint(r / s + 3.5), 0, 7), c = 0 if s = 0.
-// Codes are packed as three bit planes per 32 elements (see itq3_quantize_weights
-// in wush.h).
+// Codes are packed 3 bits each, little-endian, element e of a block at bits
+// 3e .. 3e + 2 of the block's 96 bytes (see itq3_quantize_weights in wush.h).
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -91,12 +91,15 @@ extern "C" int itq3_quantize_weights(const uint16_t* w_fp16, int64_t d_out, int6
         c[i] = static_cast<uint8_t>(q);
       }
       scales_fp16[o * nb + blk] = sbits;
-      uint32_t words[24];
-      std::memset(words, 0, sizeof(words));
+      uint8_t packed[96];
+      std::memset(packed, 0, sizeof(packed));
       for (int i = 0; i < 256; ++i)
         for (int p = 0; p < 3; ++p)
-          if ((c[i] >> p) & 1) words[p * 8 + i / 32] |= 1u << (i % 32);
-      std::memcpy(codes + (o * nb + blk) * 96, words, sizeof(words));
+          if ((c[i] >> p) & 1) {
+            const int bit = 3 * i + p;
+            packed[bit >> 3] |= static_cast<uint8_t>(1u << (bit & 7));
+          }
+      std::memcpy(codes + (o * nb + blk) * 96, packed, sizeof(packed));
     }
   }
   return status;

@@ -212,9 +212,9 @@ int wush_qgemm_int4(const uint8_t* a_codes, const void* a_scales, const uint8_t*
  *   c = clamp(rint(r / s + 3.5), 0, 7) (c = 0 when s = 0), all in fp64;
  *   dequantised w_hat = H_256 ((c - 3.5) s) / 16.
  * Packed code layout (our own; the article calls its layout "interleaved"
- * without detail): per row and 256-block, 24 little-endian uint32 words; word
- * p*8 + i holds bit p (p = 0, 1, 2) of the codes of elements 32*i .. 32*i + 31,
- * element 32*i + l in bit l.  96 bytes per 256 weights, rows * d_in * 3 / 8 in all.
+ * without detail): per row and 256-block, 96 bytes holding the 256 three-bit
+ * codes packed little-endian, element e at bits 3e .. 3e + 2 (bit b of the block
+ * is bit b % 8 of byte b / 8).  rows * d_in * 3 / 8 bytes in all.
  * ------------------------------------------------------------------------- */
 
 /* Host: w_fp16 host fp16 bits [d_out, d_in]; d_in % 256 == 0;

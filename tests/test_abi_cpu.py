@@ -59,9 +59,8 @@ def test_not_spd_status():
 
 
 def _unpack_itq3(packed, d_out, d_in):
-    words = packed.view(np.uint32).reshape(d_out, d_in // 256, 3, 8)
-    bits = (words[..., None] >> np.arange(32, dtype=np.uint32)) & 1       # [o, blk, p, i, l]
-    c = bits[:, :, 0] | (bits[:, :, 1] << 1) | (bits[:, :, 2] << 2)        # [o, blk, i, l]
+    bits = np.unpackbits(packed.reshape(-1, 96), axis=1, bitorder="little").reshape(-1, 256, 3)
+    c = bits[:, :, 0] | (bits[:, :, 1] << 1) | (bits[:, :, 2] << 2)
     return c.reshape(d_out, d_in).astype(np.uint8)
 
 

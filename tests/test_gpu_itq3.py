@@ -10,13 +10,12 @@ pytestmark = pytest.mark.gpu
 
 
 def pack_codes(c):
-    """Test-side packer restating the header's bit-plane layout."""
+    """Test-side packer restating the header's layout: 3-bit codes, element e of a
+    256-block at bits 3e .. 3e + 2 of the block's 96 little-endian bytes."""
     d_out, d_in = c.shape
-    cb = c.reshape(d_out, d_in // 256, 8, 32).astype(np.uint32)        # [o, blk, i, l]
-    words = np.zeros((d_out, d_in // 256, 3, 8), np.uint32)
-    for p in range(3):
-        words[:, :, p, :] = np.sum(((cb >> p) & 1) << np.arange(32, dtype=np.uint32), axis=3).astype(np.uint32)
-    return words.reshape(-1).view(np.uint8)
+    cb = c.reshape(d_out * d_in // 256, 256).astype(np.uint8)
+    bits = ((cb[:, :, None] >> np.arange(3, dtype=np.uint8)) & 1).reshape(-1, 768)   # bit 3e + p
+    return np.packbits(bits, axis=1, bitorder="little").reshape(-1)
 
 
 @pytest.mark.parametrize("shape", [(256, 1024), (4096, 4096)])
