@@ -59,16 +59,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase with the given parity.  Gives up (returns false)
-// after max_polls polls, after timeout_ns of wall time from the call, or as soon
-// as *abort is set by another role of the CTA.
+// after max_polls polls, after timeout_ns of wall time counted from the 256th
+// poll, or as soon as *abort is set by another role of the CTA.  The timer is
+// read only every 256 polls, so a wait that ends quickly never pays for it.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int64_t max_polls,
                                                   uint64_t timeout_ns, volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t deadline_ns = globaltimer_ns() + timeout_ns;
+  uint64_t deadline_ns = 0;
   for (int64_t i = 1; i < max_polls; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if ((i & 255) == 255 && globaltimer_ns() > deadline_ns) return false;
+    if ((i & 255) == 255) {
+      const uint64_t now = globaltimer_ns();
+      if (deadline_ns == 0) deadline_ns = now + timeout_ns;
+      else if (now > deadline_ns) return false;
+    }
   }
   return false;
 }

@@ -6,22 +6,27 @@
 // GPU implementation).  The format rules are stated in wush.h.
 //
 // A persistent CTA walks a contiguous range of 128-row x 128-column tiles of X in
-// column-major order, with three roles:
+// column-major order (so a CTA meets at most a few columns of T), with three roles:
 //   warp 0     TMA producer: each tile is two 128-byte-swizzled boxes of 64 bf16
-//              columns, landing in a 4-stage shared-memory ring;
-//   warp 1     MMA issuer (WUS/WUSH): for every b-block of the tile, y = x T^T
-//              as kind::f16 MMAs, M = 128 rows, N = b, K = 16 per instruction,
-//              with T split exactly into three bf16 parts (hi + mid + lo = the
-//              fp32 T) and the three products accumulated in fp32 in TMEM; two
-//              accumulators (one per epilogue warpgroup) let the MMAs of later tiles
-//              overlap the epilogues of earlier ones;
-//   warps 2-17 epilogue, four warpgroups each owning every fourth tile: one thread per row reads its b transformed values
-//              straight out of TMEM (tcgen05.ld 32x32b) -- or, for identity and
-//              Hadamard, out of the swizzled shared-memory tile -- and computes
-//              absmax, scale and codes in registers (hardware cvt.rn.satfinite
-//              e2m1x2), storing packed codes and scale words.  The same warps
-//              convert each new column's fp32 T into the bf16 split operand
-//              layout in shared memory, double-buffered.
+//              columns, landing in a 5-stage shared-memory ring;
+//   warp 1     MMA issuer (WUS/WUSH): y = x T^T per b-block as kind::f16 MMAs,
+//              M = 128 rows, K = 16 per instruction.  T is split exactly into three
+//              bf16 parts (hi + mid + lo = the fp32 T).  Per K-step one MMA with
+//              N = 2b multiplies the X slice by [T_hi; T_mid] stacked along N and a
+//              second, N = b, adds x T_lo^T onto the T_hi columns, so X is read
+//              twice rather than three times and two partial products land side
+//              by side in TMEM.  Quarter q (32 columns) of every tile goes to one
+//              of two TMEM slots of warpgroup q, alternating by tile, so the MMAs
+//              of the next tile overlap the epilogue of this one;
+//   warps 2-17 epilogue, four warpgroups, warpgroup q owning quarter q of every
+//              tile: one thread per row reads the partial products of its row out
+//              of TMEM (tcgen05.ld 32x32b) and adds them, y = (hi + lo) + mid --
+//              or, for identity and Hadamard, reads X out of the swizzled
+//              shared-memory tile -- and computes absmax, scale and codes in
+//              registers (hardware cvt.rn.satfinite e2m1x2 / e4m3x2), storing
+//              packed codes and scale bytes.  The same warps convert each new
+//              column's fp32 T into the stacked bf16 operand in shared memory,
+//              double-buffered.
 // Every mbarrier wait is bounded (see sm100.cuh).
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -40,20 +45,25 @@ using namespace sm100;
 
 constexpr int kTileRows = 128;
 constexpr int kTileCols = 128;                       // bf16 elements
+constexpr int kQuarterCols = 32;                     // columns of a tile owned by one epilogue warpgroup
 constexpr int kBoxCols = 64;                         // 128 bytes
-constexpr int kStages = 4;
+constexpr int kStages = 5;
 constexpr int kEpiWarps = 16;
 constexpr int kEpiThreads = kEpiWarps * 32;
-constexpr int kEpiGroups = 4;                        // epilogue warpgroups, one tile each
-constexpr int kAccs = 4;                             // TMEM accumulators (128 columns each)
+constexpr int kEpiGroups = kTileCols / kQuarterCols; // epilogue warpgroups, one quarter each
+constexpr int kSlotCols = 64;                        // TMEM columns of one quarter's partial products
+constexpr int kSets = 2;                             // accumulator sets (whole tiles), double-buffered
+constexpr int kSetCols = kEpiGroups * kSlotCols;     // 256
 constexpr int kThreads = 64 + kEpiThreads;
 constexpr int kStageBytes = kTileRows * kTileCols * 2;  // 32 KB
 constexpr int kBoxBytes = kTileRows * kBoxCols * 2;     // 16 KB
 constexpr int kTBufBytes = 24 * 1024;
-constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemCols = kSets * kSetCols;   // 512
 constexpr int64_t kDefaultPolls = int64_t(1) << 40;
 constexpr uint64_t kDeadlineNs = 4000000000ull;
 constexpr int kSmemBytes = kStages * kStageBytes + 2 * kTBufBytes + 1024 + 256;
+static_assert(kEpiGroups * 4 == kEpiWarps, "four warps per epilogue warpgroup");
+static_assert(kTmemCols == 512, "TMEM allocation is a power of two of at most 512 columns");
 
 enum Kind : int { kIdentity = 0, kHadamard = 1, kDense = 2 };
 enum Fmt : int { kMx = 0, kNv = 1, kI4 = 2 };
@@ -70,19 +80,28 @@ __device__ __forceinline__ int floor_log2(float a) {
   return e ? e - 127 : (31 - __clz(b & 0x7FFFFFu)) - 149;
 }
 
+// UE4M3 scale byte of t >= 0: round to nearest even, saturating at 448 (the
+// hardware conversion with .satfinite; the sign bit of a non-negative input is 0).
 __device__ __forceinline__ uint32_t ue4m3_rne(float t) {
-  if (!(t < 448.0f)) return 126u;
-  if (t == 0.0f) return 0u;
-  int e = floor_log2(t);
-  if (e < -6) return static_cast<uint32_t>(rintf(t * 512.0f));
-  float q = rintf(t * exp2i(3 - e));
-  if (q >= 16.0f) { q = 8.0f; ++e; }
-  return (static_cast<uint32_t>(e + 7) << 3) | (static_cast<uint32_t>(q) - 8u);
+  uint16_t h;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(0.0f), "f"(t));
+  return h & 0xFFu;
 }
 
+// Value of a UE4M3 byte (exact through fp16).
 __device__ __forceinline__ float ue4m3_value(uint32_t c) {
-  const uint32_t e = c >> 3, m = c & 7u;
-  return e == 0 ? static_cast<float>(m) * 0.001953125f : static_cast<float>(8u + m) * exp2i(static_cast<int>(e) - 10);
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>(c)));
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+}
+
+// (a, b) * s as one packed f32x2 multiply, each lane rounded to nearest like FMUL.
+__device__ __forceinline__ void mul2(float a, float b, float s, float& pa, float& pb) {
+  unsigned long long x, y, z;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a), "f"(b));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(y) : "f"(s));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(z) : "l"(x), "l"(y));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(pa), "=f"(pb) : "l"(z));
 }
 
 // Eight values -> eight E2M1 codes, element 0 in the low nibble (RNE, satfinite).
@@ -100,50 +119,67 @@ __device__ __forceinline__ uint32_t e2m1x8(float v0, float v1, float v2, float v
   return out;
 }
 
+// Eight values times s -> eight E2M1 codes, element 0 in the low nibble (RNE, satfinite).
+__device__ __forceinline__ uint32_t e2m1x8_scaled(const float* v, float s) {
+  float p[8];
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) mul2(v[i], v[i + 1], s, p[i], p[i + 1]);
+  return e2m1x8(p[0], p[1], p[2], p[3], p[4], p[5], p[6], p[7]);
+}
+
 __device__ __forceinline__ uint32_t int4_nibble(float v) {
   int q = __float2int_rn(v);
   q = q < -7 ? -7 : (q > 7 ? 7 : q);
   return static_cast<uint32_t>(q) & 0xFu;
 }
 
+// max |y_i| as a pairwise tree (max is exact, so the order is free): depth log2 B
+// instead of a B-long dependent chain.
+template <int B>
+__device__ __forceinline__ float block_amax(const float (&y)[B]) {
+  float m[B / 2];
+#pragma unroll
+  for (int i = 0; i < B / 2; ++i) m[i] = fmaxf(fabsf(y[2 * i]), fabsf(y[2 * i + 1]));
+#pragma unroll
+  for (int w = B / 4; w >= 1; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < w; ++i) m[i] = fmaxf(m[i], m[i + w]);
+  return m[0];
+}
+
 // Quantise one block of B fp32 values held by this thread.  Writes B/8 code
 // words and returns the scale (byte for MXFP4/NVFP4, fp16 bits for INT4).
 template <int B, int FMT>
 __device__ __forceinline__ uint32_t quantize_block(const float (&y)[B], float gscale, float den, uint32_t (&w)[B / 8]) {
-  float amax = 0.f;
-#pragma unroll
-  for (int i = 0; i < B; ++i) amax = fmaxf(amax, fabsf(y[i]));
+  const float amax = block_amax<B>(y);
   if constexpr (FMT == kMx) {
     int e = amax > 0.f ? floor_log2(amax) - 2 : -127;
     e = e < -127 ? -127 : (e > 127 ? 127 : e);
     const float inv = exp2i(-e);
 #pragma unroll
-    for (int q = 0; q < B / 8; ++q)
-      w[q] = amax > 0.f ? e2m1x8(y[8 * q] * inv, y[8 * q + 1] * inv, y[8 * q + 2] * inv, y[8 * q + 3] * inv,
-                                 y[8 * q + 4] * inv, y[8 * q + 5] * inv, y[8 * q + 6] * inv, y[8 * q + 7] * inv)
-                        : 0u;
+    for (int q = 0; q < B / 8; ++q) w[q] = amax > 0.f ? e2m1x8_scaled(y + 8 * q, inv) : 0u;
     return static_cast<uint32_t>(e + 127);
   } else if constexpr (FMT == kNv) {
     const uint32_t sb = ue4m3_rne(__fdiv_rn(amax, den));
     const float d = __fmul_rn(ue4m3_value(sb), gscale);
     const bool live = sb != 0u && amax > 0.f;
-    const float r = live ? __fdiv_rn(1.0f, d) : 0.f;
+    const float r = live ? __frcp_rn(d) : 0.f;
 #pragma unroll
-    for (int q = 0; q < B / 8; ++q)
-      w[q] = live ? e2m1x8(y[8 * q] * r, y[8 * q + 1] * r, y[8 * q + 2] * r, y[8 * q + 3] * r, y[8 * q + 4] * r,
-                           y[8 * q + 5] * r, y[8 * q + 6] * r, y[8 * q + 7] * r)
-                  : 0u;
+    for (int q = 0; q < B / 8; ++q) w[q] = live ? e2m1x8_scaled(y + 8 * q, r) : 0u;
     return sb;
   } else {
     const float pre = fminf(__fdiv_rn(amax, 7.0f), 65504.0f);
     const __half s16 = __float2half_rn(pre);
     const float s = __half2float(s16);
-    const float r = s > 0.f ? __fdiv_rn(1.0f, s) : 0.f;
+    const float r = s > 0.f ? __frcp_rn(s) : 0.f;
 #pragma unroll
     for (int q = 0; q < B / 8; ++q) {
+      float p[8];
+#pragma unroll
+      for (int k = 0; k < 8; k += 2) mul2(y[8 * q + k], y[8 * q + k + 1], r, p[k], p[k + 1]);
       uint32_t acc = 0;
 #pragma unroll
-      for (int k = 0; k < 8; ++k) acc |= int4_nibble(y[8 * q + k] * r) << (4 * k);
+      for (int k = 0; k < 8; ++k) acc |= int4_nibble(p[k]) << (4 * k);
       w[q] = s > 0.f ? acc : 0u;
     }
     return static_cast<uint32_t>(__half_as_ushort(s16));
@@ -169,14 +205,45 @@ __device__ __forceinline__ void fwht_normalized(float (&y)[B]) {
   for (int i = 0; i < B; ++i) y[i] *= s;
 }
 
+// (a0, a1) + (b0, b1) as one packed f32x2 add, each lane rounded to nearest like FADD.
+__device__ __forceinline__ void add2(float& a0, float& a1, float b0, float b1) {
+  unsigned long long x, y, z;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(y) : "f"(b0), "f"(b1));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(z) : "l"(x), "l"(y));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(z));
+}
+
 template <int B>
-__device__ __forceinline__ void tmem_ld_block(uint32_t taddr, float (&y)[B]) {
-  uint32_t r[B];
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[B]) {
   if constexpr (B == 32) tmem_ld_32x32b_x32(taddr, r);
   else tmem_ld_32x32b_x16(taddr, r);
-  tmem_ld_wait();
+}
+
+// Ties loaded registers to the preceding tcgen05.wait::ld: the empty asm statements
+// are ordered after it, so no use of a value is scheduled before the load landed.
+template <int B>
+__device__ __forceinline__ void tmem_tie(uint32_t (&r)[B]) {
 #pragma unroll
-  for (int i = 0; i < B; ++i) y[i] = __uint_as_float(r[i]);
+  for (int i = 0; i < B; ++i) asm volatile("" : "+r"(r[i]));
+}
+
+// y = (hi + lo) + mid for one b-block of this thread's row: the MMAs leave
+// x (T_hi + T_lo)^T in TMEM columns taddr + [0, B) and x T_mid^T in [B, 2B).
+template <int B>
+__device__ __forceinline__ void tmem_sum_parts(uint32_t taddr, float (&y)[B]) {
+  uint32_t a[B], c[B];
+  tmem_ld_cols<B>(taddr, a);
+  tmem_ld_cols<B>(taddr + B, c);
+  tmem_ld_wait();
+  tmem_tie<B>(a);
+  tmem_tie<B>(c);
+#pragma unroll
+  for (int i = 0; i < B; i += 2) {
+    y[i] = __uint_as_float(a[i]);
+    y[i + 1] = __uint_as_float(a[i + 1]);
+    add2(y[i], y[i + 1], __uint_as_float(c[i]), __uint_as_float(c[i + 1]));
+  }
 }
 
 __device__ __forceinline__ uint32_t bf16_bits_rn(float v) {
@@ -203,17 +270,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                  uint8_t* __restrict__ codes, void* __restrict__ scales, float* __restrict__ ydbg, int rows,
                  int d_in, int n_row_tiles, int n_tiles, int64_t max_polls) {
   constexpr int kBlocks = kTileCols / B;           // b-blocks per tile: 4 or 8
+  constexpr int kQBlocks = kQuarterCols / B;       // b-blocks per quarter: 1 or 2
   constexpr int kKSteps = B / 16;                  // K = 16 per MMA
+  constexpr int kN = 2 * B;                        // MMA N: T_hi and T_mid stacked (T_lo adds onto T_hi)
   constexpr int kChunk = B * 32;                   // bytes of one [B n x 16 k] bf16 operand chunk
   constexpr bool kMma = KIND == kDense;
+  static_assert(kQBlocks * kN <= kSlotCols, "a quarter's partial products must fit its TMEM slot");
+  static_assert(kSets * kSetCols <= 512, "TMEM holds 512 columns");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* tbuf = smem + kStages * kStageBytes;
   uint64_t* x_full = reinterpret_cast<uint64_t*>(tbuf + 2 * kTBufBytes);
   uint64_t* x_empty = x_full + kStages;
   uint64_t* acc_full = x_empty + kStages;
-  uint64_t* acc_empty = acc_full + kAccs;
-  uint64_t* t_full = acc_empty + kAccs;
+  uint64_t* acc_empty = acc_full + kSets;
+  uint64_t* t_full = acc_empty + kSets;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(t_full + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -223,19 +294,54 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tile_hi = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * n_tiles / gridDim.x);
   const int col_lo = tile_lo / n_row_tiles;
 
+  // Every ring and slot below has consumers that each take its phases in order,
+  // so the parity waits are unambiguous for any ring depth: the MMA warp (or all
+  // sixteen epilogue warps) for the X stages, all epilogue warps for the two TMEM
+  // accumulator sets (even and odd tiles).  Epilogue warps poll with lane 0 and
+  // release with one arrival per warp.
+  const int n_mine = tile_hi - tile_lo;
+  const int n_cols = n_mine > 0 ? (tile_hi - 1) / n_row_tiles - col_lo + 1 : 0;
+  // The epilogue threads fetch the fp32 T of this CTA's first two columns before
+  // anything else, so those reads do not queue behind the X tiles in DRAM.
+  constexpr int kTGroups = kBlocks * B * B / 4;    // float4 groups of T per column
+  constexpr int kTPer = kTGroups / kEpiThreads;    // per epilogue thread: 2 or 1
+  static_assert(kTPer * kEpiThreads == kTGroups, "T column splits evenly over the epilogue threads");
+  float4 t_pre[2][kTPer];
+  if (kMma && threadIdx.x >= 64) {
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+#pragma unroll
+      for (int p = 0; p < kTPer; ++p) {
+        const int e0 = 4 * (static_cast<int>(threadIdx.x) - 64 + p * kEpiThreads);
+        const int j = (col_lo + c) * kBlocks + e0 / (B * B);
+        t_pre[c][p] = (c < n_cols && j < nb)
+                          ? __ldg(reinterpret_cast<const float4*>(t + static_cast<int64_t>(j) * B * B + e0 % (B * B)))
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+  }
+  auto issue_load = [&](int n) {
+    const int i = tile_lo + n, s = n % kStages;
+    const int row0 = (i % n_row_tiles) * kTileRows, col0 = (i / n_row_tiles) * kTileCols;
+    uint8_t* st = smem + s * kStageBytes;
+    mbar_arrive_expect_tx(&x_full[s], kStageBytes);
+    tma_load_2d(st, &tmap_x, col0, row0, &x_full[s]);
+    tma_load_2d(st + kBoxBytes, &tmap_x, col0 + kBoxCols, row0, &x_full[s]);
+  };
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&x_full[s], 1);
-      mbar_init(&x_empty[s], kMma ? 1 : 128);
+      mbar_init(&x_empty[s], kMma ? 1 : kEpiWarps);
     }
-    for (int a = 0; a < kAccs; ++a) {
-      mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 128);
+    for (int p = 0; p < kSets; ++p) {
+      mbar_init(&acc_full[p], 1);
+      mbar_init(&acc_empty[p], kEpiWarps);
     }
     for (int b = 0; b < 2; ++b) mbar_init(&t_full[b], 1);
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tmap(&tmap_x);
+    // the ring starts empty: the first loads go out before the rest of the setup
+    for (int n = 0; n < kStages && n < n_mine; ++n) issue_load(n);
   }
   if (warp == 1 && kMma) tmem_alloc(tmem_slot, kTmemCols);
   tc_fence_before();
@@ -251,105 +357,114 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
 
   if (warp == 0) {
-    if (elect_one()) {
-      for (int i = tile_lo; i < tile_hi; ++i) {
-        const int n = i - tile_lo, s = n % kStages;
-        if (!mbar_wait_bounded(&x_empty[s], ((n / kStages) & 1) ^ 1, max_polls, kDeadlineNs, abort_flag)) {
+    if (threadIdx.x == 0) {
+      for (int n = kStages; n < n_mine; ++n) {
+        if (!mbar_wait_bounded(&x_empty[n % kStages], ((n / kStages) & 1) ^ 1, max_polls, kDeadlineNs, abort_flag)) {
           give_up();
           break;
         }
-        const int row0 = (i % n_row_tiles) * kTileRows, col0 = (i / n_row_tiles) * kTileCols;
-        uint8_t* st = smem + s * kStageBytes;
-        mbar_arrive_expect_tx(&x_full[s], kStageBytes);
-        tma_load_2d(st, &tmap_x, col0, row0, &x_full[s]);
-        tma_load_2d(st + kBoxBytes, &tmap_x, col0 + kBoxCols, row0, &x_full[s]);
+        issue_load(n);
       }
     }
   } else if (warp == 1) {
     if (kMma && elect_one()) {
-      constexpr uint32_t idesc = idesc_bf16_f32(kTileRows, B);
-      for (int i = tile_lo; i < tile_hi; ++i) {
-        const int n = i - tile_lo, s = n % kStages, a = n % kAccs;
-        const int k = i / n_row_tiles - col_lo;     // column ordinal within this CTA
-        if (!mbar_wait_bounded(&t_full[k & 1], (k >> 1) & 1, max_polls, kDeadlineNs, abort_flag) ||
-            !mbar_wait_bounded(&acc_empty[a], ((n / kAccs) & 1) ^ 1, max_polls, kDeadlineNs, abort_flag) ||
-            !mbar_wait_bounded(&x_full[s], (n / kStages) & 1, max_polls, kDeadlineNs, abort_flag)) {
-          give_up();
+      // Tile n goes to accumulator set n & 1; quarter q of it to columns
+      // 256 (n & 1) + 64 q.  Per b-block and K-step two MMAs read the same X slice:
+      // N = 2b against [T_hi; T_mid], then N = b against T_lo, accumulating onto
+      // the T_hi columns.  Descriptors are a per-tile base plus constant offsets.
+      constexpr uint32_t idesc2 = idesc_bf16_f32(kTileRows, kN);
+      constexpr uint32_t idesc1 = idesc_bf16_f32(kTileRows, B);
+      bool ok = true;
+      int col = col_lo, row_tile = tile_lo % n_row_tiles, k_ready = -1;
+      for (int n = 0; n < n_mine; ++n) {
+        const int s = n % kStages, p = n & 1, k = col - col_lo;
+        if (k != k_ready) {
+          if (!mbar_wait_bounded(&t_full[k & 1], (k >> 1) & 1, max_polls, kDeadlineNs, abort_flag)) { ok = false; break; }
+          k_ready = k;
+        }
+        if (!mbar_wait_bounded(&x_full[s], (n / kStages) & 1, max_polls, kDeadlineNs, abort_flag) ||
+            !mbar_wait_bounded(&acc_empty[p], ((n >> 1) & 1) ^ 1, max_polls, kDeadlineNs, abort_flag)) {
+          ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t sx = smem_u32(smem + s * kStageBytes);
-        const uint32_t st_ = smem_u32(tbuf + (k & 1) * kTBufBytes);
-        const uint32_t d0 = tmem + a * kTileCols;
+        const uint64_t a0 = desc_kmajor_sw128(smem_u32(smem + s * kStageBytes));
+        const uint64_t b0 = smem_desc(smem_u32(tbuf + (k & 1) * kTBufBytes), 128, 256, kLayoutNone);
+        const uint32_t d0 = tmem + p * kSetCols;
 #pragma unroll
         for (int jj = 0; jj < kBlocks; ++jj) {
-          const int col_bytes = jj * B * 2;                      // byte column of the block in the tile
-          const uint32_t abase = sx + (col_bytes / 128) * kBoxBytes + (col_bytes % 128);
+          const int col_bytes = jj * B * 2;                      // b-block jj within the tile
+          const uint32_t a_off = (col_bytes / 128) * kBoxBytes + (col_bytes % 128);
+          const uint32_t d = d0 + (jj / kQBlocks) * kSlotCols + (jj % kQBlocks) * kN;
 #pragma unroll
-          for (int sp = 0; sp < 3; ++sp) {
-#pragma unroll
-            for (int kk = 0; kk < kKSteps; ++kk) {
-              const uint64_t ad = desc_kmajor_sw128(abase + kk * 32);
-              const uint64_t bd = smem_desc(st_ + ((jj * 3 + sp) * kKSteps + kk) * kChunk, 128, 256, kLayoutNone);
-              mma_bf16(d0 + jj * B, ad, bd, idesc, (sp | kk) ? 1u : 0u);
-            }
+          for (int kk = 0; kk < kKSteps; ++kk) {
+            const uint64_t ad = a0 + ((a_off + kk * 32) >> 4);
+            const uint32_t b_off = (jj * kKSteps + kk) * 3 * kChunk;
+            mma_bf16(d, ad, b0 + (b_off >> 4), idesc2, kk ? 1u : 0u);
+            mma_bf16(d, ad, b0 + ((b_off + 2 * kChunk) >> 4), idesc1, 1u);
           }
         }
+        tc_commit(&acc_full[p]);
         tc_commit(&x_empty[s]);
-        tc_commit(&acc_full[a]);
+        if (++row_tile == n_row_tiles) { row_tile = 0; ++col; }
       }
+      if (!ok) give_up();
     }
   } else {
     // ---------------------------------------------------------------- epilogue
-    // Four warpgroups of 4 warps.  Warpgroup g takes tiles n = g, g+4, ... of the
-    // CTA's range, so four tiles are in flight at once; inside a warpgroup, warp w
-    // may read only TMEM lane quarter w % 4, i.e. rows 32*(w % 4) .. +31, and each
-    // thread handles all b-blocks of one row of the tile.
+    // Four warpgroups of 4 warps; warpgroup g owns columns [32 g, 32 g + 32) of
+    // every tile (TMEM columns 64 g .. of the tile's accumulator set).  Warp w may read only TMEM lane quarter w % 4, i.e.
+    // rows 32 (w % 4) .. + 31, and each thread handles one row of the quarter.
     const int et = threadIdx.x - 64;            // 0..511
-    const int g = et / 128;                     // warpgroup
+    const int g = et / 128;                     // warpgroup = quarter
     const int q = warp & 3;
     const int rloc = q * 32 + lane;             // row within the tile
     const float den = 6.0f * gscale;
-    const int n_cols = tile_hi > tile_lo ? (tile_hi - 1) / n_row_tiles - col_lo + 1 : 0;
+    const int n_atom_cols = (nb + 3) / 4;
 
-    // fp32 T of column col_lo + k -> the three bf16 split operands in buffer k & 1,
-    // by nthr threads (id tid); all float4 loads of a thread are issued first.
+    // Four fp32 values of T (group gi of a column: block jj, output row nrow,
+    // inputs kcol .. kcol + 3) -> the three bf16 parts in T buffer dst.  Chunk
+    // (block jj, K-step kk) holds the parts hi, mid, lo one after another, i.e. a
+    // [3b n x 16 k] K-major operand whose row n = part * b + output index.
+    auto t_store_group = [&](uint8_t* dst, int gi, float4 v) {
+      const int e0 = 4 * gi;
+      const int jj = e0 / (B * B), nrow = (e0 / B) % B, kcol = e0 % B;
+      const int kk = kcol / 16, kin = kcol % 16;
+      const int off = (nrow / 8) * 256 + (kin / 8) * 128 + (nrow % 8) * 16 + (kin % 8) * 2;
+      const float x4[4] = {v.x, v.y, v.z, v.w};
+      uint32_t h[3][4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        h[0][c] = bf16_bits_rn(x4[c]);
+        const float r1 = x4[c] - __uint_as_float(h[0][c] << 16);
+        h[1][c] = bf16_bits_rn(r1);
+        const float r2 = r1 - __uint_as_float(h[1][c] << 16);
+        h[2][c] = bf16_bits_rn(r2);
+      }
+#pragma unroll
+      for (int sp = 0; sp < 3; ++sp)
+        *reinterpret_cast<uint2*>(dst + ((jj * kKSteps + kk) * 3 + sp) * kChunk + off) =
+            make_uint2(h[sp][0] | (h[sp][1] << 16), h[sp][2] | (h[sp][3] << 16));
+    };
+    // fp32 T of column col_lo + k -> buffer k & 1, by nthr threads (id tid); all
+    // float4 loads of a thread are issued first.
     auto convert_t = [&](int k, int tid, int nthr, int bar_id) {
-      constexpr int kGroups = kBlocks * B * B / 4;
       uint8_t* dst = tbuf + (k & 1) * kTBufBytes;
       const int j0 = (col_lo + k) * kBlocks;
-      for (int base = 0; base < kGroups; base += 8 * nthr) {
+      for (int base = 0; base < kTGroups; base += 8 * nthr) {
         float4 v[8];
 #pragma unroll
         for (int p = 0; p < 8; ++p) {
           const int gi = base + tid + p * nthr;
           const int e0 = 4 * gi;
-          v[p] = (gi < kGroups && j0 + e0 / (B * B) < nb)
+          v[p] = (gi < kTGroups && j0 + e0 / (B * B) < nb)
                      ? __ldg(reinterpret_cast<const float4*>(t + static_cast<int64_t>(j0) * B * B + e0))
                      : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
         for (int p = 0; p < 8; ++p) {
           const int gi = base + tid + p * nthr;
-          if (gi >= kGroups) continue;
-          const int e0 = 4 * gi;
-          const int jj = e0 / (B * B), nrow = (e0 / B) % B, kcol = e0 % B;
-          const int kk = kcol / 16, kin = kcol % 16;
-          const int off = (nrow / 8) * 256 + (kin / 8) * 128 + (nrow % 8) * 16 + (kin % 8) * 2;
-          const float x4[4] = {v[p].x, v[p].y, v[p].z, v[p].w};
-          uint32_t h[3][4];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            h[0][c] = bf16_bits_rn(x4[c]);
-            const float r1 = x4[c] - __uint_as_float(h[0][c] << 16);
-            h[1][c] = bf16_bits_rn(r1);
-            const float r2 = r1 - __uint_as_float(h[1][c] << 16);
-            h[2][c] = bf16_bits_rn(r2);
-          }
-#pragma unroll
-          for (int sp = 0; sp < 3; ++sp)
-            *reinterpret_cast<uint2*>(dst + ((jj * 3 + sp) * kKSteps + kk) * kChunk + off) =
-                make_uint2(h[sp][0] | (h[sp][1] << 16), h[sp][2] | (h[sp][3] << 16));
+          if (gi < kTGroups) t_store_group(dst, gi, v[p]);
         }
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -357,96 +472,112 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tid == 0) mbar_arrive(&t_full[k & 1]);
     };
     if constexpr (kMma) {
-      if (n_cols > 0) convert_t(0, et, kEpiThreads, 1);
-      if (n_cols > 1) convert_t(1, et, kEpiThreads, 1);
+      // columns 0 and 1 from the values fetched at kernel entry
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int p = 0; p < kTPer; ++p) t_store_group(tbuf + c * kTBufBytes, et + p * kEpiThreads, t_pre[c][p]);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      asm volatile("bar.sync %0, %1;" ::"r"(1), "r"(kEpiThreads) : "memory");
+      if (et == 0) {
+        mbar_arrive(&t_full[0]);
+        mbar_arrive(&t_full[1]);
+      }
     }
 
-    for (int i = tile_lo + g; i < tile_hi; i += kEpiGroups) {
+    for (int i = tile_lo; i < tile_hi; ++i) {
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-      const int n = i - tile_lo, s = n % kStages, a = n % kAccs;
+      const int n = i - tile_lo, s = n % kStages;
       const int row0 = (i % n_row_tiles) * kTileRows, col0 = (i / n_row_tiles) * kTileCols;
       const int r = row0 + rloc;
       const bool row_ok = r < rows;
-      bool ok;
-      if constexpr (kMma) ok = mbar_wait_bounded(&acc_full[a], (n / kAccs) & 1, max_polls, kDeadlineNs, abort_flag);
-      else ok = mbar_wait_bounded(&x_full[s], (n / kStages) & 1, max_polls, kDeadlineNs, abort_flag);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) { give_up(); break; }
-      if constexpr (kMma) tc_fence_after();
-      const uint8_t* sx = smem + s * kStageBytes;
-      uint32_t sc_words[kBlocks / 4];
+      const int p = n & 1;
+      uint64_t* full = kMma ? &acc_full[p] : &x_full[s];
+      const uint32_t parity = kMma ? (n >> 1) & 1 : (n / kStages) & 1;
+      // lane 0 polls; once it has seen the phase complete, every lane's own
+      // try_wait succeeds at once and gives that lane its acquire
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait_bounded(full, parity, max_polls, kDeadlineNs, abort_flag);
+      __syncwarp();
+      if (!__shfl_sync(0xffffffffu, ok, 0)) { give_up(); break; }
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(full, parity, max_polls, kDeadlineNs, abort_flag))) {
+        give_up();
+        break;
+      }
+
+      float y[kQBlocks][B];
+      if constexpr (kMma) {
+        tc_fence_after();
+        const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + p * kSetCols + g * kSlotCols;
 #pragma unroll
-      for (int w4 = 0; w4 < kBlocks / 4; ++w4) sc_words[w4] = 0u;
+        for (int u = 0; u < kQBlocks; ++u) tmem_sum_parts<B>(taddr + u * kN, y[u]);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[p]);
+      } else {
+        const uint8_t* sx = smem + s * kStageBytes;
 #pragma unroll
-      for (int jj = 0; jj < kBlocks; ++jj) {
-        float y[B];
-        if constexpr (kMma) {
-          tmem_ld_block<B>(tmem + (static_cast<uint32_t>(q * 32) << 16) + a * kTileCols + jj * B, y);
-        } else {
-          const int col_bytes = jj * B * 2;
+        for (int u = 0; u < kQBlocks; ++u) {
+          const int col_bytes = (g * kQBlocks + u) * B * 2;
           const uint8_t* rowp = sx + (col_bytes / 128) * kBoxBytes + rloc * 128;
 #pragma unroll
           for (int c = 0; c < B / 8; ++c) {
             const int chunk = (col_bytes % 128) / 16 + c;
             const uint4 v = *reinterpret_cast<const uint4*>(rowp + ((chunk ^ (rloc & 7)) * 16));
-            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+            const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
-              y[8 * c + 2 * h] = bf16_lo(u[h]);
-              y[8 * c + 2 * h + 1] = bf16_hi(u[h]);
+              y[u][8 * c + 2 * h] = bf16_lo(wd[h]);
+              y[u][8 * c + 2 * h + 1] = bf16_hi(wd[h]);
             }
           }
-          if constexpr (KIND == kHadamard) fwht_normalized<B>(y);
+          if constexpr (KIND == kHadamard) fwht_normalized<B>(y[u]);
         }
-        if (jj == kBlocks - 1) {                  // the tile's values are all out of TMEM / smem
-          if constexpr (kMma) {
-            tc_fence_before();
-            mbar_arrive(&acc_empty[a]);
-          } else {
-            mbar_arrive(&x_empty[s]);
-          }
-        }
-        const int j = col0 / B + jj;
+        // The next writer of this stage is the TMA engine (async proxy): order
+        // this thread's shared-memory reads of it before that write.
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&x_empty[s]);
+      }
+
+#pragma unroll
+      for (int u = 0; u < kQBlocks; ++u) {
+        const int j = col0 / B + g * kQBlocks + u;
         const bool blk_ok = row_ok && j < nb;
         if constexpr (DBG) {
           if (blk_ok) {
-            float4* dp = reinterpret_cast<float4*>(ydbg + static_cast<int64_t>(r) * d_in + static_cast<int64_t>(j) * B);
+            float4* dp =
+                reinterpret_cast<float4*>(ydbg + static_cast<int64_t>(r) * d_in + static_cast<int64_t>(j) * B);
 #pragma unroll
-            for (int w = 0; w < B / 4; ++w) dp[w] = make_float4(y[4 * w], y[4 * w + 1], y[4 * w + 2], y[4 * w + 3]);
+            for (int w = 0; w < B / 4; ++w)
+              dp[w] = make_float4(y[u][4 * w], y[u][4 * w + 1], y[u][4 * w + 2], y[u][4 * w + 3]);
           }
         }
         uint32_t cw[B / 8];
-        const uint32_t sc = quantize_block<B, FMT>(y, gscale, den, cw);
+        const uint32_t sc = quantize_block<B, FMT>(y[u], gscale, den, cw);
         if (blk_ok) {
           uint8_t* cp = codes + static_cast<int64_t>(r) * (d_in / 2) + static_cast<int64_t>(j) * (B / 2);
           if constexpr (B == 32) *reinterpret_cast<uint4*>(cp) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
           else *reinterpret_cast<uint2*>(cp) = make_uint2(cw[0], cw[1]);
         }
         if constexpr (FMT == kI4) {
-          if (blk_ok) reinterpret_cast<uint16_t*>(scales)[static_cast<int64_t>(r) * nb + j] = static_cast<uint16_t>(sc);
-        } else {
-          sc_words[jj / 4] |= (blk_ok ? sc : 0u) << (8 * (jj % 4));
+          if (blk_ok)
+            reinterpret_cast<uint16_t*>(scales)[static_cast<int64_t>(r) * nb + j] = static_cast<uint16_t>(sc);
+        } else if (j < n_atom_cols * 4) {
+          // padding rows and columns of an existing atom are written as zero
+          static_cast<uint8_t*>(scales)[sf_offset(r, j, n_atom_cols)] = static_cast<uint8_t>(blk_ok ? sc : 0u);
         }
       }
-      if constexpr (FMT != kI4) {
-        // this thread's 4 scale bytes of each 4-column atom form one aligned word
-        const int n_atom_cols = (nb + 3) / 4;
-#pragma unroll
-        for (int w4 = 0; w4 < kBlocks / 4; ++w4) {
-          const int atom_col = col0 / B / 4 + w4;
-          if (atom_col < n_atom_cols) {
-            const int64_t off = (static_cast<int64_t>(row0 / 128) * n_atom_cols + atom_col) * 512 +
-                                (rloc & 31) * 16 + (rloc >> 5) * 4;
-            *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(scales) + off) = sc_words[w4];
-          }
-        }
-      }
+
       if constexpr (kMma) {
-        // The warpgroup that finishes the last tile of column k refills that
-        // column's T buffer with column k + 2: every MMA reading it has completed.
-        const int k = i / n_row_tiles - col_lo;
-        const bool last_of_col = (i + 1 == tile_hi) || ((i + 1) / n_row_tiles != i / n_row_tiles);
-        if (last_of_col && k + 2 < n_cols) convert_t(k + 2, et - g * 128, 128, 2 + g);
+        // Warpgroup kEpiGroups - 1 sees its slot's commit last in each tile, and a
+        // commit covers every MMA issued before it: after the last tile of column k,
+        // no MMA reads that column's T buffer any more, so it refills it with k + 2.
+        if (g == kEpiGroups - 1) {
+          const int k = i / n_row_tiles - col_lo;
+          const bool last_of_col = (i + 1 == tile_hi) || ((i + 1) / n_row_tiles != i / n_row_tiles);
+          if (last_of_col && k + 2 < n_cols) convert_t(k + 2, et - g * 128, 128, 2 + g);
+        }
       }
     }
   }
