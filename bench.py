@@ -36,6 +36,7 @@ import synth  # noqa: E402
 
 L2_BYTES = 126 * 2 ** 20
 ROTATIONS = 3
+STEPS_PER_GRAPH = 12            # steps captured per CUDA graph (four passes over the rotations)
 FP4_OVER_BF16 = 4.0          # nominal dense FP4 : BF16 tensor ratio (9 : 2.25 PFLOP/s)
 
 
@@ -51,12 +52,21 @@ def load_peaks():
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
 
 
+def source_sha(source_file: str) -> str:
+    """Hash of a kernel's source file together with the device headers it includes."""
+    csrc = os.path.dirname(source_file)
+    h = hashlib.sha1()
+    for f in [source_file] + [os.path.join(csrc, n) for n in ("sm100.cuh", "common.cuh")]:
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:12]
+
+
 def traffic_from_profiles(kernel: str, workload: str, source_file: str):
     """DRAM bytes per launch recorded by an ncu capture, if the kernel source is unchanged."""
     path = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(path):
         return None
-    sha = hashlib.sha1(open(source_file, "rb").read()).hexdigest()[:12]
+    sha = source_sha(source_file)
     for line in open(path):
         f = dict(kv.split("=", 1) for kv in line.split() if "=" in kv)
         if f.get("kernel") == kernel and f.get("workload") == workload and f.get("src_sha") == sha:
@@ -262,21 +272,33 @@ def run_gpu(args, rank, world):
             aq.wush_qgemm(acodes[r][0], acodes[r][1], wcodes[r][0], wcodes[r][1], M, N, K, fmt, alpha, y,
                           stream=stream)
 
-    # capture each kernel of each rotation as its own CUDA graph
+    # The timed steps run as CUDA graphs of STEPS_PER_GRAPH consecutive steps
+    # (rotating through the input copies), with event nodes between the kernels so
+    # that each kernel's device time is read without the graph-launch latency.
     with torch.cuda.stream(stream):
         for r in range(ROTATIONS):
             tq(r)
             gemm(r)
     stream.synchronize()
-    graphs_tq, graphs_gemm = [], []
-    for r in range(ROTATIONS):
-        g1, g2 = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g1, stream=stream):
-            tq(r)
-        with torch.cuda.graph(g2, stream=stream):
-            gemm(r)
-        graphs_tq.append(g1)
-        graphs_gemm.append(g2)
+
+    def capture(n_steps, start=0):
+        g = torch.cuda.CUDAGraph()
+        evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(n_steps)]
+        with torch.cuda.graph(g, stream=stream):
+            for j in range(n_steps):
+                r = (start + j) % ROTATIONS
+                evs[j][0].record(stream)
+                tq(r)
+                evs[j][1].record(stream)
+                gemm(r)
+                evs[j][2].record(stream)
+        return g, evs
+
+    g_main, ev_main = capture(STEPS_PER_GRAPH)
+    n_rem = args.steps % STEPS_PER_GRAPH
+    g_rem, ev_rem = capture(n_rem) if n_rem else (None, [])
+    # a graph's event nodes refer to its Event objects: keep every (graph, events) pair alive
+    g_one = [capture(1, r) for r in range(ROTATIONS)]
     if aq.wush_check_device_status(stream) != 0:
         raise RuntimeError("device status after capture")
 
@@ -286,28 +308,28 @@ def run_gpu(args, rank, world):
             dist.barrier()
 
     def timed(steps):
-        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier()
         torch.cuda.synchronize()
         with torch.cuda.stream(stream):
-            for i in range(steps):
-                r = i % ROTATIONS
-                ev[i][0].record(stream)
-                graphs_tq[r].replay()
-                ev[i][1].record(stream)
-                graphs_gemm[r].replay()
-                ev[i][2].record(stream)
+            e_start.record(stream)
+            for _ in range(steps // STEPS_PER_GRAPH):
+                g_main.replay()
+            if g_rem is not None:
+                g_rem.replay()
+            e_end.record(stream)
         torch.cuda.synchronize()
         barrier()
-        total_ms = ev[0][0].elapsed_time(ev[-1][2])
-        tq_ms = [e[0].elapsed_time(e[1]) for e in ev]
-        gm_ms = [e[1].elapsed_time(e[2]) for e in ev]
+        total_ms = e_start.elapsed_time(e_end)
+        # per-kernel device times from the event nodes of the last replay
+        evs = ev_main if steps >= STEPS_PER_GRAPH else ev_rem
+        tq_ms = [e[0].elapsed_time(e[1]) for e in evs]
+        gm_ms = [e[1].elapsed_time(e[2]) for e in evs]
         return total_ms, tq_ms, gm_ms
 
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
-            graphs_tq[i % ROTATIONS].replay()
-            graphs_gemm[i % ROTATIONS].replay()
+            g_one[i % ROTATIONS][0].replay()
     stream.synchronize()
 
     for attempt in range(2):
@@ -319,6 +341,22 @@ def run_gpu(args, rank, world):
     status = aq.wush_check_device_status(stream)
     if status != 0:
         raise RuntimeError(f"device status {status}")
+
+    # The transform alone, as a burst of back-to-back launches over the rotating
+    # inputs: inside a step it also absorbs the write-back of the GEMM's y from L2.
+    g_tq = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_tq, stream=stream):
+        for j in range(STEPS_PER_GRAPH):
+            tq(j % ROTATIONS)
+    with torch.cuda.stream(stream):
+        g_tq.replay()
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        b0.record(stream)
+        for _ in range(8):
+            g_tq.replay()
+        b1.record(stream)
+    torch.cuda.synchronize()
+    tq_burst_us = 1e3 * b0.elapsed_time(b1) / (8 * STEPS_PER_GRAPH)
 
     if world > 1:
         import torch.distributed as dist
@@ -335,14 +373,15 @@ def run_gpu(args, rank, world):
     fp4_peak = peaks["bf16_tflops"] * (FP4_OVER_BF16 if fmt != "int4" else 1.0)
     tq_bytes = (M * K * 2 + aq.wush_codes_bytes(M, K, fmt) + aq.wush_scales_bytes(M, K, fmt)
                 + (K // b) * b * b * 4)
-    gemm_kernel = "qgemm_int4_kernel" if fmt == "int4" else "qgemm_kernel"
+    gemm_kernel = ("qgemm_int4_kernel" if fmt == "int4"
+                   else "qgemm_pair_kernel" if M % 256 == 0 and N % 256 == 0 else "qgemm_kernel")
     gemm_peak_src = ("bf16 burst x 1 (the INT4 path multiplies fp16)" if fmt == "int4"
                      else f"bf16 burst x {FP4_OVER_BF16:g} (nominal dense FP4:BF16)")
     gemm_tflops = flops_step / (gm_us * 1e-6) / 1e12
     tq_gbs = tq_bytes / (tq_us * 1e-6) / 1e9
     qgemm_src = os.path.join(ROOT, "activation_quantization_b200", "csrc",
                              "qgemm_int4.cu" if fmt == "int4" else "qgemm.cu")
-    tq_src = os.path.join(ROOT, "activation_quantization_b200", "csrc", "transform_quant.cu")
+    tq_src = os.path.join(ROOT, "activation_quantization_b200", "csrc", "transform_quant_tc.cu")
 
     # end to end through the public API: pinned host X -> device, step, y -> pinned host
     if True:
@@ -373,7 +412,7 @@ def run_gpu(args, rank, world):
     result = None
     if rank == 0:
         traffic = traffic_from_profiles(gemm_kernel, args.workload, qgemm_src)
-        tq_traffic = traffic_from_profiles("transform_quant_kernel", args.workload, tq_src)
+        tq_traffic = traffic_from_profiles("tq_tc_kernel", args.workload, tq_src)
         result = {
             "metric": "transform+quant HBM GB/s; W4A4 block-scaled GEMM TFLOP/s (% of peak)",
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -381,7 +420,9 @@ def run_gpu(args, rank, world):
             "vs_baseline": None, "dtype": "e2m1 x e2m1 -> fp32 (transform in fp32)", "data": "synthetic",
             "config": describe(w, fmt, kind),
             "transform_quant": {"us": tq_us, "GB_s": tq_gbs, "bytes_per_launch": tq_bytes,
-                                "frac_of_hbm": tq_gbs / peaks["hbm_gbs"], "dram_bytes_per_launch": tq_traffic},
+                                "frac_of_hbm": tq_gbs / peaks["hbm_gbs"], "dram_bytes_per_launch": tq_traffic,
+                                "burst_us": tq_burst_us,
+                                "burst_frac_of_hbm": tq_bytes / (tq_burst_us * 1e-6) / 1e9 / peaks["hbm_gbs"]},
             "qgemm": {"us": gm_us, "TFLOP_s": gemm_tflops, "frac_of_peak": gemm_tflops / fp4_peak},
             "roofline": {"kernel": gemm_kernel, "bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak,
                          "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak, "traffic": traffic,
