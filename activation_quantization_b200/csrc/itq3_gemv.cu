@@ -4,11 +4,11 @@
 // ITQ3_S article, section "核心技术：FWHT预旋转与TurboQuant的完美融合": weights are
 // stored as uniform 3-bit codes of their FWHT-rotated 256-element blocks, and
 // the exact inverse transform is applied as the weights are loaded for the
-// matmul.  Here one warp owns one output row; lane l holds elements 8*l .. 8*l + 7
-// of each 256-block, whose codes are the 24 contiguous bits at bit 24*l of the
-// block's packed 96 bytes, so a lane decodes its eight weights with one funnel
-// shift and one bit-field extract and one FMA each, and reads its x values with
-// 16-byte shared loads.
+// matmul.  Here one warp owns one to four output rows; lane l holds elements
+// 8*l .. 8*l + 7 of each 256-block, whose codes are the 24 contiguous bits at bit
+// 24*l of the block's packed 96 bytes, so a lane decodes its eight weights with
+// one funnel shift and one bit-field extract and one FMA each, and reads its x
+// values with 16-byte loads.
 //
 // mode 0 (the article's design): the 256-point inverse FWHT of each weight
 //   block runs in registers -- index bits 0..2 inside the lane, bits 3..7 across
@@ -42,13 +42,15 @@ namespace {
 
 constexpr int kWarps = 8;
 
-// Levels (c - 3.5) s of the eight elements 8 lane .. 8 lane + 7 of one 256-block,
-// from the CTA's shared copy of its 24 code words: 3-bit codes packed
-// little-endian, element e at bits 3e .. 3e + 2 of the block.
-__device__ __forceinline__ void unpack_levels_smem(const uint32_t* words, int lane, float s, float (&v)[8]) {
+// Levels (c - 3.5) s of the eight elements 8 lane .. 8 lane + 7 of one 256-block.
+// Lane j < 24 holds word j of the block's 96 packed bytes (3-bit codes,
+// little-endian, element e at bits 3e .. 3e + 2); this lane's 24 bits start at bit
+// 24 lane, inside words (24 lane) / 32 and the one after it.
+__device__ __forceinline__ void decode_levels(uint32_t word, int lane, float s, float (&v)[8]) {
   const int bit = 24 * lane;
   const int w0 = bit >> 5;
-  const uint32_t lo = words[w0], hi = words[w0 + 1 < 24 ? w0 + 1 : 23];
+  const uint32_t lo = __shfl_sync(0xffffffffu, word, w0);
+  const uint32_t hi = __shfl_sync(0xffffffffu, word, w0 + 1 < 24 ? w0 + 1 : 23);
   const uint32_t bits = __funnelshift_r(lo, hi, bit & 31);
   const float m = -3.5f * s;
 #pragma unroll
@@ -81,89 +83,95 @@ __device__ __forceinline__ void warp_fwht256(float (&v)[8], int lane) {
   }
 }
 
-// One CTA owns kWarps consecutive output rows (one per warp).  Thread 0 fetches
-// the CTA's packed codes and scales (contiguous, kWarps * nb * 96 and
-// kWarps * nb * 2 bytes) with two bulk async copies; meanwhile all threads stage
-// the activations of the current 256-block for every token as fp32 in a double
-// buffer, so each warp reads its x values and code words from shared memory.
+// One warp owns R consecutive output rows and walks the 256-blocks of d_in in
+// windows of W blocks: it first issues every code-word and scale load of the
+// window (lanes 0..23 take the 24 words of a block, one each), then decodes each
+// block (two shuffles and a funnel shift per lane) and multiplies it into the
+// accumulators of TC tokens at a time; each x load is shared by the R rows.  Every
+// access is a plain load: x is small and stays in L1 and L2.
 // MODE 0: x is fp16 and the inverse FWHT runs on every weight block (the
 // article's fused design).  MODE 1: x is the fp32 rotated activation (H x / 16)
 // and the weights are used as their levels (c - 3.5) s.
-template <int T, int MODE>
-__global__ void __launch_bounds__(kWarps * 32) itq3_gemv_kernel(const uint8_t* __restrict__ codes,
+template <int R, int W, int TC, int MODE>
+__global__ void __launch_bounds__(kWarps * 32) itq3_gemv_kernel(const uint32_t* __restrict__ codes,
                                                                 const __half* __restrict__ scales,
                                                                 const void* __restrict__ xin, int tokens,
                                                                 int d_out, int d_in, float* __restrict__ y) {
-  extern __shared__ __align__(16) uint8_t itq3_smem[];
+  const int lane = threadIdx.x & 31;
+  const int row0 = (blockIdx.x * kWarps + (threadIdx.x >> 5)) * R;
+  if (row0 >= d_out) return;
   const int nb = d_in / 256;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int o0 = blockIdx.x * kWarps;
-  const int codes_bytes = kWarps * nb * 96;
-  const int scale_bytes = ((kWarps * nb * 2 + 15) / 16) * 16;
-  uint8_t* scodes = itq3_smem;
-  const __half* sscales = reinterpret_cast<const __half*>(itq3_smem + codes_bytes);
-  float* sx = reinterpret_cast<float*>(itq3_smem + codes_bytes + scale_bytes);   // [2][T][256]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sx + 2 * T * 256);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 1);
-
-  if (threadIdx.x == 0) {
-    sm100::mbar_init(bar, 1);
-    *abort_flag = 0;
-    sm100::fence_barrier_init();
-    sm100::mbar_arrive_expect_tx(bar, static_cast<uint32_t>(codes_bytes + kWarps * nb * 2));
-    sm100::bulk_load(scodes, codes + static_cast<int64_t>(o0) * nb * 96, static_cast<uint32_t>(codes_bytes), bar);
-    sm100::bulk_load(itq3_smem + codes_bytes, scales + static_cast<int64_t>(o0) * nb,
-                     static_cast<uint32_t>(kWarps * nb * 2), bar);
-  }
-  auto stage_x = [&](int blk, int buf) {
-    float* dst = sx + buf * T * 256;
-    for (int i = threadIdx.x; i < tokens * 256; i += kWarps * 32) {
-      const int tt = i >> 8, e = i & 255;
-      const int64_t src = static_cast<int64_t>(tt) * d_in + blk * 256 + e;
-      dst[tt * 256 + e] = MODE == 0 ? __half2float(static_cast<const __half*>(xin)[src])
-                                    : static_cast<const float*>(xin)[src];
+  for (int tc0 = 0; tc0 < tokens; tc0 += TC) {
+    float acc[R][TC];
+#pragma unroll
+    for (int rr = 0; rr < R; ++rr)
+#pragma unroll
+      for (int tt = 0; tt < TC; ++tt) acc[rr][tt] = 0.f;
+    for (int b0 = 0; b0 < nb; b0 += W) {
+      uint32_t word[R][W];
+      float sc[R][W];
+#pragma unroll
+      for (int rr = 0; rr < R; ++rr)
+#pragma unroll
+        for (int w = 0; w < W; ++w) {
+          const int row = row0 + rr, blk = b0 + w;
+          const bool live = row < d_out && blk < nb;
+          const int64_t cb = (static_cast<int64_t>(row) * nb + blk);
+          word[rr][w] = (live && lane < 24) ? __ldg(codes + cb * 24 + lane) : 0u;
+          sc[rr][w] = live ? __half2float(scales[cb]) : 0.f;
+        }
+#pragma unroll
+      for (int w = 0; w < W; ++w) {
+        const int blk = b0 + w;
+        if (blk >= nb) break;
+        float v[R][8];
+#pragma unroll
+        for (int rr = 0; rr < R; ++rr) {
+          decode_levels(word[rr][w], lane, sc[rr][w], v[rr]);
+          if constexpr (MODE == 0) {
+            warp_fwht256(v[rr], lane);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[rr][i] *= 0.0625f;
+          }
+        }
+#pragma unroll
+        for (int tt = 0; tt < TC; ++tt) {
+          const int t = tc0 + tt;
+          if (t >= tokens) break;
+          const int64_t xo = static_cast<int64_t>(t) * d_in + blk * 256 + 8 * lane;
+          float x8[8];
+          if constexpr (MODE == 0) {
+            const uint4 h = __ldg(reinterpret_cast<const uint4*>(static_cast<const __half*>(xin) + xo));
+            const uint32_t hw[4] = {h.x, h.y, h.z, h.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hw[i]));
+              x8[2 * i] = f.x;
+              x8[2 * i + 1] = f.y;
+            }
+          } else {
+            const float4 xa = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(xin) + xo));
+            const float4 xb = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(xin) + xo + 4));
+            x8[0] = xa.x; x8[1] = xa.y; x8[2] = xa.z; x8[3] = xa.w;
+            x8[4] = xb.x; x8[5] = xb.y; x8[6] = xb.z; x8[7] = xb.w;
+          }
+#pragma unroll
+          for (int rr = 0; rr < R; ++rr)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[rr][tt] = fmaf(v[rr][i], x8[i], acc[rr][tt]);
+        }
+      }
     }
-  };
-  stage_x(0, 0);
-  __syncthreads();                                   // barrier initialised, block 0 of x staged
-  const bool have_codes = sm100::mbar_wait_bounded(bar, 0, int64_t(1) << 40, 4000000000ull, abort_flag);
-  if (!have_codes && threadIdx.x == 0) atomicOr(&g_itq3_error, 1 << kErrTimeoutBarrier);
-
-  float acc[T];
 #pragma unroll
-  for (int t = 0; t < T; ++t) acc[t] = 0.f;
-  const int row = warp;
-  for (int blk = 0; blk < nb; ++blk) {
-    if (blk + 1 < nb) stage_x(blk + 1, (blk + 1) & 1);
-    float v[8];
-    unpack_levels_smem(reinterpret_cast<const uint32_t*>(scodes + (row * nb + blk) * 96), lane,
-                       __half2float(sscales[row * nb + blk]), v);
-    if constexpr (MODE == 0) {
-      warp_fwht256(v, lane);
+    for (int rr = 0; rr < R; ++rr)
 #pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] *= 0.0625f;
-    }
-    const float* xb = sx + (blk & 1) * T * 256 + 8 * lane;
+      for (int tt = 0; tt < TC; ++tt) {
+        const int t = tc0 + tt, row = row0 + rr;
+        float a = acc[rr][tt];
 #pragma unroll
-    for (int t = 0; t < T; ++t) {
-      if (t >= tokens) break;
-      const float4 xa = *reinterpret_cast<const float4*>(xb + t * 256);
-      const float4 xc = *reinterpret_cast<const float4*>(xb + t * 256 + 4);
-      acc[t] = fmaf(v[0], xa.x, acc[t]); acc[t] = fmaf(v[1], xa.y, acc[t]);
-      acc[t] = fmaf(v[2], xa.z, acc[t]); acc[t] = fmaf(v[3], xa.w, acc[t]);
-      acc[t] = fmaf(v[4], xc.x, acc[t]); acc[t] = fmaf(v[5], xc.y, acc[t]);
-      acc[t] = fmaf(v[6], xc.z, acc[t]); acc[t] = fmaf(v[7], xc.w, acc[t]);
-    }
-    __syncthreads();                                 // x block blk + 1 staged; block blk no longer read
-  }
-  if (!have_codes) return;
-#pragma unroll
-  for (int t = 0; t < T; ++t) {
-    if (t >= tokens) break;
-    float a = acc[t];
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
-    if (lane == 0) y[static_cast<int64_t>(t) * d_out + o0 + row] = a;
+        for (int off = 16; off > 0; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
+        if (lane == 0 && t < tokens && row < d_out) y[static_cast<int64_t>(t) * d_out + row] = a;
+      }
   }
 }
 
@@ -185,31 +193,19 @@ __global__ void __launch_bounds__(kWarps * 32) itq3_rotate_x_kernel(const __half
   for (int i = 0; i < 8; ++i) out[32 * i] = v[i] * 0.0625f;
 }
 
-size_t itq3_smem_bytes(int tmax, int64_t d_in) {
-  const int64_t nb = d_in / 256;
-  return static_cast<size_t>(kWarps * nb * 96 + ((kWarps * nb * 2 + 15) / 16) * 16 + 2 * tmax * 256 * 4 + 16);
-}
-
+// Rows per warp, blocks per load window and tokens per pass by token count: one
+// row and all 16 blocks of a 4096-wide row in flight per warp for a single token
+// (memory-bound), more rows sharing each x load as the token count grows.
 template <int MODE>
 int launch_gemv(const uint32_t* c32, const __half* sc, const void* x, int t, int n, int k, float* y,
                 cudaStream_t st) {
-  const int tmax = t == 1 ? 1 : (t <= 4 ? 4 : 16);
-  const size_t smem = itq3_smem_bytes(tmax, k);
-  if (smem > 200 * 1024) return WUSH_ERR_UNSUPPORTED;
-  const dim3 grid(static_cast<unsigned>(n / kWarps)), block(kWarps * 32);
-  const uint8_t* cb = reinterpret_cast<const uint8_t*>(c32);
-#define WUSH_ITQ3(TT)                                                                                          \
-  do {                                                                                                         \
-    if (smem > 48 * 1024 &&                                                                                    \
-        cudaFuncSetAttribute(itq3_gemv_kernel<TT, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,          \
-                             static_cast<int>(smem)) != cudaSuccess)                                           \
-      return WUSH_ERR_CUDA;                                                                                    \
-    itq3_gemv_kernel<TT, MODE><<<grid, block, smem, st>>>(cb, sc, x, t, n, k, y);                              \
-  } while (0)
-  if (tmax == 1) WUSH_ITQ3(1);
-  else if (tmax == 4) WUSH_ITQ3(4);
-  else WUSH_ITQ3(16);
-#undef WUSH_ITQ3
+  const dim3 block(kWarps * 32);
+  auto grid_for = [&](int rows_per_warp) {
+    return dim3(static_cast<unsigned>((n + kWarps * rows_per_warp - 1) / (kWarps * rows_per_warp)));
+  };
+  if (t == 1) itq3_gemv_kernel<1, 16, 1, MODE><<<grid_for(1), block, 0, st>>>(c32, sc, x, t, n, k, y);
+  else if (t <= 4) itq3_gemv_kernel<2, 8, 4, MODE><<<grid_for(2), block, 0, st>>>(c32, sc, x, t, n, k, y);
+  else itq3_gemv_kernel<4, 4, 4, MODE><<<grid_for(4), block, 0, st>>>(c32, sc, x, t, n, k, y);
   return launch_status();
 }
 
@@ -224,7 +220,7 @@ extern "C" int itq3_dequant_gemv(const uint8_t* codes, const void* scales_fp16, 
   if (tokens < 1 || tokens > 16 || d_out <= 0 || d_in <= 0 || d_in % 256 || d_out % 8) return WUSH_ERR_INVALID_ARG;
   if (d_out > (int64_t(1) << 30) || d_in > (int64_t(1) << 30)) return WUSH_ERR_UNSUPPORTED;
   if (mode != 0 && mode != 1) return WUSH_ERR_UNSUPPORTED;
-  if (!codes || !scales_fp16 || !x_fp16 || !y || !aligned16(codes) || !aligned16(scales_fp16))
+  if (!codes || !scales_fp16 || !x_fp16 || !y || !aligned16(codes) || !aligned16(scales_fp16) || !aligned16(x_fp16))
     return WUSH_ERR_INVALID_ARG;
   if (mode == 1 && (!workspace || !aligned16(workspace))) return WUSH_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -290,7 +286,7 @@ extern "C" int itq3_dequant_gemv_noalloc(const uint8_t* codes, const void* scale
   if (tokens < 1 || tokens > 16 || d_out <= 0 || d_in <= 0 || d_in % 256 || d_out % 8) return WUSH_ERR_INVALID_ARG;
   if (tokens * d_in > kNoAllocScratchFloats) return WUSH_ERR_BUFFER_TOO_SMALL;
   if (d_out > (int64_t(1) << 30)) return WUSH_ERR_UNSUPPORTED;
-  if (!codes || !scales_fp16 || !x_fp16 || !y || !aligned16(codes) || !aligned16(scales_fp16))
+  if (!codes || !scales_fp16 || !x_fp16 || !y || !aligned16(codes) || !aligned16(scales_fp16) || !aligned16(x_fp16))
     return WUSH_ERR_INVALID_ARG;
   float* scratch = nullptr;
   const int st = scratch_for_current_device(&scratch);

@@ -232,7 +232,8 @@ int itq3_quantize_weights(const uint16_t* w_fp16, int64_t d_out, int64_t d_in, u
  *         call into ``workspace`` (device fp32 [tokens, d_in], caller-owned
  *         scratch), then each weight is used without a transform.
  * workspace may be NULL for mode 0.  Requirements: 1 <= tokens <= 16,
- * d_in % 256 == 0, d_out % 8 == 0, codes and scales 16-byte aligned. */
+ * d_in % 256 == 0, d_out % 8 == 0, codes, scales, x_fp16 and workspace 16-byte
+ * aligned; WUSH_ERR_INVALID_ARG otherwise, before any launch. */
 int itq3_dequant_gemv(const uint8_t* codes, const void* scales_fp16, const void* x_fp16,
                       int64_t tokens, int64_t d_out, int64_t d_in, int mode, float* workspace,
                       float* y, void* stream);
