@@ -38,6 +38,8 @@ _SIGNATURES = {
     "wush_transform_amax": (_i32, [_vp, _i32, _i64, _i64, _vp, _i32, _i32, _vp, _vp]),
     "wush_qgemm": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _f32, _vp, _vp]),
     "wush_qgemm_int4": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp]),
+    "wush_qgemm_int4_workspace_bytes": (_sz, [_i64, _i64, _i64]),
+    "wush_qgemm_int4_ws": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _sz, _vp, _vp]),
     "itq3_quantize_weights": (_i32, [_vp, _i64, _i64, _vp, _vp]),
     "itq3_dequant_gemv": (_i32, [_vp, _vp, _vp, _i64, _i64, _i64, _i32, _vp, _vp, _vp]),
     "itq3_dequant_gemv_noalloc": (_i32, [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp]),
@@ -190,6 +192,17 @@ def wush_qgemm_int4(a_codes, a_scales, b_codes, b_scales, M: int, N: int, K: int
            _lib.wush_qgemm_int4(_ptr(a_codes), _ptr(a_scales), _ptr(b_codes), _ptr(b_scales), M, N, K, _ptr(y),
                                 _stream(stream)))
 
+
+def wush_qgemm_int4_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(_lib.wush_qgemm_int4_workspace_bytes(M, N, K))
+
+
+def wush_qgemm_int4_ws(a_codes, a_scales, b_codes, b_scales, M: int, N: int, K: int, workspace, y, stream=None):
+    """workspace: CUDA tensor of at least wush_qgemm_int4_workspace_bytes(M, N, K) bytes."""
+    nbytes = workspace.numel() * workspace.element_size()
+    _check("wush_qgemm_int4_ws",
+           _lib.wush_qgemm_int4_ws(_ptr(a_codes), _ptr(a_scales), _ptr(b_codes), _ptr(b_scales), M, N, K,
+                                   _ptr(workspace), nbytes, _ptr(y), _stream(stream)))
 
 def itq3_dequant_gemv(codes, scales, x, d_out: int, mode: int, y, workspace=None, stream=None):
     tokens, d_in = x.shape

@@ -296,6 +296,218 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
+// ---------------------------------------------------------------------------
+// Two-pass form.
+//
+// Dequantising inside the GEMM repeats the conversion for every output tile that
+// reads an operand row (N / 256 times for a row of A, M / 128 times for a row of
+// B); at the sizes of a transformer layer that conversion, not the tensor cores,
+// bounds the fused kernel.  The two-pass form converts each operand element once,
+// into a caller workspace (a memory-bound pass), and multiplies the fp16 operands
+// with a CTA-pair GEMM.  With no scale factors in TMEM, two 256-column fp32
+// accumulators fit, so the epilogue of one tile overlaps the main loop of the next.
+
+// out[g] = the eight fp16(q * s) of INT4 code word g (elements 8g .. 8g + 7 of the
+// row-major [rows, K] matrix), one thread per word; scales are fp16 [rows, K / 32].
+__global__ void __launch_bounds__(256) int4_dequant_kernel(const uint32_t* __restrict__ codes,
+                                                           const __half* __restrict__ scales, int64_t words,
+                                                           int words_per_row, uint4* __restrict__ out) {
+  const int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (g >= words) return;
+  const int64_t r = g / words_per_row;
+  const int c = static_cast<int>(g - r * words_per_row);
+  const __half s = scales[r * (words_per_row / 4) + c / 4];
+  uint32_t o[4];
+  dequant8(__ldg(codes + g), __halves2half2(s, s), o);
+  out[g] = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+namespace hp {
+constexpr int kRowBytes = 128;                       // 64 fp16 of an operand row per k-tile
+constexpr int kKTile = 64;
+constexpr int kABytes = 128 * kRowBytes;             // this CTA's 128 rows of A
+constexpr int kBBytes = 128 * kRowBytes;             // this CTA's 128-row half of the 256 B rows
+constexpr int kStageBytes = kABytes + kBBytes;       // 32 KB, a multiple of 1024
+constexpr int kStages = 6;
+constexpr int kAccs = 2;
+constexpr int kEpiWarps = 8;                         // two per TMEM lane quarter
+constexpr int kThreads = 64 + kEpiWarps * 32;        // producer warp, MMA warp, epilogue
+constexpr int kEpiChunk = 32 * 32 * 4;               // one warp's 32 x 32 fp32 output chunk
+constexpr int kSmemBytes = kStages * kStageBytes + kEpiWarps * kEpiChunk + 1024 /*align*/ + 256 /*barriers*/;
+constexpr uint32_t kTmemCols = 512;                  // two 256-column accumulators
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+}  // namespace hp
+
+__device__ __forceinline__ void mma_f16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// y = A B^T for fp16 A [M, K] and B [N, K] (K-major), fp32 y [M, N]; CTA pairs own
+// 256 x 256 output tiles (M fastest), each CTA loading its 128 rows of A and its
+// 128-row half of B per 64-wide k-tile into a 6-stage ring:
+//   warp 0      TMA producer (both CTAs; transaction bytes counted on the leader);
+//   warp 1      leader only: four M = 256, N = 256, K = 16 MMAs per k-tile into
+//               accumulator (tile & 1), committing stages and tiles to both CTAs;
+//   warps 2-9   epilogue (both CTAs): TMEM -> registers, release the accumulator,
+//               then 128-byte-swizzled shared chunks -> TMA stores of y.
+__global__ void __launch_bounds__(hp::kThreads, 1)
+    hgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                      const __grid_constant__ CUtensorMap tmap_y, int M, int N, int K, int64_t max_polls) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* epi_smem = smem + hp::kStages * hp::kStageBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(epi_smem + hp::kEpiWarps * hp::kEpiChunk);
+  uint64_t* empty = full + hp::kStages;
+  uint64_t* acc_full = empty + hp::kStages;
+  uint64_t* acc_empty = acc_full + hp::kAccs;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + hp::kAccs);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x / 2, n_pairs = gridDim.x / 2;
+  const int mt = M / 256, n_ptiles = mt * (N / 256);
+  const int k_tiles = K / hp::kKTile;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < hp::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < hp::kAccs; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 2 * hp::kEpiWarps);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tmap_a);
+    prefetch_tmap(&tmap_b);
+    prefetch_tmap(&tmap_y);
+  }
+  if (warp == 1) tmem_alloc_pair(tmem_slot, hp::kTmemCols);
+  tc_fence_before();
+  cluster_sync();                       // both CTAs' barriers exist before either touches the other's
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto give_up = [&]() {
+    if (!*abort_flag) {
+      *abort_flag = 1;
+      const uint32_t peer = mapa_shared(smem_u32(const_cast<int*>(abort_flag)), rank ^ 1u);
+      asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(peer), "r"(1) : "memory");
+      atomicOr(&g_int4_error, 1 << kErrTimeoutBarrier);
+    }
+  };
+
+  if (warp == 0) {
+    if (elect_one()) {
+      int it = 0;
+      bool ok = true;
+      for (int pt = pair; ok && pt < n_ptiles; pt += n_pairs) {
+        const int pm = pt % mt, pn = pt / mt;
+        const int arow = pm * 256 + static_cast<int>(rank) * 128;   // this CTA's A rows
+        const int brow = pn * 256 + static_cast<int>(rank) * 128;   // this CTA's half of the B rows
+        for (int kt = 0; kt < k_tiles; ++kt, ++it) {
+          const int s = it % hp::kStages;
+          if (!mbar_wait_bounded(&empty[s], ((it / hp::kStages) & 1) ^ 1, max_polls, kDeadlineNs, abort_flag)) {
+            give_up();
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + s * hp::kStageBytes;
+          if (leader) mbar_arrive_expect_tx(&full[s], 2 * hp::kStageBytes);
+          tma_load_2d_pair(sa, &tmap_a, kt * hp::kRowBytes, arow, &full[s]);
+          tma_load_2d_pair(sa + hp::kABytes, &tmap_b, kt * hp::kRowBytes, brow, &full[s]);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (leader && elect_one()) {
+      constexpr uint32_t idesc = idesc_f16_f32(256, 256);
+      bool ok = true;
+      int it = 0, tcount = 0;
+      for (int pt = pair; ok && pt < n_ptiles; pt += n_pairs, ++tcount) {
+        const int a = tcount & 1;
+        if (!mbar_wait_bounded(&acc_empty[a], ((tcount >> 1) & 1) ^ 1, max_polls, kDeadlineNs, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem + a * 256;
+        for (int kt = 0; kt < k_tiles; ++kt, ++it) {
+          const int s = it % hp::kStages;
+          if (!mbar_wait_bounded(&full[s], (it / hp::kStages) & 1, max_polls, kDeadlineNs, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t a0 = desc_kmajor_sw128(smem_u32(smem + s * hp::kStageBytes));
+          const uint64_t b0 = desc_kmajor_sw128(smem_u32(smem + s * hp::kStageBytes + hp::kABytes));
+#pragma unroll
+          for (int kk = 0; kk < hp::kKTile / 16; ++kk)       // 32-byte steps inside the 128-byte rows
+            mma_f16_pair(d, a0 + 2 * kk, b0 + 2 * kk, idesc, (kt | kk) ? 1u : 0u);
+          tc_commit_pair(&empty[s], 0x3);
+        }
+        if (!ok) break;
+        tc_commit_pair(&acc_full[a], 0x3);
+      }
+      if (!ok) give_up();
+    }
+  } else {
+    const int ew = warp - 2, q = warp & 3, half = ew / 4;
+    uint8_t* buf = epi_smem + ew * hp::kEpiChunk;
+    int tcount = 0;
+    for (int pt = pair; pt < n_ptiles; pt += n_pairs, ++tcount) {
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+      const int pm = pt % mt, pn = pt / mt, a = tcount & 1;
+      bool ok = mbar_wait_bounded(&acc_full[a], (tcount >> 1) & 1, max_polls, kDeadlineNs, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) { give_up(); break; }
+      tc_fence_after();
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + a * 256 + half * 128;
+      uint32_t r[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tbase + 32 * c, r[c]);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty[a]), 0));
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        if (lane == 0) bulk_wait_group_read<0>();       // the previous store has read the chunk
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<uint4*>(buf + lane * 128 + ((j ^ (lane & 7)) * 16)) =
+              make_uint4(r[c][4 * j], r[c][4 * j + 1], r[c][4 * j + 2], r[c][4 * j + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmap_y, buf, pn * 256 + half * 128 + 32 * c, pm * 256 + static_cast<int>(rank) * 128 + q * 32);
+          bulk_commit_group();
+        }
+      }
+    }
+    if (lane == 0) bulk_wait_group_all();
+  }
+  __syncwarp();
+  if (*abort_flag) {
+    const uint64_t until = globaltimer_ns() + 200000ull;
+    while (globaltimer_ns() < until) __nanosleep(1000);
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();                       // no CTA frees TMEM or exits while its pair still works
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem, hp::kTmemCols);
+}
+
 using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                               const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                               CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -313,6 +525,81 @@ EncodeFn get_encode() {
   return fn;
 }
 
+
+// Map over a row-major matrix viewed as bytes: rows x row_bytes, boxes of
+// box_rows x 128 bytes with the 128-byte swizzle (the K-major operand layout).
+bool make_operand_map(CUtensorMap* map, const void* base, int64_t rows, int64_t row_bytes, int box_rows) {
+  EncodeFn enc = get_encode();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+  const cuuint32_t box[2] = {128, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// fp32 y [rows, cols]: 32 x 32 boxes with the 128-byte swizzle (TMA stores).
+bool make_y_map32(CUtensorMap* map, float* y, int64_t rows, int64_t cols) {
+  EncodeFn enc = get_encode();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 4};
+  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+int launch_dequant(const uint8_t* codes, const void* scales, int64_t rows, int64_t K, __half* out, cudaStream_t st) {
+  const int64_t words = rows * (K / 8);
+  const int64_t blocks = (words + 255) / 256;
+  if (blocks > 0x7FFFFFFF) return WUSH_ERR_UNSUPPORTED;
+  int4_dequant_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+      reinterpret_cast<const uint32_t*>(codes), static_cast<const __half*>(scales), words, static_cast<int>(K / 8),
+      reinterpret_cast<uint4*>(out));
+  return launch_status();
+}
+
+int launch_hgemm_pair(const __half* a, const __half* b, int64_t M, int64_t N, int64_t K, float* y, cudaStream_t st) {
+  CUtensorMap ma, mb, my;
+  if (!make_operand_map(&ma, a, M, K * 2, 128) || !make_operand_map(&mb, b, N, K * 2, 128) ||
+      !make_y_map32(&my, y, M, N))
+    return WUSH_ERR_CUDA;
+  static uint64_t attr_done = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return WUSH_ERR_CUDA;
+  if (dev < 64 && !(attr_done >> dev & 1)) {
+    if (cudaFuncSetAttribute(hgemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, hp::kSmemBytes) !=
+        cudaSuccess)
+      return WUSH_ERR_CUDA;
+    attr_done |= uint64_t(1) << dev;
+  }
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 2)
+    return WUSH_ERR_CUDA;
+  const int64_t n_ptiles = (M / 256) * (N / 256);
+  const int pairs = static_cast<int>(n_ptiles < sms / 2 ? n_ptiles : sms / 2);
+  const int64_t polls = g_wait_limit_override > 0 ? g_wait_limit_override : kDefaultPolls;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+  cfg.blockDim = dim3(hp::kThreads);
+  cfg.dynamicSmemBytes = hp::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, hgemm_pair_kernel, ma, mb, my, static_cast<int>(M), static_cast<int>(N),
+                         static_cast<int>(K), polls) != cudaSuccess)
+    return WUSH_ERR_CUDA;
+  return launch_status();
+}
 }  // namespace
 }  // namespace wush
 
@@ -356,4 +643,28 @@ extern "C" int wush_qgemm_int4(const uint8_t* a_codes, const void* a_scales, con
       a_codes, static_cast<const __half*>(a_scales), b_codes, static_cast<const __half*>(b_scales), my,
       static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), polls);
   return launch_status();
+}
+
+extern "C" size_t wush_qgemm_int4_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  return static_cast<size_t>(M + N) * static_cast<size_t>(K) * 2;
+}
+
+extern "C" int wush_qgemm_int4_ws(const uint8_t* a_codes, const void* a_scales, const uint8_t* b_codes,
+                                  const void* b_scales, int64_t M, int64_t N, int64_t K, void* workspace,
+                                  size_t workspace_bytes, float* y, void* stream) {
+  if (M <= 0 || N <= 0 || K <= 0 || M % 256 || N % 256 || K % 64) return WUSH_ERR_INVALID_ARG;
+  if (M > (int64_t(1) << 30) || N > (int64_t(1) << 30) || K > (int64_t(1) << 30)) return WUSH_ERR_UNSUPPORTED;
+  if (!a_codes || !a_scales || !b_codes || !b_scales || !workspace || !y) return WUSH_ERR_INVALID_ARG;
+  if (!aligned16(a_codes) || !aligned16(b_codes) || !aligned16(workspace) || !aligned16(y) ||
+      (reinterpret_cast<uintptr_t>(a_scales) & 1u) || (reinterpret_cast<uintptr_t>(b_scales) & 1u))
+    return WUSH_ERR_INVALID_ARG;
+  if (workspace_bytes < wush_qgemm_int4_workspace_bytes(M, N, K)) return WUSH_ERR_BUFFER_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  __half* wa = static_cast<__half*>(workspace);
+  __half* wb = wa + M * K;
+  int status = launch_dequant(a_codes, a_scales, M, K, wa, st);
+  if (status == WUSH_OK) status = launch_dequant(b_codes, b_scales, N, K, wb, st);
+  if (status == WUSH_OK) status = launch_hgemm_pair(wa, wb, M, N, K, y, st);
+  return status;
 }

@@ -265,9 +265,15 @@ def run_gpu(args, rank, world):
     def tq(r):
         aq.wush_transform_quant(xs[r], t_x, kind, fmt, acodes[r][0], acodes[r][1], gx, stream=stream)
 
+    # INT4: the two-pass form (each operand dequantised once to fp16, then a CTA-pair
+    # fp16 GEMM); its workspace is allocated once, outside the timed region
+    ws = (torch.empty(aq.wush_qgemm_int4_workspace_bytes(M, N, K), dtype=torch.uint8, device=dev)
+          if fmt == "int4" else None)
+
     def gemm(r):
         if fmt == "int4":
-            aq.wush_qgemm_int4(acodes[r][0], acodes[r][1], wcodes[r][0], wcodes[r][1], M, N, K, y, stream=stream)
+            aq.wush_qgemm_int4_ws(acodes[r][0], acodes[r][1], wcodes[r][0], wcodes[r][1], M, N, K, ws, y,
+                                  stream=stream)
         else:
             aq.wush_qgemm(acodes[r][0], acodes[r][1], wcodes[r][0], wcodes[r][1], M, N, K, fmt, alpha, y,
                           stream=stream)
@@ -373,7 +379,7 @@ def run_gpu(args, rank, world):
     fp4_peak = peaks["bf16_tflops"] * (FP4_OVER_BF16 if fmt != "int4" else 1.0)
     tq_bytes = (M * K * 2 + aq.wush_codes_bytes(M, K, fmt) + aq.wush_scales_bytes(M, K, fmt)
                 + (K // b) * b * b * 4)
-    gemm_kernel = ("qgemm_int4_kernel" if fmt == "int4"
+    gemm_kernel = ("hgemm_pair_kernel" if fmt == "int4"
                    else "qgemm_pair_kernel" if M % 256 == 0 and N % 256 == 0 else "qgemm_kernel")
     gemm_peak_src = ("bf16 burst x 1 (the INT4 path multiplies fp16)" if fmt == "int4"
                      else f"bf16 burst x {FP4_OVER_BF16:g} (nominal dense FP4:BF16)")
@@ -427,7 +433,7 @@ def run_gpu(args, rank, world):
             "roofline": {"kernel": gemm_kernel, "bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak,
                          "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak, "traffic": traffic,
                          "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']:.1f} TFLOP/s, {gemm_peak_src}"},
-            "e2e": e2e, "gpu_launches": 2 * args.steps,
+            "e2e": e2e, "gpu_launches": (4 if fmt == "int4" else 2) * args.steps,
             "clocks": sampler.summary(),
         }
     return result, (w, x, wt, xc, fmt, kind)

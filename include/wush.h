@@ -201,6 +201,24 @@ int wush_qgemm(const uint8_t* a_codes, const void* a_scales, const uint8_t* b_co
 int wush_qgemm_int4(const uint8_t* a_codes, const void* a_scales, const uint8_t* b_codes,
                     const void* b_scales, int64_t M, int64_t N, int64_t K, float* y, void* stream);
 
+/* Bytes of device workspace wush_qgemm_int4_ws needs: (M + N) * K * 2 (the fp16
+ * operands); 0 if any size is <= 0. */
+size_t wush_qgemm_int4_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/* Two-pass form of wush_qgemm_int4 with the same definition of y: every INT4
+ * element of A and B is dequantised once to fp16(q * s) into ``workspace``
+ * (device, caller-owned, A's [M, K] then B's [N, K], row-major), then the fp16
+ * operands are multiplied with CTA-pair fp16 MMAs accumulating in fp32.  Cheaper
+ * than the fused form whenever the operands are reused by many output tiles (the
+ * fused form converts an element once per tile that reads it).
+ * Requirements: M % 256 == 0, N % 256 == 0, K % 64 == 0, all > 0; codes,
+ * workspace and y 16-byte aligned, scales 2-byte aligned; workspace_bytes >=
+ * wush_qgemm_int4_workspace_bytes(M, N, K), else WUSH_ERR_BUFFER_TOO_SMALL.  All
+ * checks run before any launch; three kernels are launched on ``stream``. */
+int wush_qgemm_int4_ws(const uint8_t* a_codes, const void* a_scales, const uint8_t* b_codes,
+                       const void* b_scales, int64_t M, int64_t N, int64_t K, void* workspace,
+                       size_t workspace_bytes, float* y, void* stream);
+
 /* ---------------------------------------------------------------------------
  * ITQ3_S-style 3-bit weights with a 256-wide Walsh-Hadamard rotation
  *

@@ -82,3 +82,69 @@ def test_int4_rejects_bad_shapes(lib):
     for mnk in ((100, 256, 64), (128, 200, 64), (128, 256, 48)):
         with pytest.raises(lib.WushError):
             lib.wush_qgemm_int4(z, z, z, z, *mnk, y)
+
+
+def _run_ws(lib, a_c, a_s, b_c, b_s, m, n, k, y):
+    ws = torch.empty(lib.wush_qgemm_int4_workspace_bytes(m, n, k), dtype=torch.uint8, device="cuda")
+    lib.wush_qgemm_int4_ws(a_c, a_s, b_c, b_s, m, n, k, ws, y)
+
+
+@pytest.mark.parametrize("mnk", [(256, 256, 64), (256, 512, 640), (512, 768, 2048), (256, 256, 5120)])
+def test_int4_gemm_two_pass_random(lib, mnk):
+    m, n, k = mnk
+    a_c, a_s, a_dq = _random_int4(31 + m, m, k)
+    b_c, b_s, b_dq = _random_int4(42 + n, n, k)
+    dev = "cuda"
+    args = [torch.from_numpy(v).to(dev) for v in (a_c, a_s, b_c, b_s)]
+    y = torch.full((m, n), float("nan"), dtype=torch.float32, device=dev)
+    _run_ws(lib, *args, m, n, k, y)
+    assert lib.wush_check_device_status() == 0
+    got = y.cpu().numpy().astype(np.float64)
+    assert np.isfinite(got).all()
+    err = _rel(got, G.gemm_dequantized(a_dq, b_dq))
+    assert err <= 5e-4, err
+    # the fused form rounds the same fp16 operands: the two agree to fp32 accumulation order
+    y2 = torch.empty_like(y)
+    lib.wush_qgemm_int4(*args, m, n, k, y2)
+    diff = _rel(got, y2.cpu().numpy().astype(np.float64))
+    assert diff <= 1e-5, diff
+
+
+def test_int4_two_pass_end_to_end_sampled(lib):
+    # the int4 workload at 2048 tokens through the two-pass form, oracle on 40 x 256
+    w = synth.WORKLOADS["int4"]
+    m, n, k = 2048, w.d_out, w.d_in
+    x = synth.activations(w, tokens=m)
+    wt = synth.weights(w)
+    xc = synth.activations(w, tokens=1024, calib=True)
+    tx, tw = C.calibrate(xc, wt[:2048], 32, "wush")
+    tx, tw = tx.astype(np.float32), tw.astype(np.float32)
+    dev = "cuda"
+    ac, as_ = lib.alloc_quant_outputs(m, k, "int4")
+    bc, bs = lib.alloc_quant_outputs(n, k, "int4")
+    lib.wush_transform_quant(torch.from_numpy(x).to(torch.bfloat16).to(dev), torch.from_numpy(tx).to(dev),
+                             "wush", "int4", ac, as_)
+    lib.wush_transform_quant(torch.from_numpy(wt).to(torch.bfloat16).to(dev), torch.from_numpy(tw).to(dev),
+                             "wush", "int4", bc, bs)
+    y = torch.empty((m, n), dtype=torch.float32, device=dev)
+    _run_ws(lib, ac, as_, bc, bs, m, n, k, y)
+    assert lib.wush_check_device_status() == 0
+    rng = np.random.default_rng(6)
+    rows = np.sort(rng.choice(m, 40, replace=False))
+    cols = np.sort(rng.choice(n, 256, replace=False))
+    want = G.gemm_dequantized(Q.transform_quantize(x[rows], tx, "int4")["dq"],
+                              Q.transform_quantize(wt[cols], tw, "int4")["dq"])
+    got = y.cpu().numpy()[np.ix_(rows, cols)].astype(np.float64)
+    assert _rel(got, want) <= P.GEMM_REL_FRO
+
+
+def test_int4_two_pass_rejects_bad_arguments(lib):
+    z = torch.zeros(1 << 16, dtype=torch.uint8, device="cuda")
+    y = torch.zeros(1 << 14, dtype=torch.float32, device="cuda")
+    ws = torch.zeros(1 << 20, dtype=torch.uint8, device="cuda")
+    for mnk in ((128, 256, 64), (256, 384, 64), (256, 256, 48)):
+        with pytest.raises(lib.WushError):
+            lib.wush_qgemm_int4_ws(z, z, z, z, *mnk, ws, y)
+    small = torch.zeros(lib.wush_qgemm_int4_workspace_bytes(256, 256, 64) - 16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(lib.WushError, match="BUFFER_TOO_SMALL|too small"):
+        lib.wush_qgemm_int4_ws(z, z, z, z, 256, 256, 64, small, y)
