@@ -201,8 +201,12 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t local, uint32_t rank) {
   return r;
 }
 
+// Arrive on a barrier in another CTA of the cluster (address from mapa_shared).
+// CTA-scope release: the TMEM hand-offs that use it are already ordered by
+// tcgen05.wait::ld and tcgen05.fence::before_thread_sync, and a cluster-scope
+// release would also wait for the thread's outstanding global stores.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // 2D TMA tile load issued by either CTA of a pair; the transaction bytes are
