@@ -312,11 +312,15 @@ struct Cfg2 {
   static constexpr int kSfbBytes = 2 * kAtomsK * 512;           // both 128-row halves of the N tile
   static constexpr int kCtaBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
   static constexpr int kStageBytes = ((kCtaBytes + 1023) / 1024) * 1024;
-  static constexpr int kStages = 5;
+  // MXFP4 stages are small enough for a sixth if the epilogue stages y in 1 KB
+  // chunks (32 rows x 8 fp32); NVFP4's scale tiles leave room for five with 4 KB
+  // chunks (32 rows x 32 fp32, 128-byte swizzle).
+  static constexpr int kStages = NV ? 5 : 6;
   static constexpr int kTxBytesPair = 2 * kCtaBytes;
-  static constexpr int kEpiBufs = 1;
-  static constexpr int kEpiBytes = kEpiWarps * kEpiBufs * kEpiChunkBytes;
+  static constexpr int kEpiCols = NV ? 32 : 8;                  // fp32 columns per staged chunk
+  static constexpr int kEpiBytes = kEpiWarps * 32 * kEpiCols * 4;
   static constexpr int kSmemBytes = kStages * kStageBytes + kEpiBytes + 1024 + 256;
+  static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
 
 template <bool NV>
@@ -454,8 +458,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     const int ew = warp - 2, q = warp & 3, half = ew / 4;
     const uint32_t leader_acc_empty = mapa_shared(smem_u32(acc_empty), 0);
-    uint8_t* bufs = epi_smem + ew * C::kEpiBufs * kEpiChunkBytes;
-    int buf = 0, tcount = 0;
+    uint8_t* sbuf = epi_smem + ew * 32 * C::kEpiCols * 4;
+    int tcount = 0;
     for (int pt = pair; pt < n_ptiles; pt += n_pairs, ++tcount) {
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
       const int pm = pt % mt, pn = pt / mt;
@@ -473,21 +477,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive_cluster(leader_acc_empty);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        if (lane == 0) bulk_wait_group_read<C::kEpiBufs - 1>();
-        __syncwarp();
-        uint8_t* sb = bufs + buf * kEpiChunkBytes;
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          *reinterpret_cast<float4*>(sb + lane * 128 + ((j ^ (lane & 7)) * 16)) =
-              make_float4(alpha * __uint_as_float(r[c][4 * j]), alpha * __uint_as_float(r[c][4 * j + 1]),
-                          alpha * __uint_as_float(r[c][4 * j + 2]), alpha * __uint_as_float(r[c][4 * j + 3]));
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(&tmap_y, sb, pn * 256 + half * 128 + 32 * c, pm * 256 + static_cast<int>(rank) * 128 + q * 32);
-          bulk_commit_group();
+        for (int sc = 0; sc < 32 / C::kEpiCols; ++sc) {
+          if (lane == 0) bulk_wait_group_read<0>();   // the previous store has read the chunk
+          __syncwarp();
+          if constexpr (C::kEpiCols == 32) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              *reinterpret_cast<float4*>(sbuf + lane * 128 + ((j ^ (lane & 7)) * 16)) =
+                  make_float4(alpha * __uint_as_float(r[c][4 * j]), alpha * __uint_as_float(r[c][4 * j + 1]),
+                              alpha * __uint_as_float(r[c][4 * j + 2]), alpha * __uint_as_float(r[c][4 * j + 3]));
+          } else {
+            // 32-byte rows, one per lane: the warp writes one contiguous kilobyte
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const int e = sc * 8 + 4 * j;
+              *reinterpret_cast<float4*>(sbuf + lane * 32 + j * 16) =
+                  make_float4(alpha * __uint_as_float(r[c][e]), alpha * __uint_as_float(r[c][e + 1]),
+                              alpha * __uint_as_float(r[c][e + 2]), alpha * __uint_as_float(r[c][e + 3]));
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmap_y, sbuf, pn * 256 + half * 128 + 32 * c + sc * C::kEpiCols,
+                         pm * 256 + static_cast<int>(rank) * 128 + q * 32);
+            bulk_commit_group();
+          }
         }
-        buf = (buf + 1) % C::kEpiBufs;
       }
     }
     if (lane == 0) bulk_wait_group_all();
@@ -534,17 +551,18 @@ bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t row_byte
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 2D map over fp32 y [rows, cols]: 32 x 32 boxes with 128-byte swizzle (TMA stores).
-bool make_y_map(CUtensorMap* map, float* y, int64_t rows, int64_t cols) {
+// 2D map over fp32 y [rows, cols] for TMA stores: boxes of 32 rows x box_cols; 32
+// columns (128-byte rows) use the 128-byte swizzle, 8 columns (32-byte rows) none.
+bool make_y_map(CUtensorMap* map, float* y, int64_t rows, int64_t cols, int box_cols) {
   EncodeFn enc = get_encode();
   if (!enc) return false;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 4};
-  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), 32};
   const cuuint32_t estr[2] = {1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-         CUDA_SUCCESS;
+             box_cols == 32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // 2D map over a scale buffer viewed as rows of 256 bytes (two rows per 512-byte atom).
@@ -566,7 +584,8 @@ int launch_pair(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const ui
   using C = Cfg2<NV>;
   const int64_t n_acols = (K / (NV ? 16 : 32) + 3) / 4;
   CUtensorMap ma, mb, msa, msb, my;
-  if (!make_map(&ma, a, M, K / 2, kBM) || !make_map(&mb, b, N, K / 2, kBM) || !make_y_map(&my, y, M, N) ||
+  if (!make_map(&ma, a, M, K / 2, kBM) || !make_map(&mb, b, N, K / 2, kBM) ||
+      !make_y_map(&my, y, M, N, C::kEpiCols) ||
       !make_sf_map(&msa, sfa, (M / 128) * n_acols * 512, 2 * C::kAtomsK) ||
       !make_sf_map(&msb, sfb, (N / 128) * n_acols * 512, 2 * C::kAtomsK))
     return WUSH_ERR_CUDA;
@@ -608,7 +627,7 @@ int launch(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const uint8_t
            int64_t K, float alpha, float* y, cudaStream_t st) {
   using C = Cfg<BN, NV>;
   CUtensorMap ma, mb, my;
-  if (!make_map(&ma, a, M, K / 2, kBM) || !make_map(&mb, b, N, K / 2, BN) || !make_y_map(&my, y, M, N))
+  if (!make_map(&ma, a, M, K / 2, kBM) || !make_map(&mb, b, N, K / 2, BN) || !make_y_map(&my, y, M, N, 32))
     return WUSH_ERR_CUDA;
   auto kern = qgemm_kernel<BN, NV>;
   static uint64_t attr_done = 0;  // one bit per device: dynamic shared memory opt-in done
