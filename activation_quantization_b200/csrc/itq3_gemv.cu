@@ -87,20 +87,44 @@ __device__ __forceinline__ void warp_fwht256(float (&v)[8], int lane) {
 // windows of W blocks: it first issues every code-word and scale load of the
 // window (lanes 0..23 take the 24 words of a block, one each), then decodes each
 // block (two shuffles and a funnel shift per lane) and multiplies it into the
-// accumulators of TC tokens at a time; each x load is shared by the R rows.  Every
-// access is a plain load: x is small and stays in L1 and L2.
+// accumulators of TC tokens at a time; each x load is shared by the R rows.  With
+// STAGE the CTA first copies the chunk's TC tokens of x into shared memory as fp32,
+// so the block loop waits on shared-memory latency rather than L2.
 // MODE 0: x is fp16 and the inverse FWHT runs on every weight block (the
 // article's fused design).  MODE 1: x is the fp32 rotated activation (H x / 16)
 // and the weights are used as their levels (c - 3.5) s.
-template <int R, int W, int TC, int MODE>
+template <int R, int W, int TC, int MODE, bool STAGE>
 __global__ void __launch_bounds__(kWarps * 32) itq3_gemv_kernel(const uint32_t* __restrict__ codes,
                                                                 const __half* __restrict__ scales,
                                                                 const void* __restrict__ xin, int tokens,
                                                                 int d_out, int d_in, float* __restrict__ y) {
+  extern __shared__ __align__(16) float sx[];      // STAGE: [TC][d_in] fp32
   const int lane = threadIdx.x & 31;
   const int row0 = (blockIdx.x * kWarps + (threadIdx.x >> 5)) * R;
-  if (row0 >= d_out) return;
+  if (!STAGE && row0 >= d_out) return;             // with STAGE every warp joins the barriers
   const int nb = d_in / 256;
+  // Copies tokens tc0 .. tc0 + TC - 1 of x into shared memory as fp32 (zeros past
+  // the last token); every warp of the CTA takes part.
+  auto stage_x = [&](int tc0) {
+    __syncthreads();                               // the previous chunk is no longer read
+    for (int i = threadIdx.x * 4; i < TC * d_in; i += kWarps * 32 * 4) {
+      const int tt = i / d_in, e = i - tt * d_in, t = tc0 + tt;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (t < tokens) {
+        const int64_t xo = static_cast<int64_t>(t) * d_in + e;
+        if constexpr (MODE == 0) {
+          const uint2 h = __ldg(reinterpret_cast<const uint2*>(static_cast<const __half*>(xin) + xo));
+          const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&h.x));
+          const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&h.y));
+          v = make_float4(a.x, a.y, b.x, b.y);
+        } else {
+          v = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(xin) + xo));
+        }
+      }
+      *reinterpret_cast<float4*>(sx + i) = v;
+    }
+    __syncthreads();
+  };
   for (int tc0 = 0; tc0 < tokens; tc0 += TC) {
     float acc[R][TC];
 #pragma unroll
@@ -120,6 +144,11 @@ __global__ void __launch_bounds__(kWarps * 32) itq3_gemv_kernel(const uint32_t* 
           word[rr][w] = (live && lane < 24) ? __ldg(codes + cb * 24 + lane) : 0u;
           sc[rr][w] = live ? __half2float(scales[cb]) : 0.f;
         }
+      // the first window's loads are in flight while the CTA stages x; warps past
+      // the last row (only in the last CTA) run on zero codes and store nothing
+      if constexpr (STAGE) {
+        if (b0 == 0) stage_x(tc0);
+      }
 #pragma unroll
       for (int w = 0; w < W; ++w) {
         const int blk = b0 + w;
@@ -140,7 +169,13 @@ __global__ void __launch_bounds__(kWarps * 32) itq3_gemv_kernel(const uint32_t* 
           if (t >= tokens) break;
           const int64_t xo = static_cast<int64_t>(t) * d_in + blk * 256 + 8 * lane;
           float x8[8];
-          if constexpr (MODE == 0) {
+          if constexpr (STAGE) {
+            const float* xs = sx + tt * d_in + blk * 256 + 8 * lane;
+            const float4 xa = *reinterpret_cast<const float4*>(xs);
+            const float4 xb = *reinterpret_cast<const float4*>(xs + 4);
+            x8[0] = xa.x; x8[1] = xa.y; x8[2] = xa.z; x8[3] = xa.w;
+            x8[4] = xb.x; x8[5] = xb.y; x8[6] = xb.z; x8[7] = xb.w;
+          } else if constexpr (MODE == 0) {
             const uint4 h = __ldg(reinterpret_cast<const uint4*>(static_cast<const __half*>(xin) + xo));
             const uint32_t hw[4] = {h.x, h.y, h.z, h.w};
 #pragma unroll
@@ -196,17 +231,35 @@ __global__ void __launch_bounds__(kWarps * 32) itq3_rotate_x_kernel(const __half
 // Rows per warp, blocks per load window and tokens per pass by token count: one
 // row and all 16 blocks of a 4096-wide row in flight per warp for a single token
 // (memory-bound), more rows sharing each x load as the token count grows.
+template <int R, int W, int TC, int MODE>
+int launch_one(const uint32_t* c32, const __half* sc, const void* x, int t, int n, int k, float* y, cudaStream_t st) {
+  const dim3 block(kWarps * 32);
+  const dim3 grid(static_cast<unsigned>((n + kWarps * R - 1) / (kWarps * R)));
+  const size_t smem = static_cast<size_t>(TC) * k * 4;
+  // a single token's x is read through L1 well enough; staging pays off once a
+  // chunk of several tokens is reused by every row of the CTA
+  if (TC > 1 && smem <= 160 * 1024) {
+    auto kern = itq3_gemv_kernel<R, W, TC, MODE, true>;
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+      return WUSH_ERR_CUDA;
+    kern<<<grid, block, smem, st>>>(c32, sc, x, t, n, k, y);
+  } else {
+    itq3_gemv_kernel<R, W, TC, MODE, false><<<grid, block, 0, st>>>(c32, sc, x, t, n, k, y);
+  }
+  return launch_status();
+}
+
+// Rows per warp, blocks per load window and tokens per pass by token count: one
+// row and all 16 blocks of a 4096-wide row in flight per warp for a single token
+// (memory-bound), more rows sharing each x load as the token count grows.  For
+// several tokens x is staged in shared memory when a token chunk of it fits.
 template <int MODE>
 int launch_gemv(const uint32_t* c32, const __half* sc, const void* x, int t, int n, int k, float* y,
                 cudaStream_t st) {
-  const dim3 block(kWarps * 32);
-  auto grid_for = [&](int rows_per_warp) {
-    return dim3(static_cast<unsigned>((n + kWarps * rows_per_warp - 1) / (kWarps * rows_per_warp)));
-  };
-  if (t == 1) itq3_gemv_kernel<1, 16, 1, MODE><<<grid_for(1), block, 0, st>>>(c32, sc, x, t, n, k, y);
-  else if (t <= 4) itq3_gemv_kernel<2, 8, 4, MODE><<<grid_for(2), block, 0, st>>>(c32, sc, x, t, n, k, y);
-  else itq3_gemv_kernel<4, 4, 4, MODE><<<grid_for(4), block, 0, st>>>(c32, sc, x, t, n, k, y);
-  return launch_status();
+  if (t == 1) return launch_one<1, 16, 1, MODE>(c32, sc, x, t, n, k, y, st);
+  if (t <= 4) return launch_one<2, 8, 4, MODE>(c32, sc, x, t, n, k, y, st);
+  return launch_one<4, 4, 4, MODE>(c32, sc, x, t, n, k, y, st);
 }
 
 }  // namespace
