@@ -52,6 +52,39 @@ def load_peaks():
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
 
 
+def dist_init(world: int):
+    """One process per GPU: NCCL when CUDA is present, gloo otherwise (CPU tests)."""
+    if world <= 1:
+        return None
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    backend = "nccl" if torch.cuda.is_available() else "gloo"
+    if backend == "nccl":
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(value: float, world: int) -> float:
+    """The largest ``value`` of all ranks (device time is taken as the slowest rank's)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" else torch.device("cpu")
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def source_sha(source_file: str) -> str:
     """Hash of a kernel's source file together with the device headers it includes."""
     csrc = os.path.dirname(source_file)
@@ -145,6 +178,7 @@ def cpu_threads():
 # --------------------------------------------------------------------------- workload
 
 WORKLOADS = {
+    "tiny": dict(fmt="mxfp4", kind="wush"),          # 128 x 256 x 256: a quick check, not a bench line
     "up_proj": dict(fmt="mxfp4", kind="wush"),
     "down_proj": dict(fmt="nvfp4", kind="wush"),
     "int4": dict(fmt="int4", kind="wush"),
@@ -308,14 +342,9 @@ def run_gpu(args, rank, world):
     if aq.wush_check_device_status(stream) != 0:
         raise RuntimeError("device status after capture")
 
-    def barrier():
-        if world > 1:
-            import torch.distributed as dist
-            dist.barrier()
-
     def timed(steps):
         e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        barrier()
+        barrier(world)
         torch.cuda.synchronize()
         with torch.cuda.stream(stream):
             e_start.record(stream)
@@ -325,7 +354,7 @@ def run_gpu(args, rank, world):
                 g_rem.replay()
             e_end.record(stream)
         torch.cuda.synchronize()
-        barrier()
+        barrier(world)
         total_ms = e_start.elapsed_time(e_end)
         # per-kernel device times from the event nodes of the last replay
         evs = ev_main if steps >= STEPS_PER_GRAPH else ev_rem
@@ -364,11 +393,7 @@ def run_gpu(args, rank, world):
     torch.cuda.synchronize()
     tq_burst_us = 1e3 * b0.elapsed_time(b1) / (8 * STEPS_PER_GRAPH)
 
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world)
 
     flops_step = 2.0 * M * N * K
     value = flops_step * args.steps * world / (total_ms * 1e-3) / 1e12
@@ -405,12 +430,7 @@ def run_gpu(args, rank, world):
                 y_host.copy_(y, non_blocking=True)
             e1.record(stream)
         torch.cuda.synchronize()
-        e_ms = e0.elapsed_time(e1) / e_steps
-        if world > 1:
-            import torch.distributed as dist
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(e0.elapsed_time(e1) / e_steps, world)
         e2e = {"value": flops_step * world / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": int(x_host.numel() * 2), "d2h_bytes_per_step": int(y_host.numel() * 4),
                "ms_per_step": e_ms}
@@ -506,7 +526,8 @@ def main():
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     if args.workload == "itq3":
-        run_itq3(args)
+        if rank == 0:               # a per-call latency benchmark: one rank times it
+            run_itq3(args)
         return
     spec = WORKLOADS[args.workload]
 
@@ -536,13 +557,7 @@ def main():
                                   "d2h_bytes_per_step": 0}}))
         return
 
-    if world > 1:
-        import datetime
-
-        import torch
-        import torch.distributed as dist
-        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dist_init(world)
     result, ctx = run_gpu(args, rank, world)
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
