@@ -338,6 +338,20 @@ constexpr uint32_t kTmemCols = 512;                  // two 256-column accumulat
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 }  // namespace hp
 
+// Tile order of the fp16 pair GEMM: groups of kGroupRows 256-row blocks of A, N
+// fastest inside a group, so the tiles in flight at once share a few row blocks of
+// A and a few of B (each group reads A's rows once and B once) instead of sweeping
+// all of A for every column of tiles.
+constexpr int kGroupRows = 8;
+
+__device__ __forceinline__ void pair_tile_coords(int pt, int mt, int nt, int& pm, int& pn) {
+  const int g = pt / (kGroupRows * nt);
+  const int rows = min(kGroupRows, mt - g * kGroupRows);
+  const int w = pt - g * kGroupRows * nt;
+  pm = g * kGroupRows + w % rows;
+  pn = w / rows;
+}
+
 __device__ __forceinline__ void mma_f16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                              uint32_t accumulate) {
   asm volatile(
@@ -348,8 +362,8 @@ __device__ __forceinline__ void mma_f16_pair(uint32_t tmem_d, uint64_t adesc, ui
 }
 
 // y = A B^T for fp16 A [M, K] and B [N, K] (K-major), fp32 y [M, N]; CTA pairs own
-// 256 x 256 output tiles (M fastest), each CTA loading its 128 rows of A and its
-// 128-row half of B per 64-wide k-tile into a 6-stage ring:
+// 256 x 256 output tiles (in pair_tile_coords order), each CTA loading its 128
+// rows of A and its 128-row half of B per 64-wide k-tile into a 6-stage ring:
 //   warp 0      TMA producer (both CTAs; transaction bytes counted on the leader);
 //   warp 1      leader only: four M = 256, N = 256, K = 16 MMAs per k-tile into
 //               accumulator (tile & 1), committing stages and tiles to both CTAs;
@@ -372,7 +386,7 @@ __global__ void __launch_bounds__(hp::kThreads, 1)
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
   const int pair = blockIdx.x / 2, n_pairs = gridDim.x / 2;
-  const int mt = M / 256, n_ptiles = mt * (N / 256);
+  const int mt = M / 256, nt = N / 256, n_ptiles = mt * nt;
   const int k_tiles = K / hp::kKTile;
 
   if (threadIdx.x == 0) {
@@ -410,7 +424,8 @@ __global__ void __launch_bounds__(hp::kThreads, 1)
       int it = 0;
       bool ok = true;
       for (int pt = pair; ok && pt < n_ptiles; pt += n_pairs) {
-        const int pm = pt % mt, pn = pt / mt;
+        int pm, pn;
+        pair_tile_coords(pt, mt, nt, pm, pn);
         const int arow = pm * 256 + static_cast<int>(rank) * 128;   // this CTA's A rows
         const int brow = pn * 256 + static_cast<int>(rank) * 128;   // this CTA's half of the B rows
         for (int kt = 0; kt < k_tiles; ++kt, ++it) {
@@ -465,7 +480,9 @@ __global__ void __launch_bounds__(hp::kThreads, 1)
     int tcount = 0;
     for (int pt = pair; pt < n_ptiles; pt += n_pairs, ++tcount) {
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-      const int pm = pt % mt, pn = pt / mt, a = tcount & 1;
+      int pm, pn;
+      pair_tile_coords(pt, mt, nt, pm, pn);
+      const int a = tcount & 1;
       bool ok = mbar_wait_bounded(&acc_full[a], (tcount >> 1) & 1, max_polls, kDeadlineNs, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) { give_up(); break; }
