@@ -259,7 +259,7 @@ int launch_gemv(const uint32_t* c32, const __half* sc, const void* x, int t, int
                 cudaStream_t st) {
   if (t == 1) return launch_one<1, 16, 1, MODE>(c32, sc, x, t, n, k, y, st);
   if (t <= 4) return launch_one<2, 8, 4, MODE>(c32, sc, x, t, n, k, y, st);
-  return launch_one<4, 4, 4, MODE>(c32, sc, x, t, n, k, y, st);
+  return launch_one<4, 4, 8, MODE>(c32, sc, x, t, n, k, y, st);
 }
 
 }  // namespace
