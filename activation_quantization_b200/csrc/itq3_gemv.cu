@@ -251,14 +251,15 @@ int launch_one(const uint32_t* c32, const __half* sc, const void* x, int t, int 
 }
 
 // Rows per warp, blocks per load window and tokens per pass by token count: one
-// row and all 16 blocks of a 4096-wide row in flight per warp for a single token
-// (memory-bound), more rows sharing each x load as the token count grows.  For
-// several tokens x is staged in shared memory when a token chunk of it fits.
+// row and all 16 blocks of a 4096-wide row in flight per warp for a single token,
+// four rows sharing each decoded x load once there are several tokens (measured
+// best on B200).  For several tokens x is staged in shared memory when a token
+// chunk of it fits.
 template <int MODE>
 int launch_gemv(const uint32_t* c32, const __half* sc, const void* x, int t, int n, int k, float* y,
                 cudaStream_t st) {
   if (t == 1) return launch_one<1, 16, 1, MODE>(c32, sc, x, t, n, k, y, st);
-  if (t <= 4) return launch_one<2, 8, 4, MODE>(c32, sc, x, t, n, k, y, st);
+  if (t <= 4) return launch_one<4, 4, 4, MODE>(c32, sc, x, t, n, k, y, st);
   return launch_one<4, 4, 8, MODE>(c32, sc, x, t, n, k, y, st);
 }
 
