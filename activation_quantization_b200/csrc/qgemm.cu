@@ -9,13 +9,15 @@
 // (NVFP4, kind::mxf4nvf4, block16).  Products of codes and scales are exact;
 // accumulation is fp32 in TMEM.
 //
-// A persistent CTA per SM walks 128 x BN output tiles (BN = 256, or 128 when
-// N % 256 != 0) round-robin, with three roles:
+// Two kernels.  When M and N are multiples of 256, persistent CTA pairs
+// (qgemm_pair_kernel, described above its configuration below) own 256 x 256
+// tiles.  Otherwise a persistent CTA per SM (qgemm_kernel) walks 128 x BN output
+// tiles (BN = 256, or 128 when N % 256 != 0) round-robin, with three roles:
 //   warp 0     TMA producer: per 256-wide k-tile, one 2D TMA load of the A tile
 //              (128 rows x 128 bytes, 128-byte swizzle), one of the B tile, and
 //              untiled bulk copies of the matching 512-byte scale atoms, all
-//              completing on the stage's "full" mbarrier; the 4-stage ring runs
-//              on across tile boundaries;
+//              completing on the stage's "full" mbarrier; the 3-stage (BN 256)
+//              or 4-stage (BN 128) ring runs on across tile boundaries;
 //   warp 1     allocates TMEM; one elected thread copies the stage's scale atoms
 //              into TMEM (tcgen05.cp 32x128b.warpx4) and issues the four K=64
 //              block-scaled MMAs, then commits the stage back to the producer;
