@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "wush.h"
 
 namespace wush {
@@ -38,6 +40,21 @@ inline int launch_status() {
 }
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Raises a kernel's dynamic shared-memory limit to ``bytes`` once per device;
+// ``done`` holds one bit per device (devices 64 and up are set on every call).
+// Safe to call from several host threads: setting the attribute twice is harmless.
+template <typename Kernel>
+inline int set_smem_once(Kernel kernel, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return WUSH_ERR_CUDA;
+  const uint64_t bit = dev >= 0 && dev < 64 ? uint64_t(1) << dev : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return WUSH_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return WUSH_ERR_CUDA;
+  if (bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return WUSH_OK;
+}
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }

@@ -240,9 +240,8 @@ int launch_one(const uint32_t* c32, const __half* sc, const void* x, int t, int 
   // chunk of several tokens is reused by every row of the CTA
   if (TC > 1 && smem <= 160 * 1024) {
     auto kern = itq3_gemv_kernel<R, W, TC, MODE, true>;
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
-      return WUSH_ERR_CUDA;
+    static std::atomic<uint64_t> attr_done{0};     // the limit is raised to the 160 KB cap once
+    if (smem > 48 * 1024 && set_smem_once(kern, 160 * 1024, attr_done) != WUSH_OK) return WUSH_ERR_CUDA;
     kern<<<grid, block, smem, st>>>(c32, sc, x, t, n, k, y);
   } else {
     itq3_gemv_kernel<R, W, TC, MODE, false><<<grid, block, 0, st>>>(c32, sc, x, t, n, k, y);

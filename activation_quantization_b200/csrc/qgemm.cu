@@ -284,13 +284,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 int num_sms() {
-  static int cached[64] = {};
+  static std::atomic<int> cached[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (dev < 64 && cached[dev]) return cached[dev];
+  if (dev >= 0 && dev < 64) {
+    const int c = cached[dev].load(std::memory_order_relaxed);
+    if (c) return c;
+  }
   int n = 0;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  if (dev < 64) cached[dev] = n;
+  if (dev >= 0 && dev < 64) cached[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 
@@ -592,14 +595,8 @@ int launch_pair(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const ui
       !make_sf_map(&msb, sfb, (N / 128) * n_acols * 512, 2 * C::kAtomsK))
     return WUSH_ERR_CUDA;
   auto kern = qgemm_pair_kernel<NV>;
-  static uint64_t attr_done = 0;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return WUSH_ERR_CUDA;
-  if (dev < 64 && !(attr_done >> dev & 1)) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
-      return WUSH_ERR_CUDA;
-    attr_done |= uint64_t(1) << dev;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (set_smem_once(kern, C::kSmemBytes, attr_done) != WUSH_OK) return WUSH_ERR_CUDA;
   const int n_ptiles = static_cast<int>((M / 256) * (N / 256));
   const int sms = num_sms();
   if (sms < 2) return WUSH_ERR_CUDA;
@@ -632,14 +629,8 @@ int launch(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const uint8_t
   if (!make_map(&ma, a, M, K / 2, kBM) || !make_map(&mb, b, N, K / 2, BN) || !make_y_map(&my, y, M, N, 32))
     return WUSH_ERR_CUDA;
   auto kern = qgemm_kernel<BN, NV>;
-  static uint64_t attr_done = 0;  // one bit per device: dynamic shared memory opt-in done
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return WUSH_ERR_CUDA;
-  if (dev < 64 && !(attr_done >> dev & 1)) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
-      return WUSH_ERR_CUDA;
-    attr_done |= uint64_t(1) << dev;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (set_smem_once(kern, C::kSmemBytes, attr_done) != WUSH_OK) return WUSH_ERR_CUDA;
   const int64_t polls = g_wait_limit_override > 0 ? g_wait_limit_override : kDefaultPolls;
   const int debug_never = g_wait_limit_override > 0 ? 1 : 0;
   const int n_tiles = static_cast<int>((M / kBM) * (N / BN));

@@ -585,16 +585,10 @@ int launch_hgemm_pair(const __half* a, const __half* b, int64_t M, int64_t N, in
   if (!make_operand_map(&ma, a, M, K * 2, 128) || !make_operand_map(&mb, b, N, K * 2, 128) ||
       !make_y_map32(&my, y, M, N))
     return WUSH_ERR_CUDA;
-  static uint64_t attr_done = 0;
-  int dev = 0;
+  static std::atomic<uint64_t> attr_done{0};
+  if (set_smem_once(hgemm_pair_kernel, hp::kSmemBytes, attr_done) != WUSH_OK) return WUSH_ERR_CUDA;
+  int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return WUSH_ERR_CUDA;
-  if (dev < 64 && !(attr_done >> dev & 1)) {
-    if (cudaFuncSetAttribute(hgemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, hp::kSmemBytes) !=
-        cudaSuccess)
-      return WUSH_ERR_CUDA;
-    attr_done |= uint64_t(1) << dev;
-  }
-  int sms = 0;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 2)
     return WUSH_ERR_CUDA;
   const int64_t n_ptiles = (M / 256) * (N / 256);
@@ -641,15 +635,10 @@ extern "C" int wush_qgemm_int4(const uint8_t* a_codes, const void* a_scales, con
           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
       CUDA_SUCCESS)
     return WUSH_ERR_CUDA;
-  static uint64_t attr_done = 0;
+  static std::atomic<uint64_t> attr_done{0};
+  if (set_smem_once(qgemm_int4_kernel, kSmemBytes, attr_done) != WUSH_OK) return WUSH_ERR_CUDA;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return WUSH_ERR_CUDA;
-  if (dev < 64 && !(attr_done >> dev & 1)) {
-    if (cudaFuncSetAttribute(qgemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
-        cudaSuccess)
-      return WUSH_ERR_CUDA;
-    attr_done |= uint64_t(1) << dev;
-  }
   int sms = 0;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
     return WUSH_ERR_CUDA;

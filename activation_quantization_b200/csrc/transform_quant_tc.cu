@@ -611,13 +611,16 @@ EncodeFn get_encode() {
 }
 
 int num_sms() {
-  static int cached[64] = {};
+  static std::atomic<int> cached[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (dev < 64 && cached[dev]) return cached[dev];
+  if (dev >= 0 && dev < 64) {
+    const int c = cached[dev].load(std::memory_order_relaxed);
+    if (c) return c;
+  }
   int n = 0;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  if (dev < 64) cached[dev] = n;
+  if (dev >= 0 && dev < 64) cached[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 
@@ -636,14 +639,8 @@ int launch_tc(const void* x, int64_t rows, int64_t d_in, const float* t, float g
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return WUSH_ERR_CUDA;
   auto kern = tq_tc_kernel<B, FMT, KIND, DBG>;
-  static uint64_t attr_done = 0;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return WUSH_ERR_CUDA;
-  if (dev < 64 && !(attr_done >> dev & 1)) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
-      return WUSH_ERR_CUDA;
-    attr_done |= uint64_t(1) << dev;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (set_smem_once(kern, kSmemBytes, attr_done) != WUSH_OK) return WUSH_ERR_CUDA;
   const int n_row_tiles = static_cast<int>((rows + kTileRows - 1) / kTileRows);
   const int n_col_tiles = static_cast<int>((d_in + kTileCols - 1) / kTileCols);
   const int n_tiles = n_row_tiles * n_col_tiles;
