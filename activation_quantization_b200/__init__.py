@@ -46,6 +46,7 @@ _SIGNATURES = {
     "wush_check_device_status": (_i32, [_vp]),
     "wush_debug_set_wait_limit": (_i32, [_i64]),
     "wush_debug_set_gemm_variant": (_i32, [_i32]),
+    "wush_debug_set_itq3_variant": (_i32, [_i32]),
 }
 
 EXPORTED = []
@@ -225,6 +226,10 @@ def wush_check_device_status(stream=None) -> int:
 
 def wush_debug_set_gemm_variant(variant: int):
     _check("wush_debug_set_gemm_variant", _lib.wush_debug_set_gemm_variant(int(variant)))
+
+
+def wush_debug_set_itq3_variant(variant: int):
+    _check("wush_debug_set_itq3_variant", _lib.wush_debug_set_itq3_variant(int(variant)))
 
 
 def wush_debug_set_wait_limit(max_polls: int):

@@ -22,6 +22,7 @@ int read_and_clear_error_word(int* word);
 int read_and_clear_tq_error(int* word);
 int read_and_clear_int4_error(int* word);
 int read_and_clear_itq3_error(int* word);
+int read_and_clear_itq3_tc_error(int* word);
 
 // Tensor-core form of wush_transform_quant (bf16 inputs); WUSH_ERR_UNSUPPORTED
 // for shapes it does not take.
@@ -30,6 +31,14 @@ int transform_quant_tc(const void* x, int64_t rows, int64_t d_in, const float* t
 
 // GEMM kernel choice (see wush_debug_set_gemm_variant).
 extern int g_gemm_variant;
+
+// Tensor-core form of the ITQ3 activation-side GEMV on rotated fp32 x (device
+// [tokens, d_in]); WUSH_ERR_UNSUPPORTED, before any launch, for shapes it does not take.
+int itq3_gemv_tc(const uint8_t* codes, const void* scales_fp16, const float* x_rot, int tokens, int d_out, int d_in,
+                 float* y, cudaStream_t st);
+
+// ITQ3 mode-1 kernel choice (see wush_debug_set_itq3_variant).
+extern int g_itq3_variant;
 
 // Poll limit for bounded mbarrier waits (0 = the built-in default).
 extern int64_t g_wait_limit_override;

@@ -262,6 +262,18 @@ int launch_gemv(const uint32_t* c32, const __half* sc, const void* x, int t, int
   return launch_one<4, 4, 8, MODE>(c32, sc, x, t, n, k, y, st);
 }
 
+// Mode 1 after the rotation: the tensor-core kernel (itq3_tc.cu) where the shape
+// allows it and the CUDA-core kernel above otherwise.
+int gemv_rotated(const uint8_t* codes, const void* scales_fp16, const float* x_rot, int t, int n, int k, float* y,
+                 cudaStream_t st) {
+  if (g_itq3_variant == 0) {
+    const int r = itq3_gemv_tc(codes, scales_fp16, x_rot, t, n, k, y, st);
+    if (r != WUSH_ERR_UNSUPPORTED) return r;
+  }
+  return launch_gemv<1>(reinterpret_cast<const uint32_t*>(codes), static_cast<const __half*>(scales_fp16), x_rot, t,
+                        n, k, y, st);
+}
+
 }  // namespace
 }  // namespace wush
 
@@ -286,7 +298,7 @@ extern "C" int itq3_dequant_gemv(const uint8_t* codes, const void* scales_fp16, 
   const int items = t * (k / 256);
   itq3_rotate_x_kernel<<<(items + kWarps - 1) / kWarps, block, 0, st>>>(xh, t, k, workspace);
   if (launch_status() != WUSH_OK) return WUSH_ERR_CUDA;
-  return launch_gemv<1>(c32, sc, workspace, t, n, k, y, st);
+  return gemv_rotated(codes, scales_fp16, workspace, t, n, k, y, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -347,13 +359,11 @@ extern "C" int itq3_dequant_gemv_noalloc(const uint8_t* codes, const void* scale
   // The rotation kernel writes every scratch element the GEMV then reads, so
   // nothing left there by an earlier call needs clearing.
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const auto* c32 = reinterpret_cast<const uint32_t*>(codes);
-  const auto* sc = static_cast<const __half*>(scales_fp16);
   const auto* xh = static_cast<const __half*>(x_fp16);
   const int t = static_cast<int>(tokens), n = static_cast<int>(d_out), k = static_cast<int>(d_in);
   const dim3 block(kWarps * 32);
   const int items = t * (k / 256);
   itq3_rotate_x_kernel<<<(items + kWarps - 1) / kWarps, block, 0, s>>>(xh, t, k, scratch);
   if (launch_status() != WUSH_OK) return WUSH_ERR_CUDA;
-  return launch_gemv<1>(c32, sc, scratch, t, n, k, y, s);
+  return gemv_rotated(codes, scales_fp16, scratch, t, n, k, y, s);
 }

@@ -248,7 +248,12 @@ int itq3_quantize_weights(const uint16_t* w_fp16, int64_t d_out, int64_t d_in, u
  * mode 1: the algebraically identical activation-side form
  *         sum_k ((c - 3.5) s)[o, k] (H_256 x / 16)[t, k]: x is rotated once per
  *         call into ``workspace`` (device fp32 [tokens, d_in], caller-owned
- *         scratch), then each weight is used without a transform.
+ *         scratch), then each weight is used without a transform.  When
+ *         tokens >= 3 and d_out % 128 == 0 the weights meet x on the tensor
+ *         cores: the levels
+ *         c - 3.5 are exact fp16 MMA operands and each block of rotated x is
+ *         split exactly enough (hi + lo fp16 after a power-of-two scale) that
+ *         only the fp32 accumulation rounds; otherwise CUDA cores run it.
  * workspace may be NULL for mode 0.  Requirements: 1 <= tokens <= 16,
  * d_in % 256 == 0, d_out % 8 == 0, codes, scales, x_fp16 and workspace 16-byte
  * aligned; WUSH_ERR_INVALID_ARG otherwise, before any launch. */
@@ -293,6 +298,14 @@ int wush_debug_set_wait_limit(int64_t max_polls);
  * (when N % 256 == 0), 2 single-CTA 128 x 128 tiles, so that the forms can be
  * checked against each other. */
 int wush_debug_set_gemm_variant(int variant);
+
+/* Test hook: 0 (default) lets itq3_dequant_gemv mode 1 and
+ * itq3_dequant_gemv_noalloc run the tensor-core kernel when tokens >= 3,
+ * d_out % 128 == 0 and no CTA gets more than 64 of the 256-blocks (always so for
+ * d_in <= 16384); 1
+ * always uses the CUDA-core kernel, so that the two can be checked against each
+ * other.  WUSH_ERR_INVALID_ARG for other values. */
+int wush_debug_set_itq3_variant(int variant);
 
 #ifdef __cplusplus
 }
