@@ -42,6 +42,16 @@ namespace {
 
 constexpr int kWarps = 8;
 
+// Programmatic dependent launch: the rotation kernel lets the GEMV that follows it
+// start early, and the GEMV waits for the rotation's results only where it first
+// reads them (a no-op when it was launched without the attribute).
+__device__ __forceinline__ void allow_dependent_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void wait_for_prerequisite_grid() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // Levels (c - 3.5) s of the eight elements 8 lane .. 8 lane + 7 of one 256-block.
 // Lane j < 24 holds word j of the block's 96 packed bytes (3-bit codes,
 // little-endian, element e at bits 3e .. 3e + 2); this lane's 24 bits start at bit
@@ -144,6 +154,10 @@ __global__ void __launch_bounds__(kWarps * 32) itq3_gemv_kernel(const uint32_t* 
           word[rr][w] = (live && lane < 24) ? __ldg(codes + cb * 24 + lane) : 0u;
           sc[rr][w] = live ? __half2float(scales[cb]) : 0.f;
         }
+      // x_rot comes from the rotation kernel launched just before (mode 1)
+      if constexpr (MODE == 1) {
+        if (b0 == 0 && tc0 == 0) wait_for_prerequisite_grid();
+      }
       // the first window's loads are in flight while the CTA stages x; warps past
       // the last row (only in the last CTA) run on zero codes and store nothing
       if constexpr (STAGE) {
@@ -213,6 +227,7 @@ __global__ void __launch_bounds__(kWarps * 32) itq3_gemv_kernel(const uint32_t* 
 // x_rot[t, blk*256 + e] = (H_256 x[t, blk*256 : +256])[e] / 16; one warp per (t, blk).
 __global__ void __launch_bounds__(kWarps * 32) itq3_rotate_x_kernel(const __half* __restrict__ x, int tokens,
                                                                      int d_in, float* __restrict__ x_rot) {
+  allow_dependent_launch();
   const int lane = threadIdx.x & 31;
   const int item = blockIdx.x * kWarps + (threadIdx.x >> 5);
   const int nb = d_in / 256;
@@ -233,19 +248,26 @@ __global__ void __launch_bounds__(kWarps * 32) itq3_rotate_x_kernel(const __half
 // (memory-bound), more rows sharing each x load as the token count grows.
 template <int R, int W, int TC, int MODE>
 int launch_one(const uint32_t* c32, const __half* sc, const void* x, int t, int n, int k, float* y, cudaStream_t st) {
-  const dim3 block(kWarps * 32);
-  const dim3 grid(static_cast<unsigned>((n + kWarps * R - 1) / (kWarps * R)));
   const size_t smem = static_cast<size_t>(TC) * k * 4;
   // a single token's x is read through L1 well enough; staging pays off once a
   // chunk of several tokens is reused by every row of the CTA
-  if (TC > 1 && smem <= 160 * 1024) {
-    auto kern = itq3_gemv_kernel<R, W, TC, MODE, true>;
+  const bool stage = TC > 1 && smem <= 160 * 1024;
+  auto kern = stage ? itq3_gemv_kernel<R, W, TC, MODE, true> : itq3_gemv_kernel<R, W, TC, MODE, false>;
+  if (stage) {
     static std::atomic<uint64_t> attr_done{0};     // the limit is raised to the 160 KB cap once
     if (smem > 48 * 1024 && set_smem_once(kern, 160 * 1024, attr_done) != WUSH_OK) return WUSH_ERR_CUDA;
-    kern<<<grid, block, smem, st>>>(c32, sc, x, t, n, k, y);
-  } else {
-    itq3_gemv_kernel<R, W, TC, MODE, false><<<grid, block, 0, st>>>(c32, sc, x, t, n, k, y);
   }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((n + kWarps * R - 1) / (kWarps * R)));
+  cfg.blockDim = dim3(kWarps * 32);
+  cfg.dynamicSmemBytes = stage ? smem : 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = MODE == 1 ? 1 : 0;             // mode 1 follows the rotation kernel
+  if (cudaLaunchKernelEx(&cfg, kern, c32, sc, x, t, n, k, y) != cudaSuccess) return WUSH_ERR_CUDA;
   return launch_status();
 }
 

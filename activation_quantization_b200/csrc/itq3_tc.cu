@@ -24,8 +24,10 @@
 //   * build the hi/lo B operand (K-major, 128-byte swizzle) from x_rot,
 // then a seventeenth warp issues the block's 16 MMAs (K = 16 each) and commits
 // them, so that no decode warp waits on MMA issue; the next block's decode
-// overlaps them (two A buffers, two B stages, two accumulators).
-// Codes and x_rot for the blocks ahead are staged by cp.async, three blocks deep.
+// overlaps them (two A buffers, two B stages).  Accumulators rotate over three
+// TMEM slots and are read two blocks later, when their MMAs are long done.  An
+// eighteenth warp streams code tiles and x_rot rows by TMA into a four-block ring,
+// codes and x on separate barriers so that decoding can start before x exists.
 #include <cuda.h>
 #include <cuda_fp16.h>
 
@@ -60,6 +62,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kACols = 128;               // 256 fp16 levels of a row per block
 constexpr uint32_t kDCol0 = 2 * kACols;        // accumulators after the two A buffers
 constexpr uint32_t kDCols = 32;
+constexpr int kDBufs = 3;                      // accumulators: block b in b % 3, read two blocks later
 constexpr int kMinSmem = 120 * 1024;           // > half an SM's shared memory: one CTA per SM
 constexpr int kMaxSmem = 227 * 1024;
 constexpr int kMaxLocalBlocks = 64;
@@ -80,7 +83,7 @@ struct Cfg {
 
   static int smem_bytes(int nbl_max) {
     const int b = 1024 + 2 * kBStageBytes + kStages * kStageBytes + kSlots * kRows * 4 +
-                  nbl_max * (kRows + kSlots) * 4 + 8 * (2 * kStages + 4) + 16;
+                  nbl_max * (kRows + kSlots) * 4 + 8 * (3 * kStages + kDBufs + 2) + 16;
     return b < kMinSmem ? kMinSmem : b;
   }
 };
@@ -121,6 +124,27 @@ __device__ __forceinline__ void tmem_ld_x8(uint32_t taddr, uint32_t (&r)[8]) {
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
                : "r"(taddr));
+}
+
+// tcgen05.wait::ld that also names the loaded registers, so that no use of them
+// is scheduled before the wait.
+template <int N>
+__device__ __forceinline__ void tmem_ld_wait_regs(uint32_t (&r)[N]) {
+  if constexpr (N == 8) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7])
+                 :
+                 : "memory");
+  } else {
+    static_assert(N == 4, "4 or 8 registers");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]) : : "memory");
+  }
+}
+
+// Waits until the grid this one depends on programmatically (the rotation kernel)
+// has completed and its writes are visible; a no-op without that dependency.
+__device__ __forceinline__ void wait_for_prerequisite_grid() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 __device__ __forceinline__ uint32_t cluster_nctarank() {
@@ -173,10 +197,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* red = reinterpret_cast<float*>(ring + kStages * C_::kStageBytes);   // [ranks][kSlots][rows / ranks]
   float* s_tab = red + kSlots * kRows;                              // [nbl_max][128] block scales
   float* inv_tab = s_tab + nbl_max * kRows;                         // [nbl_max][kSlots] 2^e
-  uint64_t* full = reinterpret_cast<uint64_t*>(inv_tab + nbl_max * kSlots);
-  uint64_t* empty = full + kStages;
+  uint64_t* codes_full = reinterpret_cast<uint64_t*>(inv_tab + nbl_max * kSlots);
+  uint64_t* x_full = codes_full + kStages;
+  uint64_t* empty = x_full + kStages;
   uint64_t* mma_done = empty + kStages;
-  uint64_t* a_full = mma_done + 2;
+  uint64_t* a_full = mma_done + kDBufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(a_full + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -193,31 +218,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&full[i], 1);
+      mbar_init(&codes_full[i], 1);
+      mbar_init(&x_full[i], 1);
       mbar_init(&empty[i], kDecThreads / 32);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&mma_done[i], 1);
-      mbar_init(&a_full[i], 1);
-    }
+    for (int i = 0; i < kDBufs; ++i) mbar_init(&mma_done[i], 1);
+    for (int i = 0; i < 2; ++i) mbar_init(&a_full[i], 1);
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tmap(&tmap_codes);
     prefetch_tmap(&tmap_x);
   }
   if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
-  if (warp < kMmaWarp && g == 0) {
-    // this row's block scales, loaded together (needed from the first accumulator on)
-    for (int b0 = 0; b0 < nbl; b0 += 8) {
-      __half hv[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        hv[i] = b0 + i < nbl ? scales[static_cast<int64_t>(grow) * nb + b_lo + b0 + i] : __float2half(0.f);
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        if (b0 + i < nbl) s_tab[(b0 + i) * kRows + r] = __half2float(hv[i]);
-    }
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -233,25 +245,38 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kProducerWarp) {
     // Block b -> ring stage b % kStages: the 128-row code tile (128-byte rows,
     // 128-byte swizzle; bytes 96.. belong to the next block or are zero fill) and
-    // the kSlots x 256 x_rot rows (rows past the last token are zero fill).
+    // the kSlots x 256 x_rot rows (rows past the last token are zero fill), each
+    // with its own barrier.  x_rot is written by the rotation kernel launched just
+    // before this one: the first ring's code tiles are requested before waiting
+    // for it.
     if (lane == 0) {
-      for (int b = 0; b < nbl; ++b) {
+      const int first = nbl < kStages ? nbl : kStages;
+      for (int b = 0; b < first; ++b) {
+        mbar_arrive_expect_tx(&codes_full[b], kCodeBytes);
+        tma_load_2d(ring + b * C_::kStageBytes, &tmap_codes, (b_lo + b) * 96, tile * kRows, &codes_full[b]);
+      }
+      wait_for_prerequisite_grid();
+      for (int b = 0; b < first; ++b) {
+        mbar_arrive_expect_tx(&x_full[b], C_::kXBytes);
+        tma_load_2d(ring + b * C_::kStageBytes + kCodeBytes, &tmap_x, (b_lo + b) * 256, 0, &x_full[b]);
+      }
+      for (int b = first; b < nbl; ++b) {
         const int s = b % kStages;
-        if (b >= kStages &&
-            !mbar_wait_bounded(&empty[s], ((b / kStages) & 1) ^ 1, max_polls, kDeadlineNs, abort_flag)) {
+        if (!mbar_wait_bounded(&empty[s], ((b / kStages) & 1) ^ 1, max_polls, kDeadlineNs, abort_flag)) {
           give_up();
           break;
         }
         uint8_t* st = ring + s * C_::kStageBytes;
-        mbar_arrive_expect_tx(&full[s], C_::kStageBytes);
-        tma_load_2d(st, &tmap_codes, (b_lo + b) * 96, tile * kRows, &full[s]);
-        tma_load_2d(st + kCodeBytes, &tmap_x, (b_lo + b) * 256, 0, &full[s]);
+        mbar_arrive_expect_tx(&codes_full[s], kCodeBytes);
+        tma_load_2d(st, &tmap_codes, (b_lo + b) * 96, tile * kRows, &codes_full[s]);
+        mbar_arrive_expect_tx(&x_full[s], C_::kXBytes);
+        tma_load_2d(st + kCodeBytes, &tmap_x, (b_lo + b) * 256, 0, &x_full[s]);
       }
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
     // Block b's operands are complete once the decode warps' barrier phase for it
-    // has passed: 16 MMAs (K = 16) into accumulator b & 1, then a commit.
+    // has passed: 16 MMAs (K = 16) into accumulator b % 3, then a commit.
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f16_f32(kRows, NT);
       for (int b = 0; b < nbl; ++b) {
@@ -262,13 +287,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t a0 = tmem + st * kACols;
-        const uint32_t d = tmem + kDCol0 + st * kDCols;
+        const uint32_t d = tmem + kDCol0 + (b % kDBufs) * kDCols;
         const uint64_t b0 = desc_kmajor_sw128(smem_u32(bst + st * C_::kBStageBytes));
 #pragma unroll
         for (int kk = 0; kk < 16; ++kk)
           mma_f16_tmem_a(d, a0 + 8 * kk, b0 + (kk >> 2) * (C_::kBBoxBytes >> 4) + 2 * (kk & 3), idesc,
                          kk ? 1u : 0u);
-        tc_commit(&mma_done[st]);
+        tc_commit(&mma_done[b % kDBufs]);
       }
     }
     __syncwarp();
@@ -279,65 +304,62 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int j = 0; j < kQ; ++j) acc[j] = 0.f;
 
-    // Adds block b's accumulator (this thread's row, its quarter of the token slots).
-    auto drain = [&](int b) {
-      if (!mbar_wait_bounded(&mma_done[b & 1], (b >> 1) & 1, max_polls, kDeadlineNs, abort_flag)) give_up();
-      tc_fence_after();
-      const uint32_t dcol = tmem + lane_base + kDCol0 + (b & 1) * kDCols + g * 2 * kQ;
-      float d[2 * kQ];
-      if constexpr (kQ == 4) {
-        uint32_t v[8];
-        tmem_ld_x8(dcol, v);
-        tmem_ld_wait();
+    if (g == 0) {
+      // this row's block scales, loaded together; first used two blocks from now
+      for (int b0 = 0; b0 < nbl; b0 += 8) {
+        __half hv[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) d[i] = __uint_as_float(v[i]);
-      } else {
-        uint32_t v[4];
-        tmem_ld_x4(dcol, v);
-        tmem_ld_wait();
+        for (int i = 0; i < 8; ++i)
+          hv[i] = b0 + i < nbl ? scales[static_cast<int64_t>(grow) * nb + b_lo + b0 + i] : __float2half(0.f);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) d[i] = __uint_as_float(v[i]);
+        for (int i = 0; i < 8; ++i)
+          if (b0 + i < nbl) s_tab[(b0 + i) * kRows + r] = __half2float(hv[i]);
       }
+    }
+
+    // Accumulator of block b: wait for its MMAs and start the TMEM load of this
+    // thread's row and quarter of the token slots; add() finishes it.
+    uint32_t dv[2 * kQ];
+    auto start_drain = [&](int b) {
+      if (!mbar_wait_bounded(&mma_done[b % kDBufs], (b / kDBufs) & 1, max_polls, kDeadlineNs, abort_flag))
+        give_up();
+      tc_fence_after();
+      const uint32_t dcol = tmem + lane_base + kDCol0 + (b % kDBufs) * kDCols + g * 2 * kQ;
+      if constexpr (kQ == 4) tmem_ld_x8(dcol, *reinterpret_cast<uint32_t(*)[8]>(dv));
+      else tmem_ld_x4(dcol, *reinterpret_cast<uint32_t(*)[4]>(dv));
+    };
+    auto add = [&](int b) {
       const float s = s_tab[b * kRows + r];
 #pragma unroll
       for (int j = 0; j < kQ; ++j)
-        acc[j] = fmaf(s * inv_tab[b * kSlots + g * kQ + j], d[2 * j] + d[2 * j + 1], acc[j]);
+        acc[j] = fmaf(s * inv_tab[b * kSlots + g * kQ + j], __uint_as_float(dv[2 * j]) + __uint_as_float(dv[2 * j + 1]),
+                      acc[j]);
     };
 
     // This thread's 24 code bytes start at byte 24g of its 96-byte row block: in
     // 16-byte chunks c0 = (24g) / 16 and c0 + 1, at word (24g % 16) / 4 of the pair.
     const int c0 = (24 * g) >> 4, wofs = ((24 * g) & 15) >> 2;
-    for (int b = 0; b < nbl; ++b) {
-      const int st = b & 1, s = b % kStages;
-      bool ok = mbar_wait_bounded(&full[s], (b / kStages) & 1, max_polls, kDeadlineNs, abort_flag);
+    uint32_t w[6];
+    auto load_codes = [&](int b) {
+      const int s = b % kStages;
+      const bool ok = mbar_wait_bounded(&codes_full[s], (b / kStages) & 1, max_polls, kDeadlineNs, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) give_up();
-      const uint8_t* stg = ring + s * C_::kStageBytes;
-      uint32_t W[8];
-      {
-        const uint8_t* row = stg + r * 128;
-        const uint4 u0 = *reinterpret_cast<const uint4*>(row + ((c0 ^ (r & 7)) << 4));
-        const uint4 u1 = *reinterpret_cast<const uint4*>(row + (((c0 + 1) ^ (r & 7)) << 4));
-        W[0] = u0.x; W[1] = u0.y; W[2] = u0.z; W[3] = u0.w;
-        W[4] = u1.x; W[5] = u1.y; W[6] = u1.z; W[7] = u1.w;
-      }
-      float xv[8];
-      if (slot < kSlots) {
-        const float4 a = *reinterpret_cast<const float4*>(stg + kCodeBytes + slot * 1024 + lane * 32);
-        const float4 c = *reinterpret_cast<const float4*>(stg + kCodeBytes + slot * 1024 + lane * 32 + 16);
-        xv[0] = a.x; xv[1] = a.y; xv[2] = a.z; xv[3] = a.w;
-        xv[4] = c.x; xv[5] = c.y; xv[6] = c.z; xv[7] = c.w;
-      }
-      // The next writer of this stage is the TMA engine: order these reads first.
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
-
-      // A: this row's codes 64g .. 64g + 63 -> levels in TMEM buffer st, columns 32g ..
-      // (block b - 2, the last reader of this buffer, finished before this thread's
-      // drain of it in the previous iteration returned).
-      uint32_t w[6];
+      const uint8_t* row = ring + s * C_::kStageBytes + r * 128;
+      const uint4 u0 = *reinterpret_cast<const uint4*>(row + ((c0 ^ (r & 7)) << 4));
+      const uint4 u1 = *reinterpret_cast<const uint4*>(row + (((c0 + 1) ^ (r & 7)) << 4));
+      const uint32_t W[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
 #pragma unroll
       for (int i = 0; i < 6; ++i) w[i] = wofs == 0 ? W[i] : (wofs == 2 ? W[i + 2] : W[i + 4]);
+    };
+
+    if (nbl > 0) load_codes(0);
+    for (int b = 0; b < nbl; ++b) {
+      const int st = b & 1, s = b % kStages;
+      // Block b - 2's MMAs, the last readers of A buffer and B stage st, are done
+      // once its accumulator is; its TMEM load overlaps the decode below.
+      if (b >= 2) start_drain(b - 2);
+
+      // A: this row's codes 64g .. 64g + 63 -> levels in TMEM buffer st, columns 32g ..
       const uint32_t acol = tmem + lane_base + st * kACols + 32 * g;
       {
         uint32_t lv0[16], lv1[16];
@@ -348,14 +370,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       // B: token slot t -> rows 2t (hi) and 2t + 1 (lo); lane l holds k-group l
       // (elements 8l .. 8l + 7): 128-byte box l / 8, 16-byte chunk l % 8 of the row.
-      uint8_t* bstage = bst + st * C_::kBStageBytes;
       if (slot < kSlots) {
-        const int t = slot;
+        const bool ok = mbar_wait_bounded(&x_full[s], (b / kStages) & 1, max_polls, kDeadlineNs, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) give_up();
+        const uint8_t* xs = ring + s * C_::kStageBytes + kCodeBytes + slot * 1024 + lane * 32;
+        const float4 xa = *reinterpret_cast<const float4*>(xs);
+        const float4 xb = *reinterpret_cast<const float4*>(xs + 16);
+        const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
         float m = 0.f;
 #pragma unroll
         for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(xv[i]));
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        // non-negative floats order like their bit patterns
+        m = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(m)));
         // m = 2^E * 1.f (normal: x_rot of fp16 inputs is 0 or >= 2^-28 in magnitude);
         // scale by 2^(14 - E), undo with 2^(E - 14).
         const uint32_t e = (__float_as_uint(m) >> 23) & 0xFFu;
@@ -364,27 +390,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t hw[4], lw[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const float u0 = xv[2 * i] * sc, u1 = xv[2 * i + 1] * sc;
-          const __half h0 = __float2half_rn(u0), h1 = __float2half_rn(u1);
-          const __half l0 = __float2half_rn(u0 - __half2float(h0)), l1 = __float2half_rn(u1 - __half2float(h1));
-          hw[i] = static_cast<uint32_t>(__half_as_ushort(h0)) | (static_cast<uint32_t>(__half_as_ushort(h1)) << 16);
-          lw[i] = static_cast<uint32_t>(__half_as_ushort(l0)) | (static_cast<uint32_t>(__half_as_ushort(l1)) << 16);
+          const float2 u = make_float2(xv[2 * i] * sc, xv[2 * i + 1] * sc);
+          const __half2 h = __float22half2_rn(u);
+          const float2 hf = __half22float2(h);
+          const __half2 l = __float22half2_rn(make_float2(u.x - hf.x, u.y - hf.y));
+          hw[i] = *reinterpret_cast<const uint32_t*>(&h);
+          lw[i] = *reinterpret_cast<const uint32_t*>(&l);
         }
-        uint8_t* box = bstage + (lane >> 3) * C_::kBBoxBytes;
-        const int n0 = 2 * t, n1 = 2 * t + 1;
+        uint8_t* box = bst + st * C_::kBStageBytes + (lane >> 3) * C_::kBBoxBytes;
+        const int n0 = 2 * slot, n1 = 2 * slot + 1;
         *reinterpret_cast<uint4*>(box + n0 * 128 + (((lane & 7) ^ (n0 & 7)) * 16)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
         *reinterpret_cast<uint4*>(box + n1 * 128 + (((lane & 7) ^ (n1 & 7)) * 16)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-        if (lane == 0) inv_tab[b * kSlots + t] = inv;
+        if (lane == 0) inv_tab[b * kSlots + slot] = inv;
       }
+      // This warp's reads of stage s are done (the TMA engine writes it next) and
+      // its B rows are written (the tensor cores read them): one proxy fence for both.
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
 
+      if (b + 1 < nbl) load_codes(b + 1);
+      if (b >= 2) {
+        tmem_ld_wait_regs(dv);
+        add(b - 2);
+      }
       tmem_st_wait();
-      fence_proxy_async_smem();                   // B is read by the tensor cores (async proxy)
       tc_fence_before();
       asm volatile("bar.sync 1, %0;" ::"n"(kDecThreads) : "memory");   // decode warps only
       if (tid == 0) mbar_arrive(&a_full[st]);
-      if (b > 0) drain(b - 1);
     }
-    if (nbl > 0) drain(nbl - 1);
+    for (int b = nbl >= 2 ? nbl - 2 : 0; b < nbl; ++b) {
+      start_drain(b);
+      tmem_ld_wait_regs(dv);
+      add(b);
+    }
 
     // Rank k of the cluster owns rows [k * 128 / C, (k + 1) * 128 / C): this CTA's
     // partial sums go straight into the owner's reduction buffer, slot [q][t][row].
@@ -494,13 +533,15 @@ int launch_tc(const uint8_t* codes, const __half* scales, const float* xrot, int
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = static_cast<unsigned>(ncl);
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // overlaps the rotation kernel
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   const int64_t polls = g_wait_limit_override > 0 ? g_wait_limit_override : kDefaultPolls;
   if (cudaLaunchKernelEx(&cfg, kern, mc, mx, scales, t, d_out, nb, nbl_max, y, polls) != cudaSuccess)
     return WUSH_ERR_CUDA;

@@ -533,8 +533,11 @@ def run_itq3(args):
             stream.synchronize()
             us = e0.elapsed_time(e1) / (reps * burst) * 1e3
             byts = codes.nbytes + scales.nbytes + t * d_in * 2 + t * d_out * 4
+            tc = mode == 1 and t >= 3 and d_out % 128 == 0
             print(json.dumps({"workload": f"itq3 W fp16 [{d_out}, {d_in}] 3-bit, {t} tokens",
                               "mode": "fused inverse FWHT" if mode == 0 else "activation-side rotation",
+                              "kernel": "itq3_tc_kernel (tcgen05, fp16 levels from TMEM)" if tc
+                              else "itq3_gemv_kernel (CUDA cores)",
                               "us": us, "GB_s": byts / us / 1e3, "frac_of_hbm": byts / us / 1e3 / peaks["hbm_gbs"],
                               "bytes_per_call": byts}))
 
