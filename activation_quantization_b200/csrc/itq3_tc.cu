@@ -226,7 +226,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) mbar_init(&a_full[i], 1);
     *abort_flag = 0;
     fence_barrier_init();
-    prefetch_tmap(&tmap_codes);
+    // The first ring's code tiles need nothing else: request them before the
+    // TMEM allocation and the CTA-wide barrier.
+    const int first = nbl < kStages ? nbl : kStages;
+    for (int b = 0; b < first; ++b) {
+      mbar_arrive_expect_tx(&codes_full[b], kCodeBytes);
+      tma_load_2d(ring + b * C_::kStageBytes, &tmap_codes, (b_lo + b) * 96, tile * kRows, &codes_full[b]);
+    }
     prefetch_tmap(&tmap_x);
   }
   if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
@@ -246,15 +252,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Block b -> ring stage b % kStages: the 128-row code tile (128-byte rows,
     // 128-byte swizzle; bytes 96.. belong to the next block or are zero fill) and
     // the kSlots x 256 x_rot rows (rows past the last token are zero fill), each
-    // with its own barrier.  x_rot is written by the rotation kernel launched just
-    // before this one: the first ring's code tiles are requested before waiting
-    // for it.
+    // with its own barrier.  Thread 0 has requested the first ring's code tiles;
+    // x_rot is written by the rotation kernel launched just before this one.
     if (lane == 0) {
       const int first = nbl < kStages ? nbl : kStages;
-      for (int b = 0; b < first; ++b) {
-        mbar_arrive_expect_tx(&codes_full[b], kCodeBytes);
-        tma_load_2d(ring + b * C_::kStageBytes, &tmap_codes, (b_lo + b) * 96, tile * kRows, &codes_full[b]);
-      }
       wait_for_prerequisite_grid();
       for (int b = 0; b < first; ++b) {
         mbar_arrive_expect_tx(&x_full[b], C_::kXBytes);
