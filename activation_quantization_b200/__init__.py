@@ -22,7 +22,7 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 FORMATS = {"mxfp4": 0, "nvfp4": 1, "int4": 2}
-TRANSFORMS = {"identity": 0, "hadamard": 1, "wus": 2, "wush": 3}
+TRANSFORMS = {"identity": 0, "hadamard": 1, "wus": 2, "wush": 3, "wush_diag": 4}
 IN_BF16, IN_FP32 = 0, 1
 
 _i64, _i32, _f32, _vp, _sz = ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t

@@ -1,4 +1,4 @@
-// Host-side calibration: per-block WUSH / WUS / Hadamard / identity transforms.
+// Host-side calibration: per-block WUSH / WUS / WUSH-diag / Hadamard / identity transforms.
 //
 // WUSH news article, paragraph 3: the transform combines the Cholesky factor of
 // the weights' second moment (W), the SVD components (U, S) and a Hadamard
@@ -10,6 +10,10 @@
 // W' = chol(Sigma_W), W'^T Sigma_X W' = U diag(lambda) U^T (cyclic Jacobi, fp64),
 // S = sqrt(lambda) descending, T_X = Hn S^{-1/2} U^T W'^T,
 // T_W = Hn S^{1/2} U^T W'^{-1} (Hn = H_b / sqrt(b); WUS drops Hn).
+// WUSH-diag (paragraphs 6 and 8: the data-aware component approximated by a
+// diagonal matrix) is the same construction on the moments' diagonals:
+// T_X = Hn D, T_W = Hn D^{-1}, D = diag((sigma_w,k / sigma_x,k)^{1/4}), each
+// diagonal floored at 1e-12 of its largest entry (1 if all are zero).
 // Runs in fp64 on the host's cores (OpenMP over blocks); not on the timed path.
 #include <cmath>
 #include <cstdint>
@@ -118,6 +122,22 @@ int block_pair(const double* sx, const double* sw, int b, int kind, float* tx, f
     for (int i = 0; i < bb; ++i) tx[i] = tw[i] = static_cast<float>(hn[i]);
     return WUSH_OK;
   }
+  if (kind == WUSH_T_WUSH_DIAG) {
+    double mx = 0.0, mw = 0.0;
+    for (int k = 0; k < b; ++k) {
+      mx = std::fmax(mx, sx[k * b + k]);
+      mw = std::fmax(mw, sw[k * b + k]);
+    }
+    const double fx = kEigFloor * (mx > 0 ? mx : 1.0), fw = kEigFloor * (mw > 0 ? mw : 1.0);
+    std::vector<double> d(b);
+    for (int k = 0; k < b; ++k) d[k] = std::pow(std::fmax(sw[k * b + k], fw) / std::fmax(sx[k * b + k], fx), 0.25);
+    for (int i = 0; i < b; ++i)
+      for (int j = 0; j < b; ++j) {
+        tx[i * b + j] = static_cast<float>(hn[i * b + j] * d[j]);
+        tw[i * b + j] = static_cast<float>(hn[i * b + j] / d[j]);
+      }
+    return WUSH_OK;
+  }
   std::vector<double> l(bb), linv(bb), m(bb), tmp(bb), u(bb), lam(b);
   if (!cholesky(sw, l.data(), b)) {
     double tr = 0.0;
@@ -224,8 +244,8 @@ extern "C" int wush_calibrate_from_moments(const double* sigma_x, const double* 
                                            int block, int kind, float* t_x, float* t_w) {
   if (!t_x || !t_w || !is_pow2(block) || block < 2 || block > 256 || d_in <= 0 || d_in % block)
     return WUSH_ERR_INVALID_ARG;
-  if (kind < WUSH_T_IDENTITY || kind > WUSH_T_WUSH) return WUSH_ERR_UNSUPPORTED;
-  if ((kind == WUSH_T_WUS || kind == WUSH_T_WUSH) && (!sigma_x || !sigma_w)) return WUSH_ERR_INVALID_ARG;
+  if (kind < WUSH_T_IDENTITY || kind > WUSH_T_WUSH_DIAG) return WUSH_ERR_UNSUPPORTED;
+  if (kind >= WUSH_T_WUS && (!sigma_x || !sigma_w)) return WUSH_ERR_INVALID_ARG;
   const int64_t nb = d_in / block, bb = static_cast<int64_t>(block) * block;
   int status = WUSH_OK;
 #pragma omp parallel for schedule(dynamic, 1)
@@ -245,7 +265,7 @@ extern "C" int wush_calibrate(const float* x_calib, int64_t n_calib, const float
                               int64_t d_in, int block, int kind, float* t_x, float* t_w) {
   if (!t_x || !t_w || !is_pow2(block) || block < 2 || block > 256 || d_in <= 0 || d_in % block)
     return WUSH_ERR_INVALID_ARG;
-  if (kind < WUSH_T_IDENTITY || kind > WUSH_T_WUSH) return WUSH_ERR_UNSUPPORTED;
+  if (kind < WUSH_T_IDENTITY || kind > WUSH_T_WUSH_DIAG) return WUSH_ERR_UNSUPPORTED;
   if (kind == WUSH_T_IDENTITY || kind == WUSH_T_HADAMARD)
     return wush_calibrate_from_moments(nullptr, nullptr, d_in, block, kind, t_x, t_w);
   if (!x_calib || !w || n_calib <= 0 || d_out <= 0) return WUSH_ERR_INVALID_ARG;

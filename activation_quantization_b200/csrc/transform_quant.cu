@@ -275,9 +275,10 @@ int launch_fmt(const void* x, bool xf32, int64_t rows, int64_t d_in, const float
 int check_common(const void* x, int x_dtype, int64_t rows, int64_t d_in, const float* t, int kind, int b) {
   if (rows < 0 || d_in <= 0 || d_in % b) return WUSH_ERR_INVALID_ARG;
   if (x_dtype != WUSH_IN_BF16 && x_dtype != WUSH_IN_FP32) return WUSH_ERR_UNSUPPORTED;
-  if (kind < WUSH_T_IDENTITY || kind > WUSH_T_WUSH) return WUSH_ERR_UNSUPPORTED;
+  if (kind < WUSH_T_IDENTITY || kind > WUSH_T_WUSH_DIAG) return WUSH_ERR_UNSUPPORTED;
   if (rows > 0 && (!x || !aligned16(x))) return WUSH_ERR_INVALID_ARG;
-  if ((kind == WUSH_T_WUS || kind == WUSH_T_WUSH) && (!t || !aligned16(t))) return WUSH_ERR_INVALID_ARG;
+  // WUS, WUSH and WUSH-diag are applied as dense per-block matrices
+  if (kind >= WUSH_T_WUS && (!t || !aligned16(t))) return WUSH_ERR_INVALID_ARG;
   if ((d_in / b + kBlocksPerCta - 1) / kBlocksPerCta > 65535) return WUSH_ERR_UNSUPPORTED;
   if ((rows + kRowsPerCta - 1) / kRowsPerCta > 0x7FFFFFFF) return WUSH_ERR_UNSUPPORTED;
   return WUSH_OK;

@@ -266,7 +266,9 @@ def run_gpu(args, rank, world):
 
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
-    spec = WORKLOADS[args.workload]
+    spec = dict(WORKLOADS[args.workload])
+    if args.transform:
+        spec["kind"] = args.transform
     fmt, kind = spec["fmt"], spec["kind"]
     w, x, wt, xc = build_inputs(args.workload, args.tokens)
     M, N, K = w.tokens, w.d_out, w.d_in
@@ -552,6 +554,8 @@ def main():
     ap.add_argument("--impl", default="wush", choices=["wush", "reference"])
     ap.add_argument("--workload", default="up_proj", choices=sorted(WORKLOADS) + ["itq3"])
     ap.add_argument("--tokens", type=int, default=None, help="override the workload's token count")
+    ap.add_argument("--transform", default=None, choices=["identity", "hadamard", "wus", "wush", "wush_diag"],
+                    help="override the workload's block transform (calibrated from the same tokens)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -561,7 +565,9 @@ def main():
         if rank == 0:               # a per-call latency benchmark: one rank times it
             run_itq3(args)
         return
-    spec = WORKLOADS[args.workload]
+    spec = dict(WORKLOADS[args.workload])
+    if args.transform:
+        spec["kind"] = args.transform
 
     if args.impl == "reference":
         if rank != 0:

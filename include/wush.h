@@ -62,7 +62,8 @@ typedef enum {
   WUSH_T_IDENTITY = 0,
   WUSH_T_HADAMARD = 1,
   WUSH_T_WUS = 2,
-  WUSH_T_WUSH = 3
+  WUSH_T_WUSH = 3,
+  WUSH_T_WUSH_DIAG = 4
 } wush_transform;
 
 typedef enum { WUSH_IN_BF16 = 0, WUSH_IN_FP32 = 1 } wush_input_dtype;
@@ -85,6 +86,11 @@ int wush_block_size(int fmt);
  *   S = diag(sqrt(lambda)) (descending),  Hn = H_b / sqrt(b),
  *   T_X = Hn S^{-1/2} U^T W'^T,   T_W = T_X^{-T} = Hn S^{1/2} U^T W'^{-1}.
  * WUS drops Hn; HADAMARD gives T_X = T_W = Hn; IDENTITY gives I.
+ * WUSH_DIAG (paragraphs 6 and 8: the data-aware component approximated by a
+ * diagonal matrix) runs the same construction on the diagonals of the two
+ * moments, which gives T_X = Hn D, T_W = Hn D^{-1} with
+ * D = diag((Sigma_W[k][k] / Sigma_X[k][k])^{1/4}); each diagonal is floored at
+ * 1e-12 of its largest entry (1 if all are zero).  It applies like WUSH (dense T).
  * Columns of U are signed so that their largest-magnitude entry is positive
  * (ties: lowest index); eigenvalues are floored at 1e-12 * max.  A Cholesky
  * failure is retried once with Sigma_W + 1e-8 * mean(diag) I; if that fails
@@ -140,7 +146,7 @@ size_t wush_scales_bytes(int64_t rows, int64_t d_in, int fmt);
  *   sign of y even when the magnitude rounds to 0; an all-zero block gives +0.
  *
  * x:       device [rows, d_in], bf16 (x_dtype = WUSH_IN_BF16) or fp32.
- * t:       device fp32 [d_in/b, b, b] for WUS/WUSH; ignored (may be NULL) for
+ * t:       device fp32 [d_in/b, b, b] for WUS/WUSH/WUSH_DIAG; ignored (may be NULL) for
  *          IDENTITY and HADAMARD (computed with in-register butterflies, then
  *          scaled by the fp32 constant 1/sqrt(b)).
  * codes:   device, wush_codes_bytes(rows, d_in, fmt) bytes.

@@ -31,6 +31,16 @@ Conventions the pages leave open: eigenvalues in descending order; each column
 of U is negated if needed so that its largest-magnitude entry is positive (ties
 to the lowest index); eigenvalues are floored at 1e-12 * max(lambda); a failed
 Cholesky is retried once on Sigma_W + 1e-8 * mean(diag(Sigma_W)) I.
+
+"wush_diag" is the simplification the WUSH news article offers for costly or
+constrained deployments (paragraphs 6 and 8: approximate the data-aware component
+by a diagonal matrix).  Reading: the same construction run on the diagonals of
+the two moments.  Then W' = diag(sqrt(sigma_w)), W'^T Sigma_X W' is diagonal, U
+is the identity (no reordering), and
+    T_X = Hn D,   T_W = Hn D^(-1),   D = diag((sigma_w,k / sigma_x,k)^(1/4)),
+so T_W^T T_X = I still holds and the diagonal moments balance:
+T_X diag(Sigma_X) T_X^T = T_W diag(Sigma_W) T_W^T = Hn diag(sqrt(sigma_x sigma_w)) Hn^T.
+Each diagonal is floored at 1e-12 times its largest entry (1 if all are zero).
 """
 from __future__ import annotations
 
@@ -38,7 +48,7 @@ import numpy as np
 
 from .transforms import normalized_hadamard
 
-KINDS = ("identity", "hadamard", "wus", "wush")
+KINDS = ("identity", "hadamard", "wus", "wush", "wush_diag")
 
 
 class NotPositiveDefinite(ValueError):
@@ -81,6 +91,13 @@ def _sorted_eig(m: np.ndarray):
     return lam, u
 
 
+def _floored_diag(sigma: np.ndarray) -> np.ndarray:
+    """Diagonal of a second moment, floored at 1e-12 of its largest entry."""
+    d = np.diag(np.asarray(sigma, dtype=np.float64)).copy()
+    top = d.max() if d.max() > 0 else 1.0
+    return np.maximum(d, 1e-12 * top)
+
+
 def block_transform_pair(sigma_x: np.ndarray, sigma_w: np.ndarray, kind: str):
     """(T_X, T_W) for one b x b block from its two second moments, fp64."""
     b = sigma_x.shape[0]
@@ -89,6 +106,9 @@ def block_transform_pair(sigma_x: np.ndarray, sigma_w: np.ndarray, kind: str):
     hn = normalized_hadamard(b)
     if kind == "hadamard":
         return hn.copy(), hn.copy()
+    if kind == "wush_diag":
+        d = (_floored_diag(sigma_w) / _floored_diag(sigma_x)) ** 0.25
+        return hn @ np.diag(d), hn @ np.diag(1.0 / d)
     if kind not in ("wus", "wush"):
         raise ValueError(kind)
     wp = _cholesky(sigma_w)

@@ -23,7 +23,7 @@ def tiny_layer_losses():
     wt = synth.weights(w)
     out = {}
     for fmt, b in (("mxfp4", 32), ("nvfp4", 16), ("int4", 32)):
-        for kind in ("identity", "hadamard", "wus", "wush"):
+        for kind in ("identity", "hadamard", "wus", "wush", "wush_diag"):
             tx, tw = calibrate.calibrate(xc, wt, b, kind)
             tx32, tw32 = tx.astype(np.float32), tw.astype(np.float32)
             gs = None

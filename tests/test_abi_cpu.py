@@ -30,7 +30,7 @@ def test_every_declared_symbol_is_exported():
     assert set(names) <= set(aq._SIGNATURES), "binding lacks a signature"
 
 
-@pytest.mark.parametrize("kind", ["identity", "hadamard", "wus", "wush"])
+@pytest.mark.parametrize("kind", ["identity", "hadamard", "wus", "wush", "wush_diag"])
 def test_calibrate_matches_oracle(kind):
     w = synth.WORKLOADS["tiny"]
     xc, wt = synth.activations(w, calib=True), synth.weights(w)

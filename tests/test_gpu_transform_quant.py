@@ -66,7 +66,7 @@ def run_gpu_t(lib, xt_cpu, t, kind, fmt, gs):
             P.decode_scales(scales.cpu().numpy(), rows, d_in, fmt), y.cpu().numpy())
 
 
-@pytest.mark.parametrize("kind", ["identity", "hadamard", "wus", "wush"])
+@pytest.mark.parametrize("kind", ["identity", "hadamard", "wus", "wush", "wush_diag"])
 def test_tiny_fp32_mxfp4(lib, kind):
     w = synth.WORKLOADS["tiny"]
     x = synth.activations(w)
@@ -77,7 +77,7 @@ def test_tiny_fp32_mxfp4(lib, kind):
 
 
 @pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4", "int4"])
-@pytest.mark.parametrize("kind", ["identity", "hadamard", "wus", "wush"])
+@pytest.mark.parametrize("kind", ["identity", "hadamard", "wus", "wush", "wush_diag"])
 def test_ragged_rows_bf16(lib, fmt, kind):
     # 300 rows: two full 128-row tiles and a ragged tail; the full d_in of the workload
     w = synth.WORKLOADS[FMT_WORKLOAD[fmt]]

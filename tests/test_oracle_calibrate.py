@@ -116,3 +116,57 @@ def test_tiny_losses_regression_and_claims():
     for kind in ("wus", "wush"):
         assert gold[f"nvfp4/{kind}"] < min(gold["nvfp4/identity"], gold["nvfp4/hadamard"])
     assert gold["int4/wush"] < 0.2 * gold["int4/identity"]
+    # The diagonal approximation (paragraphs 6 and 8 offer it as a simplification)
+    # keeps most of the gain on this layer, whose channels are independent with a
+    # few large ones; the pages print no number for it.
+    for fmt in ("mxfp4", "nvfp4", "int4"):
+        assert gold[f"{fmt}/wush_diag"] < min(gold[f"{fmt}/identity"], gold[f"{fmt}/hadamard"])
+        assert gold[f"{fmt}/wush_diag"] < 1.1 * gold[f"{fmt}/wush"]
+
+
+def test_wush_diag_two_by_two_closed_form():
+    # b = 2, Sigma_X = diag(16, 1), Sigma_W = diag(1, 16): D = diag((1/16)^(1/4), 16^(1/4))
+    # = diag(0.5, 2) and Hn = [[1, 1], [1, -1]] / sqrt(2); the off-diagonal moment
+    # entries play no part in the diagonal variant.
+    r = 1 / np.sqrt(2)
+    want_x = r * np.array([[0.5, 2.0], [0.5, -2.0]])
+    want_w = r * np.array([[2.0, 0.5], [2.0, -0.5]])
+    for off in (0.0, 0.7):
+        sx = np.array([[16.0, off], [off, 1.0]])
+        sw = np.array([[1.0, -off], [-off, 16.0]])
+        tx, tw = C.block_transform_pair(sx, sw, "wush_diag")
+        assert np.allclose(tx, want_x, atol=1e-15) and np.allclose(tw, want_w, atol=1e-15)
+
+
+def test_wush_diag_is_wush_on_diagonal_moments():
+    # With diagonal moments whose products sigma_x * sigma_w already descend, the
+    # full construction (Cholesky, eigendecomposition, sign convention) has U = I
+    # and reduces to the diagonal variant.
+    rng = np.random.default_rng(7)
+    b = 32
+    prod = np.sort(rng.uniform(0.1, 50.0, b))[::-1]
+    sw_d = rng.uniform(0.01, 3.0, b)
+    sx_d = prod / sw_d
+    full = C.block_transform_pair(np.diag(sx_d), np.diag(sw_d), "wush")
+    diag = C.block_transform_pair(np.diag(sx_d), np.diag(sw_d), "wush_diag")
+    for a, d in zip(full, diag):
+        assert np.allclose(a, d, rtol=1e-12, atol=1e-12)
+
+
+def test_wush_diag_inverse_transpose_and_balanced_diagonals():
+    x, w, sx, sw = _moments(5)
+    tx, tw = C.block_transform_pair(sx, sw, "wush_diag")
+    assert np.allclose(tw.T @ tx, np.eye(32), atol=1e-12)
+    assert np.allclose((tw @ w.T).T @ (tx @ x.T), w @ x.T, rtol=1e-9, atol=1e-9)
+    dx, dw = np.diag(np.diag(sx)), np.diag(np.diag(sw))
+    assert np.allclose(tx @ dx @ tx.T, tw @ dw @ tw.T, rtol=1e-10, atol=1e-12)
+
+
+def test_wush_diag_floors_dead_channels():
+    sx = np.diag([4.0, 0.0, 1.0, 2.0])
+    sw = np.diag([1.0, 1.0, 0.0, 3.0])
+    tx, tw = C.block_transform_pair(sx, sw, "wush_diag")
+    assert np.isfinite(tx).all() and np.isfinite(tw).all()
+    assert np.allclose(tw.T @ tx, np.eye(4), atol=1e-9)
+    tx0, tw0 = C.block_transform_pair(np.zeros((4, 4)), np.zeros((4, 4)), "wush_diag")
+    assert np.allclose(tx0, T.normalized_hadamard(4)) and np.allclose(tw0, T.normalized_hadamard(4))
