@@ -36,7 +36,9 @@ _SIGNATURES = {
     "wush_scales_bytes": (_sz, [_i64, _i64, _i32]),
     "wush_transform_quant": (_i32, [_vp, _i32, _i64, _i64, _vp, _i32, _i32, _f32, _vp, _vp, _vp, _vp]),
     "wush_transform_amax": (_i32, [_vp, _i32, _i64, _i64, _vp, _i32, _i32, _vp, _vp]),
+    "wush_transform_quant_nvfp4_dynamic": (_i32, [_vp, _i32, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp]),
     "wush_qgemm": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _f32, _vp, _vp]),
+    "wush_qgemm_nvfp4_dynamic": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _f32, _vp, _vp]),
     "wush_qgemm_int4": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp]),
     "wush_qgemm_int4_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "wush_qgemm_int4_ws": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _sz, _vp, _vp]),
@@ -179,6 +181,30 @@ def wush_transform_amax(x, t, kind, block: int, amax_out, stream=None):
     _check("wush_transform_amax",
            _lib.wush_transform_amax(_ptr(x), x_dtype, rows, d_in, _ptr(t), _enum(TRANSFORMS, kind), block,
                                     _ptr(amax_out), _stream(stream)))
+
+
+def wush_transform_quant_nvfp4_dynamic(x, t, kind, amax, codes, scales, global_scale_out=None, y_debug=None,
+                                       stream=None):
+    """NVFP4 transform + quantisation whose per-tensor scale is derived on the device from
+    ``amax`` (a CUDA fp32 scalar, e.g. from wush_transform_amax); the scale is written to
+    ``global_scale_out`` (CUDA fp32 scalar) if given."""
+    import torch
+    x_dtype = IN_FP32 if x.dtype == torch.float32 else IN_BF16
+    if x.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("x must be bf16 or fp32")
+    rows, d_in = x.shape
+    _check("wush_transform_quant_nvfp4_dynamic",
+           _lib.wush_transform_quant_nvfp4_dynamic(_ptr(x), x_dtype, rows, d_in, _ptr(t), _enum(TRANSFORMS, kind),
+                                                   _ptr(amax), _ptr(global_scale_out), _ptr(codes), _ptr(scales),
+                                                   _ptr(y_debug), _stream(stream)))
+
+
+def wush_qgemm_nvfp4_dynamic(a_codes, a_scales, b_codes, b_scales, M: int, N: int, K: int, a_global_scale,
+                             b_global_scale: float, y, stream=None):
+    """NVFP4 GEMM with alpha = *a_global_scale (CUDA fp32 scalar) * b_global_scale, formed on the device."""
+    _check("wush_qgemm_nvfp4_dynamic",
+           _lib.wush_qgemm_nvfp4_dynamic(_ptr(a_codes), _ptr(a_scales), _ptr(b_codes), _ptr(b_scales), M, N, K,
+                                         _ptr(a_global_scale), float(b_global_scale), _ptr(y), _stream(stream)))
 
 
 def wush_qgemm(a_codes, a_scales, b_codes, b_scales, M: int, N: int, K: int, fmt, alpha: float, y,

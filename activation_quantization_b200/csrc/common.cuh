@@ -26,8 +26,13 @@ int read_and_clear_itq3_tc_error(int* word);
 
 // Tensor-core form of wush_transform_quant (bf16 inputs); WUSH_ERR_UNSUPPORTED
 // for shapes it does not take.
+// gs_amax (device, optional): NVFP4 takes its per-tensor scale from this amax
+// (nvfp4_dynamic_scale) instead of gscale, and CTA 0 writes it to gs_out if given.
+int transform_amax_tc(const void* x, int64_t rows, int64_t d_in, const float* t, int kind, int block,
+                      float* amax_out, cudaStream_t st);
 int transform_quant_tc(const void* x, int64_t rows, int64_t d_in, const float* t, int kind, int fmt,
-                       float gscale, uint8_t* codes, void* scales, float* ydbg, cudaStream_t st);
+                       float gscale, const float* gs_amax, float* gs_out, uint8_t* codes, void* scales, float* ydbg,
+                       cudaStream_t st);
 
 // GEMM kernel choice (see wush_debug_set_gemm_variant).
 extern int g_gemm_variant;
@@ -63,6 +68,15 @@ inline int set_smem_once(Kernel kernel, int bytes, std::atomic<uint64_t>& done) 
     return WUSH_ERR_CUDA;
   if (bit) done.fetch_or(bit, std::memory_order_acq_rel);
   return WUSH_OK;
+}
+
+// Dynamic NVFP4 per-tensor scale from the device amax of the transformed tensor:
+// s_g = fp32(amax / 2688), 2688 = 6 * 448 (largest E2M1 magnitude times largest
+// UE4M3 block scale); 1 when that is below 1e-30 (an all-zero or denormal tensor,
+// whose codes are zero whatever the scale).
+__device__ __forceinline__ float nvfp4_dynamic_scale(float amax) {
+  const float g = __fdiv_rn(amax, 2688.0f);
+  return g >= 1e-30f ? g : 1.0f;
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }

@@ -92,8 +92,8 @@ template <int BN, bool NV>
 __global__ void __launch_bounds__(kThreads, 1)
     qgemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                  const uint8_t* __restrict__ sfa, const uint8_t* __restrict__ sfb,
-                 const __grid_constant__ CUtensorMap tmap_y, int M, int N, int K, float alpha, int64_t max_polls,
-                 int debug_never) {
+                 const __grid_constant__ CUtensorMap tmap_y, int M, int N, int K, float alpha,
+                 const float* __restrict__ alpha_scale, int64_t max_polls, int debug_never) {
   using C = Cfg<BN, NV>;
   constexpr int kStages = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -229,6 +229,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ew = warp - 2;
     const int q = warp & 3;
     const int half = ew / 4;
+    // alpha times the device factor (a per-tensor scale computed on the device)
+    const float alpha_eff = alpha_scale ? __fmul_rn(__ldg(alpha_scale), alpha) : alpha;
     uint8_t* bufs = epi_smem + ew * C::kEpiBufs * kEpiChunkBytes;
     int buf = 0, tcount = 0;
     for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++tcount) {
@@ -256,8 +258,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int j = 0; j < 8; ++j)
           *reinterpret_cast<float4*>(sb + lane * 128 + ((j ^ (lane & 7)) * 16)) =
-              make_float4(alpha * __uint_as_float(r[c][4 * j]), alpha * __uint_as_float(r[c][4 * j + 1]),
-                          alpha * __uint_as_float(r[c][4 * j + 2]), alpha * __uint_as_float(r[c][4 * j + 3]));
+              make_float4(alpha_eff * __uint_as_float(r[c][4 * j]), alpha_eff * __uint_as_float(r[c][4 * j + 1]),
+                          alpha_eff * __uint_as_float(r[c][4 * j + 2]), alpha_eff * __uint_as_float(r[c][4 * j + 3]));
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -333,7 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     qgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                       const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
                       const __grid_constant__ CUtensorMap tmap_y, int M, int N, int K, float alpha,
-                      int64_t max_polls, int debug_never) {
+                      const float* __restrict__ alpha_scale, int64_t max_polls, int debug_never) {
   using C = Cfg2<NV>;
   constexpr int kSt = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -462,6 +464,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     const int ew = warp - 2, q = warp & 3, half = ew / 4;
+    // alpha times the device factor (a per-tensor scale computed on the device)
+    const float alpha_eff = alpha_scale ? __fmul_rn(__ldg(alpha_scale), alpha) : alpha;
     const uint32_t leader_acc_empty = mapa_shared(smem_u32(acc_empty), 0);
     uint8_t* sbuf = epi_smem + ew * 32 * C::kEpiCols * 4;
     int tcount = 0;
@@ -490,16 +494,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 8; ++j)
               *reinterpret_cast<float4*>(sbuf + lane * 128 + ((j ^ (lane & 7)) * 16)) =
-                  make_float4(alpha * __uint_as_float(r[c][4 * j]), alpha * __uint_as_float(r[c][4 * j + 1]),
-                              alpha * __uint_as_float(r[c][4 * j + 2]), alpha * __uint_as_float(r[c][4 * j + 3]));
+                  make_float4(alpha_eff * __uint_as_float(r[c][4 * j]), alpha_eff * __uint_as_float(r[c][4 * j + 1]),
+                              alpha_eff * __uint_as_float(r[c][4 * j + 2]), alpha_eff * __uint_as_float(r[c][4 * j + 3]));
           } else {
             // 32-byte rows, one per lane: the warp writes one contiguous kilobyte
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
               const int e = sc * 8 + 4 * j;
               *reinterpret_cast<float4*>(sbuf + lane * 32 + j * 16) =
-                  make_float4(alpha * __uint_as_float(r[c][e]), alpha * __uint_as_float(r[c][e + 1]),
-                              alpha * __uint_as_float(r[c][e + 2]), alpha * __uint_as_float(r[c][e + 3]));
+                  make_float4(alpha_eff * __uint_as_float(r[c][e]), alpha_eff * __uint_as_float(r[c][e + 1]),
+                              alpha_eff * __uint_as_float(r[c][e + 2]), alpha_eff * __uint_as_float(r[c][e + 3]));
             }
           }
           fence_proxy_async_smem();
@@ -585,7 +589,7 @@ bool make_sf_map(CUtensorMap* map, const void* base, int64_t bytes, int box_rows
 
 template <bool NV>
 int launch_pair(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const uint8_t* sfb, int64_t M, int64_t N,
-                int64_t K, float alpha, float* y, cudaStream_t st) {
+                int64_t K, float alpha, const float* alpha_scale, float* y, cudaStream_t st) {
   using C = Cfg2<NV>;
   const int64_t n_acols = (K / (NV ? 16 : 32) + 3) / 4;
   CUtensorMap ma, mb, msa, msb, my;
@@ -616,14 +620,14 @@ int launch_pair(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const ui
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, kern, ma, mb, msa, msb, my, static_cast<int>(M), static_cast<int>(N),
-                         static_cast<int>(K), alpha, polls, debug_never) != cudaSuccess)
+                         static_cast<int>(K), alpha, alpha_scale, polls, debug_never) != cudaSuccess)
     return WUSH_ERR_CUDA;
   return launch_status();
 }
 
 template <int BN, bool NV>
 int launch(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const uint8_t* sfb, int64_t M, int64_t N,
-           int64_t K, float alpha, float* y, cudaStream_t st) {
+           int64_t K, float alpha, const float* alpha_scale, float* y, cudaStream_t st) {
   using C = Cfg<BN, NV>;
   CUtensorMap ma, mb, my;
   if (!make_map(&ma, a, M, K / 2, kBM) || !make_map(&mb, b, N, K / 2, BN) || !make_y_map(&my, y, M, N, 32))
@@ -638,7 +642,7 @@ int launch(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const uint8_t
   if (sms <= 0) return WUSH_ERR_CUDA;
   const dim3 grid(static_cast<unsigned>(n_tiles < sms ? n_tiles : sms));
   kern<<<grid, kThreads, C::kSmemBytes, st>>>(ma, mb, sfa, sfb, my, static_cast<int>(M), static_cast<int>(N),
-                                              static_cast<int>(K), alpha, polls, debug_never);
+                                              static_cast<int>(K), alpha, alpha_scale, polls, debug_never);
   return launch_status();
 }
 
@@ -647,9 +651,10 @@ int launch(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const uint8_t
 
 using namespace wush;
 
-extern "C" int wush_qgemm(const uint8_t* a_codes, const void* a_scales, const uint8_t* b_codes,
-                          const void* b_scales, int64_t M, int64_t N, int64_t K, int fmt, float alpha, float* y,
-                          void* stream) {
+namespace {
+
+int qgemm_impl(const uint8_t* a_codes, const void* a_scales, const uint8_t* b_codes, const void* b_scales, int64_t M,
+               int64_t N, int64_t K, int fmt, float alpha, const float* alpha_scale, float* y, void* stream) {
   if (fmt != WUSH_FMT_MXFP4 && fmt != WUSH_FMT_NVFP4) return WUSH_ERR_UNSUPPORTED;
   if (M <= 0 || N <= 0 || K <= 0 || M % 128 || N % 128 || K % 256) return WUSH_ERR_INVALID_ARG;
   if (M > (int64_t(1) << 30) || N > (int64_t(1) << 30) || K > (int64_t(1) << 30) || N / 128 > 65535 * 128)
@@ -662,14 +667,31 @@ extern "C" int wush_qgemm(const uint8_t* a_codes, const void* a_scales, const ui
   const auto* sb = static_cast<const uint8_t*>(b_scales);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool nv = fmt == WUSH_FMT_NVFP4;
+  const float* as = alpha_scale;
   if (M % 256 == 0 && N % 256 == 0 && g_gemm_variant == 0) {
-    return nv ? launch_pair<true>(a_codes, sa, b_codes, sb, M, N, K, alpha, y, st)
-              : launch_pair<false>(a_codes, sa, b_codes, sb, M, N, K, alpha, y, st);
+    return nv ? launch_pair<true>(a_codes, sa, b_codes, sb, M, N, K, alpha, as, y, st)
+              : launch_pair<false>(a_codes, sa, b_codes, sb, M, N, K, alpha, as, y, st);
   }
   if (N % 256 == 0 && g_gemm_variant != 2) {
-    return nv ? launch<256, true>(a_codes, sa, b_codes, sb, M, N, K, alpha, y, st)
-              : launch<256, false>(a_codes, sa, b_codes, sb, M, N, K, alpha, y, st);
+    return nv ? launch<256, true>(a_codes, sa, b_codes, sb, M, N, K, alpha, as, y, st)
+              : launch<256, false>(a_codes, sa, b_codes, sb, M, N, K, alpha, as, y, st);
   }
-  return nv ? launch<128, true>(a_codes, sa, b_codes, sb, M, N, K, alpha, y, st)
-            : launch<128, false>(a_codes, sa, b_codes, sb, M, N, K, alpha, y, st);
+  return nv ? launch<128, true>(a_codes, sa, b_codes, sb, M, N, K, alpha, as, y, st)
+            : launch<128, false>(a_codes, sa, b_codes, sb, M, N, K, alpha, as, y, st);
+}
+
+}  // namespace
+
+extern "C" int wush_qgemm(const uint8_t* a_codes, const void* a_scales, const uint8_t* b_codes,
+                          const void* b_scales, int64_t M, int64_t N, int64_t K, int fmt, float alpha, float* y,
+                          void* stream) {
+  return qgemm_impl(a_codes, a_scales, b_codes, b_scales, M, N, K, fmt, alpha, nullptr, y, stream);
+}
+
+extern "C" int wush_qgemm_nvfp4_dynamic(const uint8_t* a_codes, const void* a_scales, const uint8_t* b_codes,
+                                        const void* b_scales, int64_t M, int64_t N, int64_t K,
+                                        const float* a_global_scale, float b_global_scale, float* y, void* stream) {
+  if (!a_global_scale || (reinterpret_cast<uintptr_t>(a_global_scale) & 3u)) return WUSH_ERR_INVALID_ARG;
+  return qgemm_impl(a_codes, a_scales, b_codes, b_scales, M, N, K, WUSH_FMT_NVFP4, b_global_scale, a_global_scale,
+                    y, stream);
 }

@@ -126,9 +126,15 @@ __device__ __forceinline__ void dense_apply(const float* __restrict__ tj, const 
 
 template <int B, int KIND, int FMT, bool XF32, bool DBG>
 __global__ void __launch_bounds__(kRowsPerCta) transform_quant_kernel(
-    const void* __restrict__ x, int64_t rows, int64_t d_in, const float* __restrict__ t, float gscale,
-    uint8_t* __restrict__ codes, void* __restrict__ scales, float* __restrict__ ydbg,
-    float* __restrict__ amax_out) {
+    const void* __restrict__ x, int64_t rows, int64_t d_in, const float* __restrict__ t, float gscale_arg,
+    const float* __restrict__ gs_amax, float* __restrict__ gs_out, uint8_t* __restrict__ codes,
+    void* __restrict__ scales, float* __restrict__ ydbg, float* __restrict__ amax_out) {
+  // NVFP4 per-tensor scale: the caller's, or derived from a device amax
+  float gscale = gscale_arg;
+  if (FMT == kNv && gs_amax) {
+    gscale = nvfp4_dynamic_scale(__ldg(gs_amax));
+    if (gs_out && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *gs_out = gscale;
+  }
   constexpr int CH = kBlocksPerCta;
   __shared__ __align__(16) float s_t[KIND == kDense ? CH * B * B : 4];
   __shared__ __align__(16) uint8_t s_sf[512];
@@ -244,14 +250,15 @@ __global__ void __launch_bounds__(kRowsPerCta) transform_quant_kernel(
 
 template <int B, int FMT>
 int launch_fmt(const void* x, bool xf32, int64_t rows, int64_t d_in, const float* t, int kind, float gscale,
-               uint8_t* codes, void* scales, float* ydbg, float* amax_out, cudaStream_t st) {
+               uint8_t* codes, void* scales, float* ydbg, float* amax_out, cudaStream_t st,
+               const float* gs_amax = nullptr, float* gs_out = nullptr) {
   const dim3 grid(static_cast<unsigned>((rows + kRowsPerCta - 1) / kRowsPerCta),
                   static_cast<unsigned>((d_in / B + kBlocksPerCta - 1) / kBlocksPerCta));
   const dim3 block(kRowsPerCta);
   const int k = kind == WUSH_T_IDENTITY ? kIdentity : (kind == WUSH_T_HADAMARD ? kHadamard : kDense);
 #define WUSH_TQ_LAUNCH(KK, XF, DB)                                                                \
-  transform_quant_kernel<B, KK, FMT, XF, DB><<<grid, block, 0, st>>>(x, rows, d_in, t, gscale, codes, \
-                                                                     scales, ydbg, amax_out)
+  transform_quant_kernel<B, KK, FMT, XF, DB><<<grid, block, 0, st>>>(x, rows, d_in, t, gscale, gs_amax, \
+                                                                     gs_out, codes, scales, ydbg, amax_out)
 #define WUSH_TQ_KIND(XF, DB)                       \
   do {                                             \
     if (k == kIdentity) WUSH_TQ_LAUNCH(kIdentity, XF, DB); \
@@ -320,7 +327,8 @@ extern "C" int wush_transform_quant(const void* x, int x_dtype, int64_t rows, in
   const bool xf32 = x_dtype == WUSH_IN_FP32;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (!xf32) {
-    const int tc = transform_quant_tc(x, rows, d_in, t, kind, fmt, global_scale, codes, scales, y_debug, s);
+    const int tc =
+        transform_quant_tc(x, rows, d_in, t, kind, fmt, global_scale, nullptr, nullptr, codes, scales, y_debug, s);
     if (tc != WUSH_ERR_UNSUPPORTED) return tc;
   }
   if (fmt == WUSH_FMT_MXFP4)
@@ -328,6 +336,29 @@ extern "C" int wush_transform_quant(const void* x, int x_dtype, int64_t rows, in
   if (fmt == WUSH_FMT_NVFP4)
     return launch_fmt<16, kNv>(x, xf32, rows, d_in, t, kind, global_scale, codes, scales, y_debug, nullptr, s);
   return launch_fmt<32, kI4>(x, xf32, rows, d_in, t, kind, 0.f, codes, scales, y_debug, nullptr, s);
+}
+
+extern "C" int wush_transform_quant_nvfp4_dynamic(const void* x, int x_dtype, int64_t rows, int64_t d_in,
+                                                  const float* t, int kind, const float* amax,
+                                                  float* global_scale_out, uint8_t* codes, void* scales,
+                                                  float* y_debug, void* stream) {
+  int st = check_common(x, x_dtype, rows, d_in, t, kind, 16);
+  if (st != WUSH_OK) return st;
+  if (!amax || (reinterpret_cast<uintptr_t>(amax) & 3u)) return WUSH_ERR_INVALID_ARG;
+  if (global_scale_out && (reinterpret_cast<uintptr_t>(global_scale_out) & 3u)) return WUSH_ERR_INVALID_ARG;
+  if (rows == 0) return WUSH_OK;
+  if (!codes || !scales || !aligned16(codes) || !aligned16(scales)) return WUSH_ERR_INVALID_ARG;
+  if (y_debug && !aligned16(y_debug)) return WUSH_ERR_INVALID_ARG;
+  const bool xf32 = x_dtype == WUSH_IN_FP32;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!xf32) {
+    // the placeholder scale 1 is never used: the kernel reads the amax
+    const int tc = transform_quant_tc(x, rows, d_in, t, kind, WUSH_FMT_NVFP4, 1.0f, amax, global_scale_out, codes,
+                                      scales, y_debug, s);
+    if (tc != WUSH_ERR_UNSUPPORTED) return tc;
+  }
+  return launch_fmt<16, kNv>(x, xf32, rows, d_in, t, kind, 1.0f, codes, scales, y_debug, nullptr, s, amax,
+                             global_scale_out);
 }
 
 extern "C" int wush_transform_amax(const void* x, int x_dtype, int64_t rows, int64_t d_in, const float* t,
@@ -340,6 +371,10 @@ extern "C" int wush_transform_amax(const void* x, int x_dtype, int64_t rows, int
   if (cudaMemsetAsync(amax_out, 0, sizeof(float), s) != cudaSuccess) return WUSH_ERR_CUDA;
   if (rows == 0) return WUSH_OK;
   const bool xf32 = x_dtype == WUSH_IN_FP32;
+  if (!xf32) {
+    const int tc = transform_amax_tc(x, rows, d_in, t, kind, block, amax_out, s);
+    if (tc != WUSH_ERR_UNSUPPORTED) return tc;
+  }
   if (block == 32)
     return launch_fmt<32, kAmax>(x, xf32, rows, d_in, t, kind, 0.f, nullptr, nullptr, nullptr, amax_out, s);
   return launch_fmt<16, kAmax>(x, xf32, rows, d_in, t, kind, 0.f, nullptr, nullptr, nullptr, amax_out, s);

@@ -66,7 +66,8 @@ static_assert(kEpiGroups * 4 == kEpiWarps, "four warps per epilogue warpgroup");
 static_assert(kTmemCols == 512, "TMEM allocation is a power of two of at most 512 columns");
 
 enum Kind : int { kIdentity = 0, kHadamard = 1, kDense = 2 };
-enum Fmt : int { kMx = 0, kNv = 1, kI4 = 2 };
+// kAm: no quantisation; the kernel's only output is max |T x| over the tensor
+enum Fmt : int { kMx = 0, kNv = 1, kI4 = 2, kAm = 3 };
 
 __device__ int g_tq_error = 0;
 
@@ -266,8 +267,8 @@ __device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64
 
 template <int B, int FMT, int KIND, bool DBG>
 __global__ void __launch_bounds__(kThreads, 1)
-    tq_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* __restrict__ t, float gscale,
-                 uint8_t* __restrict__ codes, void* __restrict__ scales, float* __restrict__ ydbg, int rows,
+    tq_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* __restrict__ t, float gscale_arg,
+                 const float* __restrict__ gs_amax, float* __restrict__ gs_out, uint8_t* __restrict__ codes, void* __restrict__ scales, float* __restrict__ ydbg, int rows,
                  int d_in, int n_row_tiles, int n_tiles, int64_t max_polls) {
   constexpr int kBlocks = kTileCols / B;           // b-blocks per tile: 4 or 8
   constexpr int kQBlocks = kQuarterCols / B;       // b-blocks per quarter: 1 or 2
@@ -419,6 +420,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int g = et / 128;                     // warpgroup = quarter
     const int q = warp & 3;
     const int rloc = q * 32 + lane;             // row within the tile
+    // NVFP4 per-tensor scale: the caller's, or derived from a device amax
+    float gscale = gscale_arg;
+    if (FMT == kNv && gs_amax) {
+      gscale = nvfp4_dynamic_scale(__ldg(gs_amax));
+      if (gs_out && blockIdx.x == 0 && et == 0) *gs_out = gscale;
+    }
     const float den = 6.0f * gscale;
     const int n_atom_cols = (nb + 3) / 4;
 
@@ -485,6 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
 
+    float run_max = 0.f;                        // kAm: this thread's max |y|
     for (int i = tile_lo; i < tile_hi; ++i) {
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
       const int n = i - tile_lo, s = n % kStages;
@@ -553,19 +561,26 @@ __global__ void __launch_bounds__(kThreads, 1)
               dp[w] = make_float4(y[u][4 * w], y[u][4 * w + 1], y[u][4 * w + 2], y[u][4 * w + 3]);
           }
         }
-        uint32_t cw[B / 8];
-        const uint32_t sc = quantize_block<B, FMT>(y[u], gscale, den, cw);
-        if (blk_ok) {
-          uint8_t* cp = codes + static_cast<int64_t>(r) * (d_in / 2) + static_cast<int64_t>(j) * (B / 2);
-          if constexpr (B == 32) *reinterpret_cast<uint4*>(cp) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-          else *reinterpret_cast<uint2*>(cp) = make_uint2(cw[0], cw[1]);
-        }
-        if constexpr (FMT == kI4) {
-          if (blk_ok)
-            reinterpret_cast<uint16_t*>(scales)[static_cast<int64_t>(r) * nb + j] = static_cast<uint16_t>(sc);
-        } else if (j < n_atom_cols * 4) {
-          // padding rows and columns of an existing atom are written as zero
-          static_cast<uint8_t*>(scales)[sf_offset(r, j, n_atom_cols)] = static_cast<uint8_t>(blk_ok ? sc : 0u);
+        if constexpr (FMT == kAm) {
+          if (blk_ok) {
+#pragma unroll
+            for (int e = 0; e < B; ++e) run_max = fmaxf(run_max, fabsf(y[u][e]));
+          }
+        } else {
+          uint32_t cw[B / 8];
+          const uint32_t sc = quantize_block<B, FMT>(y[u], gscale, den, cw);
+          if (blk_ok) {
+            uint8_t* cp = codes + static_cast<int64_t>(r) * (d_in / 2) + static_cast<int64_t>(j) * (B / 2);
+            if constexpr (B == 32) *reinterpret_cast<uint4*>(cp) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+            else *reinterpret_cast<uint2*>(cp) = make_uint2(cw[0], cw[1]);
+          }
+          if constexpr (FMT == kI4) {
+            if (blk_ok)
+              reinterpret_cast<uint16_t*>(scales)[static_cast<int64_t>(r) * nb + j] = static_cast<uint16_t>(sc);
+          } else if (j < n_atom_cols * 4) {
+            // padding rows and columns of an existing atom are written as zero
+            static_cast<uint8_t*>(scales)[sf_offset(r, j, n_atom_cols)] = static_cast<uint8_t>(blk_ok ? sc : 0u);
+          }
         }
       }
 
@@ -579,6 +594,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (last_of_col && k + 2 < n_cols) convert_t(k + 2, et - g * 128, 128, 2 + g);
         }
       }
+    }
+    if constexpr (FMT == kAm) {
+      // non-negative floats order like their bit patterns; gs_out holds the
+      // tensor's running amax (zeroed by the caller)
+      const uint32_t m = __reduce_max_sync(0xffffffffu, __float_as_uint(run_max));
+      if (lane == 0 && m) atomicMax(reinterpret_cast<unsigned int*>(gs_out), m);
     }
   }
 
@@ -625,8 +646,8 @@ int num_sms() {
 }
 
 template <int B, int FMT, int KIND, bool DBG>
-int launch_tc(const void* x, int64_t rows, int64_t d_in, const float* t, float gscale, uint8_t* codes,
-              void* scales, float* ydbg, cudaStream_t st) {
+int launch_tc(const void* x, int64_t rows, int64_t d_in, const float* t, float gscale, const float* gs_amax,
+              float* gs_out, uint8_t* codes, void* scales, float* ydbg, cudaStream_t st) {
   EncodeFn enc = get_encode();
   if (!enc) return WUSH_ERR_CUDA;
   CUtensorMap map;
@@ -648,18 +669,18 @@ int launch_tc(const void* x, int64_t rows, int64_t d_in, const float* t, float g
   if (sms <= 0) return WUSH_ERR_CUDA;
   const int grid = n_tiles < sms ? n_tiles : sms;
   const int64_t polls = g_wait_limit_override > 0 ? g_wait_limit_override : kDefaultPolls;
-  kern<<<grid, kThreads, kSmemBytes, st>>>(map, t, gscale, codes, scales, ydbg, static_cast<int>(rows),
+  kern<<<grid, kThreads, kSmemBytes, st>>>(map, t, gscale, gs_amax, gs_out, codes, scales, ydbg, static_cast<int>(rows),
                                            static_cast<int>(d_in), n_row_tiles, n_tiles, polls);
   return launch_status();
 }
 
 template <int B, int FMT>
 int dispatch_kind(int kind, const void* x, int64_t rows, int64_t d_in, const float* t, float gscale,
-                  uint8_t* codes, void* scales, float* ydbg, cudaStream_t st) {
+                  const float* gs_amax, float* gs_out, uint8_t* codes, void* scales, float* ydbg, cudaStream_t st) {
   const int k = kind == WUSH_T_IDENTITY ? kIdentity : (kind == WUSH_T_HADAMARD ? kHadamard : kDense);
-#define WUSH_TC(KK)                                                                                     \
-  return ydbg ? launch_tc<B, FMT, KK, true>(x, rows, d_in, t, gscale, codes, scales, ydbg, st)          \
-              : launch_tc<B, FMT, KK, false>(x, rows, d_in, t, gscale, codes, scales, ydbg, st)
+#define WUSH_TC(KK)                                                                                             \
+  return ydbg ? launch_tc<B, FMT, KK, true>(x, rows, d_in, t, gscale, gs_amax, gs_out, codes, scales, ydbg, st) \
+              : launch_tc<B, FMT, KK, false>(x, rows, d_in, t, gscale, gs_amax, gs_out, codes, scales, ydbg, st)
   if (k == kIdentity) { WUSH_TC(kIdentity); }
   if (k == kHadamard) { WUSH_TC(kHadamard); }
   WUSH_TC(kDense);
@@ -681,13 +702,29 @@ int read_and_clear_tq_error(int* word) {
 // Tensor-core form of wush_transform_quant for bf16 inputs whose rows are 16-byte
 // aligned and whose sizes fit int32 indexing.  Returns WUSH_ERR_UNSUPPORTED when the
 // shape is outside that, so the caller can use the one-row-per-thread kernel.
+// max |T x| of a bf16 tensor into *amax_out (atomicMax on its bits; the caller
+// zeroes it first) by the tensor-core kernel; WUSH_ERR_UNSUPPORTED for shapes it
+// does not take.
+int transform_amax_tc(const void* x, int64_t rows, int64_t d_in, const float* t, int kind, int block,
+                      float* amax_out, cudaStream_t st) {
+  if (d_in % 8 || rows > (int64_t(1) << 30) || d_in > (int64_t(1) << 30)) return WUSH_ERR_UNSUPPORTED;
+  if (block == 32)
+    return dispatch_kind<32, kAm>(kind, x, rows, d_in, t, 1.0f, nullptr, amax_out, nullptr, nullptr, nullptr, st);
+  if (block == 16)
+    return dispatch_kind<16, kAm>(kind, x, rows, d_in, t, 1.0f, nullptr, amax_out, nullptr, nullptr, nullptr, st);
+  return WUSH_ERR_UNSUPPORTED;
+}
+
 int transform_quant_tc(const void* x, int64_t rows, int64_t d_in, const float* t, int kind, int fmt,
-                       float gscale, uint8_t* codes, void* scales, float* ydbg, cudaStream_t st) {
+                       float gscale, const float* gs_amax, float* gs_out, uint8_t* codes, void* scales, float* ydbg,
+                       cudaStream_t st) {
   if (d_in % 8 || rows > (int64_t(1) << 30) || d_in > (int64_t(1) << 30) || rows * (d_in / 2) > (int64_t(1) << 62))
     return WUSH_ERR_UNSUPPORTED;
-  if (fmt == WUSH_FMT_MXFP4) return dispatch_kind<32, kMx>(kind, x, rows, d_in, t, gscale, codes, scales, ydbg, st);
-  if (fmt == WUSH_FMT_NVFP4) return dispatch_kind<16, kNv>(kind, x, rows, d_in, t, gscale, codes, scales, ydbg, st);
-  return dispatch_kind<32, kI4>(kind, x, rows, d_in, t, gscale, codes, scales, ydbg, st);
+  if (fmt == WUSH_FMT_MXFP4)
+    return dispatch_kind<32, kMx>(kind, x, rows, d_in, t, gscale, nullptr, nullptr, codes, scales, ydbg, st);
+  if (fmt == WUSH_FMT_NVFP4)
+    return dispatch_kind<16, kNv>(kind, x, rows, d_in, t, gscale, gs_amax, gs_out, codes, scales, ydbg, st);
+  return dispatch_kind<32, kI4>(kind, x, rows, d_in, t, gscale, nullptr, nullptr, codes, scales, ydbg, st);
 }
 
 }  // namespace wush

@@ -298,8 +298,20 @@ def run_gpu(args, rank, world):
 
     stream = torch.cuda.Stream(device=dev)
 
+    # NVFP4 with --dynamic-scale: each step derives the activations' per-tensor scale
+    # on the device (an amax pass over T x, then the quantiser and the GEMM's alpha
+    # read it), instead of the static calibrated scale
+    dynamic = fmt == "nvfp4" and args.dynamic_scale
+    dyn_amax = torch.zeros(1, dtype=torch.float32, device=dev)
+    dyn_gs = torch.zeros(1, dtype=torch.float32, device=dev)
+
     def tq_into(x_in, acode):
-        aq.wush_transform_quant(x_in, t_x, kind, fmt, acode[0], acode[1], gx, stream=stream)
+        if dynamic:
+            aq.wush_transform_amax(x_in, t_x, kind, b, dyn_amax, stream=stream)
+            aq.wush_transform_quant_nvfp4_dynamic(x_in, t_x, kind, dyn_amax, acode[0], acode[1], dyn_gs,
+                                                  stream=stream)
+        else:
+            aq.wush_transform_quant(x_in, t_x, kind, fmt, acode[0], acode[1], gx, stream=stream)
 
     def tq(r):
         tq_into(xs[r], acodes[r])
@@ -312,6 +324,9 @@ def run_gpu(args, rank, world):
     def gemm_into(acode, wcode, y_out):
         if fmt == "int4":
             aq.wush_qgemm_int4_ws(acode[0], acode[1], wcode[0], wcode[1], M, N, K, ws, y_out, stream=stream)
+        elif dynamic:
+            aq.wush_qgemm_nvfp4_dynamic(acode[0], acode[1], wcode[0], wcode[1], M, N, K, dyn_gs, gw, y_out,
+                                        stream=stream)
         else:
             aq.wush_qgemm(acode[0], acode[1], wcode[0], wcode[1], M, N, K, fmt, alpha, y_out, stream=stream)
 
@@ -475,7 +490,9 @@ def run_gpu(args, rank, world):
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "e2m1 x e2m1 -> fp32 (transform in fp32)", "data": "synthetic",
-            "config": describe(w, fmt, kind),
+            "config": dict(describe(w, fmt, kind), **({"nvfp4_scale": "dynamic: device amax pass + scale every step "
+                                                                 "(inside the transform's time)"}
+                                                       if dynamic else {})),
             "transform_quant": {"us": tq_us, "GB_s": tq_gbs, "bytes_per_launch": tq_bytes,
                                 "frac_of_hbm": tq_gbs / peaks["hbm_gbs"], "dram_bytes_per_launch": tq_traffic,
                                 "burst_us": tq_burst_us,
@@ -484,7 +501,7 @@ def run_gpu(args, rank, world):
             "roofline": {"kernel": gemm_kernel, "bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak,
                          "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak, "traffic": traffic,
                          "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']:.1f} TFLOP/s, {gemm_peak_src}"},
-            "e2e": e2e, "gpu_launches": (4 if fmt == "int4" else 2) * args.steps,
+            "e2e": e2e, "gpu_launches": (4 if fmt == "int4" else 3 if dynamic else 2) * args.steps,
             "clocks": sampler.summary(),
         }
     return result, (w, x, wt, xc, fmt, kind)
@@ -557,6 +574,8 @@ def main():
     ap.add_argument("--transform", default=None, choices=["identity", "hadamard", "wus", "wush", "wush_diag"],
                     help="override the workload's block transform (calibrated from the same tokens)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--dynamic-scale", action="store_true",
+                    help="NVFP4: derive the activations' per-tensor scale on the device every step")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     rank = int(os.environ.get("RANK", 0))

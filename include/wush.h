@@ -167,6 +167,23 @@ int wush_transform_quant(const void* x, int x_dtype, int64_t rows, int64_t d_in,
 int wush_transform_amax(const void* x, int x_dtype, int64_t rows, int64_t d_in,
                         const float* t, int kind, int block, float* amax_out, void* stream);
 
+/* Dynamic per-tensor NVFP4 scale: wush_transform_quant for NVFP4 whose
+ * global_scale is derived on the device from ``amax`` (device fp32, e.g.
+ * written by wush_transform_amax on the same x, t and kind with block 16,
+ * earlier in the stream) as
+ *   global_scale = fp32(amax / 2688)   (2688 = 6 * 448),
+ *   or 1 if that is below 1e-30 (an all-zero tensor: every code is 0).
+ * The scale is written to device *global_scale_out (if not NULL) for
+ * wush_qgemm_nvfp4_dynamic; with rows = 0 nothing is launched or written.
+ * The pages name NVFP4 only; the static calibrated scale of
+ * wush_transform_quant is the default reading, this is the per-batch variant.
+ * Other arguments and requirements as in wush_transform_quant; amax and
+ * global_scale_out 4-byte aligned. */
+int wush_transform_quant_nvfp4_dynamic(const void* x, int x_dtype, int64_t rows, int64_t d_in,
+                                       const float* t, int kind, const float* amax,
+                                       float* global_scale_out, uint8_t* codes, void* scales,
+                                       float* y_debug, void* stream);
+
 /* ---------------------------------------------------------------------------
  * Block-scaled FP4 GEMM on tcgen05 tensor cores (device)
  *
@@ -187,6 +204,15 @@ int wush_transform_amax(const void* x, int x_dtype, int64_t rows, int64_t d_in,
 int wush_qgemm(const uint8_t* a_codes, const void* a_scales, const uint8_t* b_codes,
                const void* b_scales, int64_t M, int64_t N, int64_t K, int fmt, float alpha,
                float* y, void* stream);
+
+/* NVFP4 wush_qgemm whose alpha is formed on the device as
+ *   alpha = fp32(*a_global_scale * b_global_scale),
+ * a_global_scale a device fp32 (4-byte aligned), e.g. written by
+ * wush_transform_quant_nvfp4_dynamic earlier in the stream; b_global_scale the
+ * weights' static scale.  Other arguments as in wush_qgemm with fmt NVFP4. */
+int wush_qgemm_nvfp4_dynamic(const uint8_t* a_codes, const void* a_scales, const uint8_t* b_codes,
+                             const void* b_scales, int64_t M, int64_t N, int64_t K,
+                             const float* a_global_scale, float b_global_scale, float* y, void* stream);
 
 /* ---------------------------------------------------------------------------
  * INT4 GEMM with per-32-group fp16 scales (device)

@@ -143,3 +143,17 @@ def nvfp4_global_scale(y_rows: np.ndarray) -> np.float32:
     """
     amax = float(np.max(np.abs(np.asarray(y_rows, dtype=np.float64))))
     return np.float32(amax / (6.0 * 448.0))
+
+
+def nvfp4_dynamic_global_scale(y_rows: np.ndarray) -> np.float32:
+    """Per-batch NVFP4 scale: s_g = fp32(amax / 2688) of the transformed tensor being
+    quantised, or 1 when that is below 1e-30 (all-zero input: every code is 0).
+
+    Reading: the pages name NVFP4 without its scale rule; the static calibrated
+    scale (nvfp4_global_scale on calibration tokens) is the default, and this is
+    the per-batch variant of the same rule.  amax is the exact maximum of the
+    fp32 values and the quotient is rounded once to fp32.
+    """
+    amax = np.float32(np.max(np.abs(np.asarray(y_rows, dtype=np.float32)))) if np.size(y_rows) else np.float32(0)
+    g = np.float32(np.float64(amax) / 2688.0)
+    return g if g >= np.float32(1e-30) else np.float32(1.0)

@@ -129,14 +129,21 @@ def test_empty_rows_is_noop(lib):
     assert int(codes.sum()) == 0
 
 
-def test_amax_matches_oracle(lib):
-    w = synth.WORKLOADS["down_proj"]
-    x = synth.activations(w, tokens=200)
-    t = _transform("wush", "nvfp4", w)
-    out = torch.empty(1, dtype=torch.float32, device="cuda")
-    lib.wush_transform_amax(_as_input(x, True).cuda(), torch.from_numpy(t).cuda(), "wush", 16, out)
+@pytest.mark.parametrize("kind", ["identity", "hadamard", "wush"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4"])
+def test_amax_matches_oracle(lib, kind, fmt):
+    # bf16 x runs the tensor-core kernel's amax mode, fp32 x the one-row-per-thread
+    # kernel; 300 rows leave a ragged row tile, whose padding rows must not count
+    w = synth.WORKLOADS[FMT_WORKLOAD[fmt]]
+    x = synth.activations(w, tokens=300)
+    t = _transform(kind, fmt, w)
+    tt = None if kind in ("identity", "hadamard") else torch.from_numpy(t).cuda()
     want = np.max(np.abs(T.apply_block_transform(x, t)))
-    assert abs(float(out.item()) - want) <= 1e-5 * want
+    for bf16 in (True, False):
+        out = torch.full((1,), float("nan"), dtype=torch.float32, device="cuda")
+        lib.wush_transform_amax(_as_input(x, bf16).cuda(), tt, kind, P.Q.BLOCK[fmt], out)
+        torch.cuda.synchronize()
+        assert abs(float(out.item()) - want) <= 1e-5 * want, (bf16, float(out.item()), want)
 
 
 @pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4", "int4"])

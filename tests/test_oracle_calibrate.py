@@ -170,3 +170,19 @@ def test_wush_diag_floors_dead_channels():
     assert np.allclose(tw.T @ tx, np.eye(4), atol=1e-9)
     tx0, tw0 = C.block_transform_pair(np.zeros((4, 4)), np.zeros((4, 4)), "wush_diag")
     assert np.allclose(tx0, T.normalized_hadamard(4)) and np.allclose(tw0, T.normalized_hadamard(4))
+
+
+def test_nvfp4_dynamic_global_scale_rule():
+    # s_g = fp32(amax / 2688), rounded once; 1 for (near-)zero tensors
+    from fractions import Fraction
+    assert C.nvfp4_dynamic_global_scale(np.array([2688.0, -1.0])) == np.float32(1.0)
+    assert C.nvfp4_dynamic_global_scale(np.array([-5376.0])) == np.float32(2.0)
+    assert C.nvfp4_dynamic_global_scale(np.zeros(7)) == np.float32(1.0)
+    assert C.nvfp4_dynamic_global_scale(np.array([1e-27])) == np.float32(1.0)   # 3.7e-31 < 1e-30
+    rng = np.random.default_rng(3)
+    for a in rng.uniform(1e-3, 1e4, 200).astype(np.float32):
+        g = C.nvfp4_dynamic_global_scale(np.array([a]))
+        exact = Fraction(float(a)) / 2688
+        nbrs = (np.nextafter(g, np.float32(0)), np.nextafter(g, np.float32(np.inf)))
+        assert all(abs(Fraction(float(g)) - exact) <= abs(Fraction(float(n)) - exact) for n in nbrs)
+        assert g == C.nvfp4_global_scale(np.array([a]))                       # same rule as the static scale
