@@ -32,10 +32,14 @@ _SIGNATURES = {
     "wush_block_size": (_i32, [_i32]),
     "wush_calibrate": (_i32, [_vp, _i64, _vp, _i64, _i64, _i32, _i32, _vp, _vp]),
     "wush_calibrate_from_moments": (_i32, [_vp, _vp, _i64, _i32, _i32, _vp, _vp]),
+    "wush_calibrate_shared": (_i32, [_vp, _i64, _vp, _i64, _i64, _i32, _i32, _i32, _vp, _vp, _vp]),
+    "wush_calibrate_shared_from_moments": (_i32, [_vp, _vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp]),
     "wush_codes_bytes": (_sz, [_i64, _i64, _i32]),
     "wush_scales_bytes": (_sz, [_i64, _i64, _i32]),
     "wush_transform_quant": (_i32, [_vp, _i32, _i64, _i64, _vp, _i32, _i32, _f32, _vp, _vp, _vp, _vp]),
     "wush_transform_amax": (_i32, [_vp, _i32, _i64, _i64, _vp, _i32, _i32, _vp, _vp]),
+    "wush_transform_quant_indexed": (_i32, [_vp, _i32, _i64, _i64, _vp, _vp, _i32, _i32, _i32, _f32, _vp, _vp, _vp,
+                                             _vp]),
     "wush_transform_quant_nvfp4_dynamic": (_i32, [_vp, _i32, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp]),
     "wush_qgemm": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _f32, _vp, _vp]),
     "wush_qgemm_nvfp4_dynamic": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _f32, _vp, _vp]),
@@ -119,6 +123,35 @@ def wush_calibrate(x_calib: np.ndarray, w: np.ndarray, block: int, kind):
     return tx, tw
 
 
+def wush_calibrate_shared(x_calib: np.ndarray, w: np.ndarray, block: int, kind, groups: int):
+    """(t_x, t_w) fp32 [groups, block, block] and the block -> group index int32 [d_in/block]."""
+    x, xp = _host(x_calib, np.float32)
+    wt, wp = _host(w, np.float32)
+    d_in = x.shape[1]
+    if wt.shape[1] != d_in:
+        raise ValueError("d_in mismatch")
+    tx = np.empty((groups, block, block), np.float32)
+    tw = np.empty_like(tx)
+    index = np.empty(d_in // block, np.int32)
+    _check("wush_calibrate_shared",
+           _lib.wush_calibrate_shared(xp, x.shape[0], wp, wt.shape[0], d_in, block, _enum(TRANSFORMS, kind),
+                                      int(groups), tx.ctypes.data, tw.ctypes.data, index.ctypes.data))
+    return tx, tw, index
+
+
+def wush_calibrate_shared_from_moments(sigma_x: np.ndarray, sigma_w: np.ndarray, kind, groups: int):
+    sx, sxp = _host(sigma_x, np.float64)
+    sw, swp = _host(sigma_w, np.float64)
+    nb, b, _ = sx.shape
+    tx = np.empty((groups, b, b), np.float32)
+    tw = np.empty_like(tx)
+    index = np.empty(nb, np.int32)
+    _check("wush_calibrate_shared_from_moments",
+           _lib.wush_calibrate_shared_from_moments(sxp, swp, nb * b, b, _enum(TRANSFORMS, kind), int(groups),
+                                                   tx.ctypes.data, tw.ctypes.data, index.ctypes.data))
+    return tx, tw, index
+
+
 def wush_calibrate_from_moments(sigma_x: np.ndarray, sigma_w: np.ndarray, kind):
     sx, sxp = _host(sigma_x, np.float64)
     sw, swp = _host(sigma_w, np.float64)
@@ -172,6 +205,20 @@ def wush_transform_quant(x, t, kind, fmt, codes, scales, global_scale: float = 0
            _lib.wush_transform_quant(_ptr(x), x_dtype, rows, d_in, _ptr(t), _enum(TRANSFORMS, kind),
                                      _enum(FORMATS, fmt), float(global_scale), _ptr(codes), _ptr(scales),
                                      _ptr(y_debug), _stream(stream)))
+
+
+def wush_transform_quant_indexed(x, t, t_index, kind, fmt, codes, scales, global_scale: float = 0.0, y_debug=None,
+                                 stream=None):
+    """wush_transform_quant with shared transforms: t CUDA fp32 [n_t, b, b], t_index CUDA int32 [d_in/b]."""
+    import torch
+    x_dtype = IN_FP32 if x.dtype == torch.float32 else IN_BF16
+    if x.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("x must be bf16 or fp32")
+    rows, d_in = x.shape
+    _check("wush_transform_quant_indexed",
+           _lib.wush_transform_quant_indexed(_ptr(x), x_dtype, rows, d_in, _ptr(t), _ptr(t_index), int(t.shape[0]),
+                                             _enum(TRANSFORMS, kind), _enum(FORMATS, fmt), float(global_scale),
+                                             _ptr(codes), _ptr(scales), _ptr(y_debug), _stream(stream)))
 
 
 def wush_transform_amax(x, t, kind, block: int, amax_out, stream=None):

@@ -275,3 +275,106 @@ extern "C" int wush_calibrate(const float* x_calib, int64_t n_calib, const float
   block_moments(w, d_out, d_in, block, sw.data());
   return wush_calibrate_from_moments(sx.data(), sw.data(), d_in, block, kind, t_x, t_w);
 }
+
+// ---------------------------------------------------------------------------
+// Transform sharing (WUSH news article, paragraph 6: share transform matrices
+// between similar blocks).  The pages give no algorithm.  Reading: a block's
+// feature is its two moments divided by their traces, flattened; k-means (Lloyd)
+// groups the features, with centres started at blocks round(i * nb / groups)
+// (halves to even), squared Euclidean distance, ties to the lowest group, empty
+// groups keeping their centre, until no block changes group (at most 50
+// rounds).  Each group's transform comes from its members' mean moments.
+extern "C" int wush_calibrate_shared_from_moments(const double* sigma_x, const double* sigma_w, int64_t d_in,
+                                                  int block, int kind, int groups, float* t_x, float* t_w,
+                                                  int32_t* index) {
+  if (!sigma_x || !sigma_w || !t_x || !t_w || !index || !is_pow2(block) || block < 2 || block > 256 || d_in <= 0 ||
+      d_in % block)
+    return WUSH_ERR_INVALID_ARG;
+  if (kind < WUSH_T_WUS || kind > WUSH_T_WUSH_DIAG) return WUSH_ERR_UNSUPPORTED;
+  const int64_t nb = d_in / block, bb = static_cast<int64_t>(block) * block, nf = 2 * bb;
+  if (groups < 1 || groups > nb) return WUSH_ERR_INVALID_ARG;
+  std::vector<double> feat(static_cast<size_t>(nb * nf));
+  for (int64_t j = 0; j < nb; ++j) {
+    for (int m = 0; m < 2; ++m) {
+      const double* sg = (m == 0 ? sigma_x : sigma_w) + j * bb;
+      double tr = 0.0;
+      for (int k = 0; k < block; ++k) tr += sg[k * block + k];
+      const double dv = tr > 0 ? tr : 1.0;
+      for (int64_t e = 0; e < bb; ++e) feat[j * nf + m * bb + e] = sg[e] / dv;
+    }
+  }
+  std::vector<double> centres(static_cast<size_t>(groups * nf));
+  for (int g = 0; g < groups; ++g) {
+    const int64_t src = static_cast<int64_t>(std::nearbyint(static_cast<double>(g) * nb / groups));
+    std::memcpy(&centres[g * nf], &feat[src * nf], sizeof(double) * nf);
+  }
+  std::vector<int32_t> assign(nb, -1), next(nb);
+  for (int it = 0; it < 50; ++it) {
+    for (int64_t j = 0; j < nb; ++j) {
+      int best = 0;
+      double best_d = 0.0;
+      for (int g = 0; g < groups; ++g) {
+        double d = 0.0;
+        for (int64_t f = 0; f < nf; ++f) {
+          const double v = feat[j * nf + f] - centres[g * nf + f];
+          d += v * v;
+        }
+        if (g == 0 || d < best_d) { best = g; best_d = d; }
+      }
+      next[j] = best;
+    }
+    if (next == assign) break;
+    assign = next;
+    for (int g = 0; g < groups; ++g) {
+      int64_t cnt = 0;
+      std::vector<double> acc(nf, 0.0);
+      for (int64_t j = 0; j < nb; ++j)
+        if (assign[j] == g) {
+          ++cnt;
+          for (int64_t f = 0; f < nf; ++f) acc[f] += feat[j * nf + f];
+        }
+      if (cnt)
+        for (int64_t f = 0; f < nf; ++f) centres[g * nf + f] = acc[f] / cnt;
+    }
+  }
+  std::vector<double> gx(static_cast<size_t>(groups * bb), 0.0), gw(static_cast<size_t>(groups * bb), 0.0);
+  std::vector<int64_t> cnt(groups, 0);
+  for (int64_t j = 0; j < nb; ++j) {
+    const int g = assign[j];
+    index[j] = g;
+    ++cnt[g];
+    for (int64_t e = 0; e < bb; ++e) {
+      gx[g * bb + e] += sigma_x[j * bb + e];
+      gw[g * bb + e] += sigma_w[j * bb + e];
+    }
+  }
+  for (int g = 0; g < groups; ++g) {
+    if (cnt[g] == 0) {
+      // a group left empty (its start tied with an earlier group's) maps no block:
+      // its transform comes from its starting block's moments
+      const int64_t src = static_cast<int64_t>(std::nearbyint(static_cast<double>(g) * nb / groups));
+      std::memcpy(&gx[g * bb], sigma_x + src * bb, sizeof(double) * bb);
+      std::memcpy(&gw[g * bb], sigma_w + src * bb, sizeof(double) * bb);
+      continue;
+    }
+    for (int64_t e = 0; e < bb; ++e) {
+      gx[g * bb + e] /= static_cast<double>(cnt[g]);
+      gw[g * bb + e] /= static_cast<double>(cnt[g]);
+    }
+  }
+  return wush_calibrate_from_moments(gx.data(), gw.data(), static_cast<int64_t>(groups) * block, block, kind, t_x,
+                                     t_w);
+}
+
+extern "C" int wush_calibrate_shared(const float* x_calib, int64_t n_calib, const float* w, int64_t d_out,
+                                     int64_t d_in, int block, int kind, int groups, float* t_x, float* t_w,
+                                     int32_t* index) {
+  if (!x_calib || !w || n_calib <= 0 || d_out <= 0 || !is_pow2(block) || block < 2 || block > 256 || d_in <= 0 ||
+      d_in % block)
+    return WUSH_ERR_INVALID_ARG;
+  const size_t n = static_cast<size_t>(d_in / block) * block * block;
+  std::vector<double> sx(n), sw(n);
+  block_moments(x_calib, n_calib, d_in, block, sx.data());
+  block_moments(w, d_out, d_in, block, sw.data());
+  return wush_calibrate_shared_from_moments(sx.data(), sw.data(), d_in, block, kind, groups, t_x, t_w, index);
+}

@@ -30,9 +30,11 @@ int read_and_clear_itq3_tc_error(int* word);
 // (nvfp4_dynamic_scale) instead of gscale, and CTA 0 writes it to gs_out if given.
 int transform_amax_tc(const void* x, int64_t rows, int64_t d_in, const float* t, int kind, int block,
                       float* amax_out, cudaStream_t st);
-int transform_quant_tc(const void* x, int64_t rows, int64_t d_in, const float* t, int kind, int fmt,
-                       float gscale, const float* gs_amax, float* gs_out, uint8_t* codes, void* scales, float* ydbg,
-                       cudaStream_t st);
+// t_index (device int32 [d_in/b], optional): block j uses transform t[t_index[j]],
+// clamped to [0, n_t), instead of t[j].
+int transform_quant_tc(const void* x, int64_t rows, int64_t d_in, const float* t, const int* t_index, int n_t,
+                       int kind, int fmt, float gscale, const float* gs_amax, float* gs_out, uint8_t* codes,
+                       void* scales, float* ydbg, cudaStream_t st);
 
 // GEMM kernel choice (see wush_debug_set_gemm_variant).
 extern int g_gemm_variant;

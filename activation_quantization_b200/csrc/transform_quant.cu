@@ -126,7 +126,8 @@ __device__ __forceinline__ void dense_apply(const float* __restrict__ tj, const 
 
 template <int B, int KIND, int FMT, bool XF32, bool DBG>
 __global__ void __launch_bounds__(kRowsPerCta) transform_quant_kernel(
-    const void* __restrict__ x, int64_t rows, int64_t d_in, const float* __restrict__ t, float gscale_arg,
+    const void* __restrict__ x, int64_t rows, int64_t d_in, const float* __restrict__ t,
+    const int* __restrict__ t_index, int n_t, float gscale_arg,
     const float* __restrict__ gs_amax, float* __restrict__ gs_out, uint8_t* __restrict__ codes,
     void* __restrict__ scales, float* __restrict__ ydbg, float* __restrict__ amax_out) {
   // NVFP4 per-tensor scale: the caller's, or derived from a device amax
@@ -147,9 +148,18 @@ __global__ void __launch_bounds__(kRowsPerCta) transform_quant_kernel(
   const int64_t r = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + tid;
 
   if constexpr (KIND == kDense) {
-    const float4* src = reinterpret_cast<const float4*>(t + j0 * B * B);
+    // block j's T is t[j], or t[t_index[j]] (clamped to the n_t transforms)
+    constexpr int kQuads = B * B / 4;
     float4* dst = reinterpret_cast<float4*>(s_t);
-    for (int i = tid; i < nblk * B * B / 4; i += kRowsPerCta) dst[i] = __ldg(src + i);
+    for (int i = tid; i < nblk * kQuads; i += kRowsPerCta) {
+      const int k = i / kQuads;
+      int64_t jt = j0 + k;
+      if (t_index) {
+        const int v = __ldg(t_index + j0 + k);
+        jt = v < 0 ? 0 : (v >= n_t ? n_t - 1 : v);
+      }
+      dst[i] = __ldg(reinterpret_cast<const float4*>(t + jt * B * B) + (i - k * kQuads));
+    }
   }
   if constexpr (FMT == kMx || FMT == kNv) reinterpret_cast<uint32_t*>(s_sf)[tid] = 0u;
   __syncthreads();
@@ -251,14 +261,14 @@ __global__ void __launch_bounds__(kRowsPerCta) transform_quant_kernel(
 template <int B, int FMT>
 int launch_fmt(const void* x, bool xf32, int64_t rows, int64_t d_in, const float* t, int kind, float gscale,
                uint8_t* codes, void* scales, float* ydbg, float* amax_out, cudaStream_t st,
-               const float* gs_amax = nullptr, float* gs_out = nullptr) {
+               const float* gs_amax = nullptr, float* gs_out = nullptr, const int* t_index = nullptr, int n_t = 0) {
   const dim3 grid(static_cast<unsigned>((rows + kRowsPerCta - 1) / kRowsPerCta),
                   static_cast<unsigned>((d_in / B + kBlocksPerCta - 1) / kBlocksPerCta));
   const dim3 block(kRowsPerCta);
   const int k = kind == WUSH_T_IDENTITY ? kIdentity : (kind == WUSH_T_HADAMARD ? kHadamard : kDense);
 #define WUSH_TQ_LAUNCH(KK, XF, DB)                                                                \
-  transform_quant_kernel<B, KK, FMT, XF, DB><<<grid, block, 0, st>>>(x, rows, d_in, t, gscale, gs_amax, \
-                                                                     gs_out, codes, scales, ydbg, amax_out)
+  transform_quant_kernel<B, KK, FMT, XF, DB><<<grid, block, 0, st>>>(x, rows, d_in, t, t_index, n_t, gscale, \
+                                                                     gs_amax, gs_out, codes, scales, ydbg, amax_out)
 #define WUSH_TQ_KIND(XF, DB)                       \
   do {                                             \
     if (k == kIdentity) WUSH_TQ_LAUNCH(kIdentity, XF, DB); \
@@ -327,8 +337,8 @@ extern "C" int wush_transform_quant(const void* x, int x_dtype, int64_t rows, in
   const bool xf32 = x_dtype == WUSH_IN_FP32;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (!xf32) {
-    const int tc =
-        transform_quant_tc(x, rows, d_in, t, kind, fmt, global_scale, nullptr, nullptr, codes, scales, y_debug, s);
+    const int tc = transform_quant_tc(x, rows, d_in, t, nullptr, 0, kind, fmt, global_scale, nullptr, nullptr, codes,
+                                      scales, y_debug, s);
     if (tc != WUSH_ERR_UNSUPPORTED) return tc;
   }
   if (fmt == WUSH_FMT_MXFP4)
@@ -336,6 +346,36 @@ extern "C" int wush_transform_quant(const void* x, int x_dtype, int64_t rows, in
   if (fmt == WUSH_FMT_NVFP4)
     return launch_fmt<16, kNv>(x, xf32, rows, d_in, t, kind, global_scale, codes, scales, y_debug, nullptr, s);
   return launch_fmt<32, kI4>(x, xf32, rows, d_in, t, kind, 0.f, codes, scales, y_debug, nullptr, s);
+}
+
+extern "C" int wush_transform_quant_indexed(const void* x, int x_dtype, int64_t rows, int64_t d_in, const float* t,
+                                            const int32_t* t_index, int n_t, int kind, int fmt, float global_scale,
+                                            uint8_t* codes, void* scales, float* y_debug, void* stream) {
+  const int b = wush_block_size(fmt);
+  if (b == 0) return WUSH_ERR_UNSUPPORTED;
+  if (kind < WUSH_T_WUS) return WUSH_ERR_INVALID_ARG;   // only dense transforms are shared
+  int st = check_common(x, x_dtype, rows, d_in, t, kind, b);
+  if (st != WUSH_OK) return st;
+  if (!t_index || (reinterpret_cast<uintptr_t>(t_index) & 3u) || n_t < 1) return WUSH_ERR_INVALID_ARG;
+  if (rows == 0) return WUSH_OK;
+  if (!codes || !scales || !aligned16(codes) || !aligned16(scales)) return WUSH_ERR_INVALID_ARG;
+  if (y_debug && !aligned16(y_debug)) return WUSH_ERR_INVALID_ARG;
+  if (fmt == WUSH_FMT_NVFP4 && !(global_scale >= 1e-30f && global_scale < 1e30f)) return WUSH_ERR_INVALID_ARG;
+  const bool xf32 = x_dtype == WUSH_IN_FP32;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!xf32) {
+    const int tc = transform_quant_tc(x, rows, d_in, t, t_index, n_t, kind, fmt, global_scale, nullptr, nullptr,
+                                      codes, scales, y_debug, s);
+    if (tc != WUSH_ERR_UNSUPPORTED) return tc;
+  }
+  if (fmt == WUSH_FMT_MXFP4)
+    return launch_fmt<32, kMx>(x, xf32, rows, d_in, t, kind, 0.f, codes, scales, y_debug, nullptr, s, nullptr,
+                               nullptr, t_index, n_t);
+  if (fmt == WUSH_FMT_NVFP4)
+    return launch_fmt<16, kNv>(x, xf32, rows, d_in, t, kind, global_scale, codes, scales, y_debug, nullptr, s,
+                               nullptr, nullptr, t_index, n_t);
+  return launch_fmt<32, kI4>(x, xf32, rows, d_in, t, kind, 0.f, codes, scales, y_debug, nullptr, s, nullptr, nullptr,
+                             t_index, n_t);
 }
 
 extern "C" int wush_transform_quant_nvfp4_dynamic(const void* x, int x_dtype, int64_t rows, int64_t d_in,
@@ -353,8 +393,8 @@ extern "C" int wush_transform_quant_nvfp4_dynamic(const void* x, int x_dtype, in
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (!xf32) {
     // the placeholder scale 1 is never used: the kernel reads the amax
-    const int tc = transform_quant_tc(x, rows, d_in, t, kind, WUSH_FMT_NVFP4, 1.0f, amax, global_scale_out, codes,
-                                      scales, y_debug, s);
+    const int tc = transform_quant_tc(x, rows, d_in, t, nullptr, 0, kind, WUSH_FMT_NVFP4, 1.0f, amax,
+                                      global_scale_out, codes, scales, y_debug, s);
     if (tc != WUSH_ERR_UNSUPPORTED) return tc;
   }
   return launch_fmt<16, kNv>(x, xf32, rows, d_in, t, kind, 1.0f, codes, scales, y_debug, nullptr, s, amax,

@@ -267,7 +267,8 @@ __device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64
 
 template <int B, int FMT, int KIND, bool DBG>
 __global__ void __launch_bounds__(kThreads, 1)
-    tq_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* __restrict__ t, float gscale_arg,
+    tq_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const float* __restrict__ t,
+                 const int* __restrict__ t_index, int n_t, float gscale_arg,
                  const float* __restrict__ gs_amax, float* __restrict__ gs_out, uint8_t* __restrict__ codes, void* __restrict__ scales, float* __restrict__ ydbg, int rows,
                  int d_in, int n_row_tiles, int n_tiles, int64_t max_polls) {
   constexpr int kBlocks = kTileCols / B;           // b-blocks per tile: 4 or 8
@@ -307,6 +308,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int kTGroups = kBlocks * B * B / 4;    // float4 groups of T per column
   constexpr int kTPer = kTGroups / kEpiThreads;    // per epilogue thread: 2 or 1
   static_assert(kTPer * kEpiThreads == kTGroups, "T column splits evenly over the epilogue threads");
+  // T of block j: t[j], or t[t_index[j]] (clamped to the n_t transforms) when
+  // blocks share transforms
+  auto t_block = [&](int j) -> const float* {
+    int jt = j;
+    if (t_index) {
+      const int v = __ldg(t_index + j);
+      jt = v < 0 ? 0 : (v >= n_t ? n_t - 1 : v);
+    }
+    return t + static_cast<int64_t>(jt) * B * B;
+  };
   float4 t_pre[2][kTPer];
   if (kMma && threadIdx.x >= 64) {
 #pragma unroll
@@ -315,9 +326,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int p = 0; p < kTPer; ++p) {
         const int e0 = 4 * (static_cast<int>(threadIdx.x) - 64 + p * kEpiThreads);
         const int j = (col_lo + c) * kBlocks + e0 / (B * B);
-        t_pre[c][p] = (c < n_cols && j < nb)
-                          ? __ldg(reinterpret_cast<const float4*>(t + static_cast<int64_t>(j) * B * B + e0 % (B * B)))
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
+        t_pre[c][p] = (c < n_cols && j < nb) ? __ldg(reinterpret_cast<const float4*>(t_block(j) + e0 % (B * B)))
+                                             : make_float4(0.f, 0.f, 0.f, 0.f);
       }
   }
   auto issue_load = [&](int n) {
@@ -465,7 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int gi = base + tid + p * nthr;
           const int e0 = 4 * gi;
           v[p] = (gi < kTGroups && j0 + e0 / (B * B) < nb)
-                     ? __ldg(reinterpret_cast<const float4*>(t + static_cast<int64_t>(j0) * B * B + e0))
+                     ? __ldg(reinterpret_cast<const float4*>(t_block(j0 + e0 / (B * B)) + e0 % (B * B)))
                      : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
@@ -646,8 +656,8 @@ int num_sms() {
 }
 
 template <int B, int FMT, int KIND, bool DBG>
-int launch_tc(const void* x, int64_t rows, int64_t d_in, const float* t, float gscale, const float* gs_amax,
-              float* gs_out, uint8_t* codes, void* scales, float* ydbg, cudaStream_t st) {
+int launch_tc(const void* x, int64_t rows, int64_t d_in, const float* t, const int* t_index, int n_t, float gscale,
+              const float* gs_amax, float* gs_out, uint8_t* codes, void* scales, float* ydbg, cudaStream_t st) {
   EncodeFn enc = get_encode();
   if (!enc) return WUSH_ERR_CUDA;
   CUtensorMap map;
@@ -669,18 +679,22 @@ int launch_tc(const void* x, int64_t rows, int64_t d_in, const float* t, float g
   if (sms <= 0) return WUSH_ERR_CUDA;
   const int grid = n_tiles < sms ? n_tiles : sms;
   const int64_t polls = g_wait_limit_override > 0 ? g_wait_limit_override : kDefaultPolls;
-  kern<<<grid, kThreads, kSmemBytes, st>>>(map, t, gscale, gs_amax, gs_out, codes, scales, ydbg, static_cast<int>(rows),
+  kern<<<grid, kThreads, kSmemBytes, st>>>(map, t, t_index, n_t, gscale, gs_amax, gs_out, codes, scales, ydbg,
+                                           static_cast<int>(rows),
                                            static_cast<int>(d_in), n_row_tiles, n_tiles, polls);
   return launch_status();
 }
 
 template <int B, int FMT>
-int dispatch_kind(int kind, const void* x, int64_t rows, int64_t d_in, const float* t, float gscale,
-                  const float* gs_amax, float* gs_out, uint8_t* codes, void* scales, float* ydbg, cudaStream_t st) {
+int dispatch_kind(int kind, const void* x, int64_t rows, int64_t d_in, const float* t, const int* t_index, int n_t,
+                  float gscale, const float* gs_amax, float* gs_out, uint8_t* codes, void* scales, float* ydbg,
+                  cudaStream_t st) {
   const int k = kind == WUSH_T_IDENTITY ? kIdentity : (kind == WUSH_T_HADAMARD ? kHadamard : kDense);
 #define WUSH_TC(KK)                                                                                             \
-  return ydbg ? launch_tc<B, FMT, KK, true>(x, rows, d_in, t, gscale, gs_amax, gs_out, codes, scales, ydbg, st) \
-              : launch_tc<B, FMT, KK, false>(x, rows, d_in, t, gscale, gs_amax, gs_out, codes, scales, ydbg, st)
+  return ydbg ? launch_tc<B, FMT, KK, true>(x, rows, d_in, t, t_index, n_t, gscale, gs_amax, gs_out, codes, scales, \
+                                            ydbg, st)                                                             \
+              : launch_tc<B, FMT, KK, false>(x, rows, d_in, t, t_index, n_t, gscale, gs_amax, gs_out, codes, scales, \
+                                             ydbg, st)
   if (k == kIdentity) { WUSH_TC(kIdentity); }
   if (k == kHadamard) { WUSH_TC(kHadamard); }
   WUSH_TC(kDense);
@@ -709,22 +723,27 @@ int transform_amax_tc(const void* x, int64_t rows, int64_t d_in, const float* t,
                       float* amax_out, cudaStream_t st) {
   if (d_in % 8 || rows > (int64_t(1) << 30) || d_in > (int64_t(1) << 30)) return WUSH_ERR_UNSUPPORTED;
   if (block == 32)
-    return dispatch_kind<32, kAm>(kind, x, rows, d_in, t, 1.0f, nullptr, amax_out, nullptr, nullptr, nullptr, st);
+    return dispatch_kind<32, kAm>(kind, x, rows, d_in, t, nullptr, 0, 1.0f, nullptr, amax_out, nullptr, nullptr,
+                                  nullptr, st);
   if (block == 16)
-    return dispatch_kind<16, kAm>(kind, x, rows, d_in, t, 1.0f, nullptr, amax_out, nullptr, nullptr, nullptr, st);
+    return dispatch_kind<16, kAm>(kind, x, rows, d_in, t, nullptr, 0, 1.0f, nullptr, amax_out, nullptr, nullptr,
+                                  nullptr, st);
   return WUSH_ERR_UNSUPPORTED;
 }
 
-int transform_quant_tc(const void* x, int64_t rows, int64_t d_in, const float* t, int kind, int fmt,
-                       float gscale, const float* gs_amax, float* gs_out, uint8_t* codes, void* scales, float* ydbg,
-                       cudaStream_t st) {
+int transform_quant_tc(const void* x, int64_t rows, int64_t d_in, const float* t, const int* t_index, int n_t,
+                       int kind, int fmt, float gscale, const float* gs_amax, float* gs_out, uint8_t* codes,
+                       void* scales, float* ydbg, cudaStream_t st) {
   if (d_in % 8 || rows > (int64_t(1) << 30) || d_in > (int64_t(1) << 30) || rows * (d_in / 2) > (int64_t(1) << 62))
     return WUSH_ERR_UNSUPPORTED;
   if (fmt == WUSH_FMT_MXFP4)
-    return dispatch_kind<32, kMx>(kind, x, rows, d_in, t, gscale, nullptr, nullptr, codes, scales, ydbg, st);
+    return dispatch_kind<32, kMx>(kind, x, rows, d_in, t, t_index, n_t, gscale, nullptr, nullptr, codes, scales,
+                                  ydbg, st);
   if (fmt == WUSH_FMT_NVFP4)
-    return dispatch_kind<16, kNv>(kind, x, rows, d_in, t, gscale, gs_amax, gs_out, codes, scales, ydbg, st);
-  return dispatch_kind<32, kI4>(kind, x, rows, d_in, t, gscale, nullptr, nullptr, codes, scales, ydbg, st);
+    return dispatch_kind<16, kNv>(kind, x, rows, d_in, t, t_index, n_t, gscale, gs_amax, gs_out, codes, scales,
+                                  ydbg, st);
+  return dispatch_kind<32, kI4>(kind, x, rows, d_in, t, t_index, n_t, gscale, nullptr, nullptr, codes, scales, ydbg,
+                                st);
 }
 
 }  // namespace wush

@@ -214,12 +214,16 @@ class OracleLeg:
     work, as on the GPU side); ``step(rows)`` is the timed part.
     """
 
-    def __init__(self, w, x, wt, xc, fmt, kind):
+    def __init__(self, w, x, wt, xc, fmt, kind, groups=0):
         from oracle import calibrate as C
         from oracle import quant as Q
         from oracle import transforms as T
         self.w, self.x, self.fmt = w, x, fmt
-        tx, tw = C.calibrate(xc, wt, w.block, kind)
+        if groups:      # shared transforms, expanded to one per block
+            sx, sw, idx = C.shared_transforms(C.block_moments(xc, w.block), C.block_moments(wt, w.block), kind, groups)
+            tx, tw = sx[idx], sw[idx]
+        else:
+            tx, tw = C.calibrate(xc, wt, w.block, kind)
         self.tx, tw = tx.astype(np.float32), tw.astype(np.float32)
         self.gx = gw = None
         if fmt == "nvfp4":
@@ -240,8 +244,8 @@ class OracleLeg:
         return int(min(self.w.tokens, max(16, 16 * seconds / max(dt, 1e-3))))
 
 
-def time_oracle(w, x, wt, xc, fmt, kind, target_s=12.0):
-    leg = OracleLeg(w, x, wt, xc, fmt, kind)
+def time_oracle(w, x, wt, xc, fmt, kind, target_s=12.0, groups=0):
+    leg = OracleLeg(w, x, wt, xc, fmt, kind, groups)
     rows = leg.rows_for(target_s / 3)
     t0 = time.perf_counter()
     reps = 0
@@ -275,8 +279,23 @@ def run_gpu(args, rank, world):
     b = w.block
 
     # offline: calibration (host C++), weight transform + quantisation (GPU), NVFP4 scales
-    tx, tw = aq.wush_calibrate(xc, wt, b, kind)
+    groups = args.share_groups
+    if groups:
+        if kind in ("identity", "hadamard"):
+            raise SystemExit("--share-groups needs a dense transform (wus, wush, wush_diag)")
+        tx_s, tw_s, t_idx = aq.wush_calibrate_shared(xc, wt, b, kind, groups)
+        tx, tw = tx_s[t_idx], tw_s[t_idx]                  # expanded, for the offline NVFP4 scales
+        t_xs, t_ws = torch.from_numpy(tx_s).to(dev), torch.from_numpy(tw_s).to(dev)
+        t_idx_dev = torch.from_numpy(t_idx).to(dev)
+    else:
+        tx, tw = aq.wush_calibrate(xc, wt, b, kind)
     t_x, t_w = torch.from_numpy(tx).to(dev), torch.from_numpy(tw).to(dev)
+
+    def quant(x_in, t_full, t_shared, fmt_, codes_, scales_, gs_, stream_=None):
+        if groups:
+            aq.wush_transform_quant_indexed(x_in, t_shared, t_idx_dev, kind, fmt_, codes_, scales_, gs_, stream=stream_)
+        else:
+            aq.wush_transform_quant(x_in, t_full, kind, fmt_, codes_, scales_, gs_, stream=stream_)
     gx = gw = 0.0
     if fmt == "nvfp4":
         amax = torch.empty(1, dtype=torch.float32, device=dev)
@@ -290,7 +309,7 @@ def run_gpu(args, rank, world):
     wcodes = []
     for _ in range(ROTATIONS):
         bc, bs = aq.alloc_quant_outputs(N, K, fmt, dev)
-        aq.wush_transform_quant(torch.from_numpy(wt).to(torch.bfloat16).to(dev), t_w, kind, fmt, bc, bs, gw)
+        quant(torch.from_numpy(wt).to(torch.bfloat16).to(dev), t_w, t_ws if groups else None, fmt, bc, bs, gw)
         wcodes.append((bc, bs))
     acodes = [aq.alloc_quant_outputs(M, K, fmt, dev) for _ in range(ROTATIONS)]
     y = torch.empty((M, N), dtype=torch.float32, device=dev)
@@ -302,6 +321,8 @@ def run_gpu(args, rank, world):
     # on the device (an amax pass over T x, then the quantiser and the GEMM's alpha
     # read it), instead of the static calibrated scale
     dynamic = fmt == "nvfp4" and args.dynamic_scale
+    if dynamic and groups:
+        raise SystemExit("--share-groups applies to the static-scale path only")
     dyn_amax = torch.zeros(1, dtype=torch.float32, device=dev)
     dyn_gs = torch.zeros(1, dtype=torch.float32, device=dev)
 
@@ -311,7 +332,7 @@ def run_gpu(args, rank, world):
             aq.wush_transform_quant_nvfp4_dynamic(x_in, t_x, kind, dyn_amax, acode[0], acode[1], dyn_gs,
                                                   stream=stream)
         else:
-            aq.wush_transform_quant(x_in, t_x, kind, fmt, acode[0], acode[1], gx, stream=stream)
+            quant(x_in, t_x, t_xs if groups else None, fmt, acode[0], acode[1], gx, stream)
 
     def tq(r):
         tq_into(xs[r], acodes[r])
@@ -490,9 +511,12 @@ def run_gpu(args, rank, world):
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "e2m1 x e2m1 -> fp32 (transform in fp32)", "data": "synthetic",
-            "config": dict(describe(w, fmt, kind), **({"nvfp4_scale": "dynamic: device amax pass + scale every step "
-                                                                 "(inside the transform's time)"}
-                                                       if dynamic else {})),
+            "config": dict(describe(w, fmt, kind),
+                           **({"nvfp4_scale": "dynamic: device amax pass + scale every step "
+                                              "(inside the transform's time)"} if dynamic else {}),
+                           **({"transform_sharing": f"{groups} shared transforms for {K // b} blocks "
+                                                    f"({groups * b * b * 4} B of T_X instead of {K * b * 4} B)"}
+                              if groups else {})),
             "transform_quant": {"us": tq_us, "GB_s": tq_gbs, "bytes_per_launch": tq_bytes,
                                 "frac_of_hbm": tq_gbs / peaks["hbm_gbs"], "dram_bytes_per_launch": tq_traffic,
                                 "burst_us": tq_burst_us,
@@ -574,6 +598,8 @@ def main():
     ap.add_argument("--transform", default=None, choices=["identity", "hadamard", "wus", "wush", "wush_diag"],
                     help="override the workload's block transform (calibrated from the same tokens)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--share-groups", type=int, default=0,
+                    help="share the dense transforms among this many groups of similar blocks")
     ap.add_argument("--dynamic-scale", action="store_true",
                     help="NVFP4: derive the activations' per-tensor scale on the device every step")
     args = ap.parse_args()
@@ -592,7 +618,7 @@ def main():
         if rank != 0:
             return
         w, x, wt, xc = build_inputs(args.workload, args.tokens)
-        leg = OracleLeg(w, x, wt, xc, spec["fmt"], spec["kind"])
+        leg = OracleLeg(w, x, wt, xc, spec["fmt"], spec["kind"], args.share_groups)
         step_rows = leg.rows_for(1.5)
         times = []
         for i in range(args.warmup + args.steps):
@@ -619,7 +645,7 @@ def main():
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
             w, x, wt, xc, fmt, kind = ctx
-            result["cpu_baseline"] = time_oracle(w, x, wt, xc, fmt, kind)
+            result["cpu_baseline"] = time_oracle(w, x, wt, xc, fmt, kind, groups=args.share_groups)
         print(json.dumps(result))
     if world > 1:
         import torch.distributed as dist

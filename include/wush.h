@@ -108,6 +108,25 @@ int wush_calibrate(const float* x_calib, int64_t n_calib, const float* w, int64_
 int wush_calibrate_from_moments(const double* sigma_x, const double* sigma_w, int64_t d_in,
                                 int block, int kind, float* t_x, float* t_w);
 
+/* Transform sharing (WUSH news article, paragraph 6: share transform matrices
+ * between similar blocks; the pages give no algorithm).  The d_in/block blocks
+ * are put in ``groups`` groups by k-means over their moments divided by their
+ * traces (both moments, flattened): centres start at blocks
+ * round(g * nb / groups) (halves to even), squared Euclidean distance, ties to
+ * the lowest group, empty groups keep their centre, until no block moves (at most
+ * 50 rounds).  Each group's transform (kind WUS, WUSH or WUSH_DIAG) comes from
+ * its members' mean moments (a group left empty: from its starting block).
+ * Outputs: t_x, t_w host fp32 [groups, block, block]; index host int32
+ * [d_in/block], block j -> group.  1 <= groups <= d_in/block; apply with
+ * wush_transform_quant_indexed.  groups = d_in/block reproduces the per-block
+ * transforms. */
+int wush_calibrate_shared(const float* x_calib, int64_t n_calib, const float* w, int64_t d_out,
+                          int64_t d_in, int block, int kind, int groups, float* t_x, float* t_w,
+                          int32_t* index);
+int wush_calibrate_shared_from_moments(const double* sigma_x, const double* sigma_w, int64_t d_in,
+                                       int block, int kind, int groups, float* t_x, float* t_w,
+                                       int32_t* index);
+
 /* ---------------------------------------------------------------------------
  * Output buffer sizes for wush_transform_quant (bytes)
  *
@@ -158,6 +177,16 @@ size_t wush_scales_bytes(int64_t rows, int64_t d_in, int fmt);
 int wush_transform_quant(const void* x, int x_dtype, int64_t rows, int64_t d_in,
                          const float* t, int kind, int fmt, float global_scale,
                          uint8_t* codes, void* scales, float* y_debug, void* stream);
+
+/* wush_transform_quant with shared transforms: block j of every row uses
+ * t[t_index[j]].  t: device fp32 [n_t, b, b]; t_index: device int32 [d_in/b]
+ * (4-byte aligned), each entry clamped to [0, n_t - 1] on use; kind WUS, WUSH or
+ * WUSH_DIAG (WUSH_ERR_INVALID_ARG otherwise).  Other arguments as in
+ * wush_transform_quant.  With t_index[j] = j it equals wush_transform_quant. */
+int wush_transform_quant_indexed(const void* x, int x_dtype, int64_t rows, int64_t d_in,
+                                 const float* t, const int32_t* t_index, int n_t, int kind, int fmt,
+                                 float global_scale, uint8_t* codes, void* scales, float* y_debug,
+                                 void* stream);
 
 /* max |T x| over a whole [rows, d_in] tensor, written as one fp32 to device
  * *amax_out (the call zeroes it first, in stream order).  Used offline for the

@@ -157,3 +157,54 @@ def nvfp4_dynamic_global_scale(y_rows: np.ndarray) -> np.float32:
     amax = np.float32(np.max(np.abs(np.asarray(y_rows, dtype=np.float32)))) if np.size(y_rows) else np.float32(0)
     g = np.float32(np.float64(amax) / 2688.0)
     return g if g >= np.float32(1e-30) else np.float32(1.0)
+
+
+def group_blocks(sigma_x: np.ndarray, sigma_w: np.ndarray, groups: int, iters: int = 50) -> np.ndarray:
+    """Block -> group index [nb] for transform sharing (WUSH news article,
+    paragraph 6: share transform matrices between similar blocks).
+
+    Reading (the pages give no algorithm): blocks are similar when their second
+    moments have a similar shape.  Each block's feature is its two moments
+    divided by their traces, flattened; k-means (Lloyd) groups the features with
+    centres started at blocks round(i * nb / groups), squared Euclidean distance,
+    ties to the lowest group, empty groups keeping their centre, until no block
+    changes group (at most ``iters`` rounds).
+    """
+    nb = sigma_x.shape[0]
+    if not 1 <= groups <= nb:
+        raise ValueError(groups)
+
+    def unit(s):
+        tr = np.trace(s, axis1=1, axis2=2)[:, None, None]
+        return s / np.where(tr > 0, tr, 1.0)
+
+    feat = np.concatenate([unit(sigma_x).reshape(nb, -1), unit(sigma_w).reshape(nb, -1)], axis=1)
+    centres = feat[[int(round(i * nb / groups)) for i in range(groups)]].copy()
+    assign = np.full(nb, -1)
+    for _ in range(iters):
+        d = ((feat[:, None, :] - centres[None, :, :]) ** 2).sum(axis=2)
+        new = np.argmin(d, axis=1)                     # first minimum: ties to the lowest group
+        if np.array_equal(new, assign):
+            break
+        assign = new
+        for g in range(groups):
+            members = assign == g
+            if members.any():
+                centres[g] = feat[members].mean(axis=0)
+    return assign
+
+
+def shared_transforms(sigma_x: np.ndarray, sigma_w: np.ndarray, kind: str, groups: int):
+    """(T_X [groups, b, b], T_W [groups, b, b], index [nb]) with one transform per
+    group of similar blocks, computed from the group's mean moments."""
+    index = group_blocks(sigma_x, sigma_w, groups)
+    nb = sigma_x.shape[0]
+    start = [int(round(g * nb / groups)) for g in range(groups)]
+    # a group left empty (its start tied with an earlier group's) maps no block; its
+    # transform comes from its starting block's moments
+    sx = np.stack([sigma_x[index == g].mean(axis=0) if (index == g).any() else sigma_x[start[g]]
+                   for g in range(groups)])
+    sw = np.stack([sigma_w[index == g].mean(axis=0) if (index == g).any() else sigma_w[start[g]]
+                   for g in range(groups)])
+    tx, tw = transforms_from_moments(sx, sw, kind)
+    return tx, tw, index

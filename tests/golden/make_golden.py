@@ -31,6 +31,12 @@ def tiny_layer_losses():
                 gs = calibrate.nvfp4_global_scale(
                     transforms.apply_block_transform(xc, tx32).astype(np.float32))
             out[f"{fmt}/{kind}"] = loss.layer_loss(x, wt, tx32, tw32, fmt, gs)
+    # WUSH shared among groups of similar blocks (MXFP4, 8 blocks of 32)
+    mx, mw = calibrate.block_moments(xc, 32), calibrate.block_moments(wt, 32)
+    for groups in (1, 2, 4):
+        sx, sw, idx = calibrate.shared_transforms(mx, mw, "wush", groups)
+        out[f"mxfp4/wush_shared{groups}"] = loss.layer_loss(x, wt, sx[idx].astype(np.float32),
+                                                            sw[idx].astype(np.float32), "mxfp4")
     return out
 
 

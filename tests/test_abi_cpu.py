@@ -97,3 +97,21 @@ def test_argument_validation_before_launch():
     assert lib.wush_calibrate(None, 0, None, 0, 64, 24, 3, 16, 16) == -1                      # block
     assert lib.itq3_quantize_weights(16, 4, 100, 16, 16) == -1
     assert lib.wush_status_string(-5) == b"a bounded device wait gave up"
+
+
+@pytest.mark.parametrize("kind", ["wus", "wush", "wush_diag"])
+def test_calibrate_shared_matches_oracle(kind):
+    w = synth.WORKLOADS["tiny"]
+    xc, wt = synth.activations(w, calib=True), synth.weights(w)
+    for b in (16, 32):
+        for groups in (1, 2, 3, 256 // b):
+            tx, tw, idx = aq.wush_calibrate_shared(xc, wt, b, kind, groups)
+            ox, ow, oidx = C.shared_transforms(C.block_moments(xc, b), C.block_moments(wt, b), kind, groups)
+            assert np.array_equal(idx, oidx)
+            for got, want in ((tx, ox), (tw, ow)):
+                scale = np.abs(want).max(axis=(1, 2), keepdims=True)
+                assert np.max(np.abs(got - want) / scale) < 1e-6
+    with pytest.raises(aq.WushError):
+        aq.wush_calibrate_shared(xc, wt, 32, kind, 0)
+    with pytest.raises(aq.WushError):
+        aq.wush_calibrate_shared(xc, wt, 32, kind, 9)      # more groups than blocks

@@ -192,3 +192,43 @@ def test_full_size_ring_repeatable(lib, kind, fmt):
     rng = np.random.default_rng(11)
     sel = np.unique(np.concatenate([rng.integers(0, w.tokens, 48), [0, w.tokens - 1]]))
     P.compare_transform_quant(x, t, fmt, gs if fmt == "nvfp4" else None, c, s, None, rows_sel=sel)
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4", "int4"])
+@pytest.mark.parametrize("bf16", [True, False])
+def test_indexed_transforms_equal_expanded(lib, fmt, bf16):
+    # shared transforms (4 groups of similar blocks) through the index map give the
+    # same codes and scales as the same transforms expanded to one per block; two
+    # planted out-of-range entries are clamped to the first and last transform
+    w = synth.WORKLOADS[FMT_WORKLOAD[fmt]]
+    b = P.Q.BLOCK[fmt]
+    x = synth.activations(w, tokens=300)
+    xc, wt = _calib_inputs(w.name, 1024)
+    tx, _, idx = C.shared_transforms(C.block_moments(xc, b), C.block_moments(wt, b), "wush", 4)
+    ts = tx.astype(np.float32)
+    idx = idx.astype(np.int32)
+    idx[0], idx[-1] = -3, 99
+    t_full = ts[np.clip(idx, 0, len(ts) - 1)]
+    gs = _global_scale(x, t_full, fmt)
+    xt = _as_input(x, bf16).cuda()
+    rows, d_in = x.shape
+    c1, s1 = lib.alloc_quant_outputs(rows, d_in, fmt)
+    c2, s2 = lib.alloc_quant_outputs(rows, d_in, fmt)
+    lib.wush_transform_quant_indexed(xt, torch.from_numpy(ts).cuda(), torch.from_numpy(idx).cuda(), "wush", fmt,
+                                     c1, s1, gs)
+    lib.wush_transform_quant(xt, torch.from_numpy(t_full).cuda(), "wush", fmt, c2, s2, gs)
+    torch.cuda.synchronize()
+    assert lib.wush_check_device_status() == 0
+    assert torch.equal(c1, c2) and torch.equal(s1, s2)
+    P.compare_transform_quant(x, t_full, fmt, gs if fmt == "nvfp4" else None,
+                              P.unpack_nibbles(c1.cpu().numpy(), rows, d_in), P.decode_scales(s1.cpu().numpy(), rows, d_in, fmt))
+
+
+def test_indexed_transform_rejects_non_dense_kinds(lib):
+    xt = torch.zeros((128, 256), dtype=torch.bfloat16, device="cuda")
+    t = torch.zeros((1, 32, 32), dtype=torch.float32, device="cuda")
+    idx = torch.zeros(8, dtype=torch.int32, device="cuda")
+    codes, scales = lib.alloc_quant_outputs(128, 256, "mxfp4")
+    for kind in ("identity", "hadamard"):
+        with pytest.raises(lib.WushError):
+            lib.wush_transform_quant_indexed(xt, t, idx, kind, "mxfp4", codes, scales)

@@ -122,6 +122,11 @@ def test_tiny_losses_regression_and_claims():
     for fmt in ("mxfp4", "nvfp4", "int4"):
         assert gold[f"{fmt}/wush_diag"] < min(gold[f"{fmt}/identity"], gold[f"{fmt}/hadamard"])
         assert gold[f"{fmt}/wush_diag"] < 1.1 * gold[f"{fmt}/wush"]
+    # Sharing transforms among groups of similar blocks (paragraph 6 offers it to save
+    # storage) keeps most of WUSH's gain on this layer even with one or two groups.
+    for groups in (1, 2, 4):
+        assert gold[f"mxfp4/wush_shared{groups}"] < gold["mxfp4/hadamard"]
+    assert gold["mxfp4/wush_shared4"] < gold["mxfp4/wush_shared1"]
 
 
 def test_wush_diag_two_by_two_closed_form():
@@ -186,3 +191,62 @@ def test_nvfp4_dynamic_global_scale_rule():
         nbrs = (np.nextafter(g, np.float32(0)), np.nextafter(g, np.float32(np.inf)))
         assert all(abs(Fraction(float(g)) - exact) <= abs(Fraction(float(n)) - exact) for n in nbrs)
         assert g == C.nvfp4_global_scale(np.array([a]))                       # same rule as the static scale
+
+
+def _block_family_moments(nb=8, b=16, seed=11):
+    # two moment shapes, A on even blocks and B on odd ones, each block scaled by
+    # its own positive factor: trace-normalised features coincide within a family
+    rng = np.random.default_rng(seed)
+    fa, fb = rng.standard_normal((b, b)), rng.standard_normal((b, b))
+    a, bm = fa @ fa.T + b * np.eye(b), fb @ fb.T + 0.1 * np.eye(b)
+    wa = rng.standard_normal((b, b)); wa = wa @ wa.T + np.eye(b)
+    sx = np.stack([(a if j % 2 == 0 else bm) * rng.uniform(0.5, 4.0) for j in range(nb)])
+    sw = np.stack([wa * rng.uniform(0.5, 4.0) for _ in range(nb)])
+    return sx, sw
+
+
+def test_shared_transforms_with_one_group_per_block_are_per_block():
+    _, _, sx, sw = _moments(9)
+    sx = np.stack([sx, 2 * sx + np.eye(32), sx.T @ sx / 10 + np.eye(32)])
+    sw = np.stack([sw, sw + 0.1 * np.eye(32), 3 * sw])
+    tx, tw, idx = C.shared_transforms(sx, sw, "wush", 3)
+    assert list(idx) == [0, 1, 2]
+    px, pw = C.transforms_from_moments(sx, sw, "wush")
+    assert np.allclose(tx, px, rtol=1e-13, atol=1e-13) and np.allclose(tw, pw, rtol=1e-13, atol=1e-13)
+
+
+def test_shared_transforms_one_group_uses_mean_moments():
+    sx, sw = _block_family_moments()
+    tx, tw, idx = C.shared_transforms(sx, sw, "wush", 1)
+    assert not idx.any()
+    want_x, want_w = C.block_transform_pair(sx.mean(axis=0), sw.mean(axis=0), "wush")
+    assert np.allclose(tx[0], want_x, rtol=1e-13, atol=1e-13) and np.allclose(tw[0], want_w, rtol=1e-13, atol=1e-13)
+
+
+def test_group_blocks_separates_planted_families_and_converges():
+    sx, sw = _block_family_moments()
+    idx = C.group_blocks(sx, sw, 2)
+    # the partition, not its labels: both centres start on even blocks here
+    assert len(set(idx[0::2])) == 1 and len(set(idx[1::2])) == 1 and idx[0] != idx[1]
+    # converged Lloyd: every block sits in its nearest group centre
+    rng = np.random.default_rng(4)
+    sx2 = np.stack([s + np.diag(rng.uniform(0, 3, 16)) for s in sx])
+    for g in (2, 3, 5):
+        idx = C.group_blocks(sx2, sw, g)
+        unit = lambda s: s / np.trace(s, axis1=1, axis2=2)[:, None, None]
+        feat = np.concatenate([unit(sx2).reshape(8, -1), unit(sw).reshape(8, -1)], axis=1)
+        cen = np.stack([feat[idx == k].mean(axis=0) for k in range(g) if (idx == k).any()])
+        used = [k for k in range(g) if (idx == k).any()]
+        d = ((feat[:, None, :] - cen[None]) ** 2).sum(axis=2)
+        assert all(used[int(np.argmin(d[j]))] == idx[j] for j in range(8))
+
+
+def test_group_blocks_empty_group_rule():
+    # identical blocks: every distance ties, all blocks join group 0, group 1 stays
+    # empty and takes its starting block's moments
+    _, _, sx, sw = _moments(3)
+    sxs, sws = np.stack([sx] * 4), np.stack([sw] * 4)
+    tx, tw, idx = C.shared_transforms(sxs, sws, "wush", 2)
+    assert not idx.any()
+    one_x, one_w = C.block_transform_pair(sx, sw, "wush")
+    assert np.allclose(tx, one_x) and np.allclose(tw, one_w)
