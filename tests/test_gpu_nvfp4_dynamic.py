@@ -120,3 +120,26 @@ def test_dynamic_rejects_missing_amax(lib):
     y = torch.zeros(128 * 128, dtype=torch.float32, device="cuda")
     with pytest.raises(lib.WushError):
         lib.wush_qgemm_nvfp4_dynamic(z, z, z, z, 128, 128, 256, None, 1.0, y)
+
+
+@pytest.mark.parametrize("m, n", [(256, 256), (128, 256), (128, 384)])   # pair, 128 x 256, 128 x 128 tiles
+def test_dynamic_alpha_in_every_gemm_kernel(lib, m, n):
+    # random NVFP4 operands; the device factor must give the same y as host alpha,
+    # bit for bit, in each of the GEMM's kernel forms
+    k = 512
+    rng = np.random.default_rng(m + n)
+    a_codes = torch.from_numpy(rng.integers(0, 256, m * k // 2, dtype=np.uint8)).cuda()
+    b_codes = torch.from_numpy(rng.integers(0, 256, n * k // 2, dtype=np.uint8)).cuda()
+    def scales(rows):
+        sb = (0x28 + rng.integers(0, 0x30, (rows, k // 16))).astype(np.uint8)   # UE4M3 0.03 .. 30
+        return torch.from_numpy(P.swizzle_scales(sb)).cuda()
+    a_s, b_s = scales(m), scales(n)
+    gx = torch.tensor([0.0123], dtype=torch.float32, device="cuda")
+    gw = 0.0377
+    y_dyn = torch.full((m, n), float("nan"), dtype=torch.float32, device="cuda")
+    y_sta = torch.full((m, n), float("nan"), dtype=torch.float32, device="cuda")
+    lib.wush_qgemm_nvfp4_dynamic(a_codes, a_s, b_codes, b_s, m, n, k, gx, gw, y_dyn)
+    lib.wush_qgemm(a_codes, a_s, b_codes, b_s, m, n, k, "nvfp4", float(np.float32(0.0123) * np.float32(gw)), y_sta)
+    torch.cuda.synchronize()
+    assert lib.wush_check_device_status() == 0
+    assert torch.isfinite(y_dyn).all() and torch.equal(y_dyn, y_sta)
