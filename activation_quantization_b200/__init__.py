@@ -34,6 +34,9 @@ _SIGNATURES = {
     "wush_calibrate_from_moments": (_i32, [_vp, _vp, _i64, _i32, _i32, _vp, _vp]),
     "wush_calibrate_shared": (_i32, [_vp, _i64, _vp, _i64, _i64, _i32, _i32, _i32, _vp, _vp, _vp]),
     "wush_calibrate_shared_from_moments": (_i32, [_vp, _vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp]),
+    "wush_save_transforms": (_i32, [ctypes.c_char_p, _i32, _i32, _i64, _vp, _vp, _vp, _i64]),
+    "wush_transforms_file_info": (_i32, [ctypes.c_char_p, _vp, _vp, _vp, _vp, _vp]),
+    "wush_load_transforms": (_i32, [ctypes.c_char_p, _vp, _vp, _i64, _vp, _i64]),
     "wush_codes_bytes": (_sz, [_i64, _i64, _i32]),
     "wush_scales_bytes": (_sz, [_i64, _i64, _i32]),
     "wush_transform_quant": (_i32, [_vp, _i32, _i64, _i64, _vp, _i32, _i32, _f32, _vp, _vp, _vp, _vp]),
@@ -137,6 +140,45 @@ def wush_calibrate_shared(x_calib: np.ndarray, w: np.ndarray, block: int, kind, 
            _lib.wush_calibrate_shared(xp, x.shape[0], wp, wt.shape[0], d_in, block, _enum(TRANSFORMS, kind),
                                       int(groups), tx.ctypes.data, tw.ctypes.data, index.ctypes.data))
     return tx, tw, index
+
+
+def wush_save_transforms(path, t_x: np.ndarray, t_w: np.ndarray, kind, index: np.ndarray | None = None):
+    """Write fp32 T_X, T_W [n_t, b, b] (and the block -> transform index, if given) to ``path``."""
+    tx, txp = _host(t_x, np.float32)
+    tw, twp = _host(t_w, np.float32)
+    if tx.ndim != 3 or tx.shape != tw.shape or tx.shape[1] != tx.shape[2]:
+        raise ValueError("t_x and t_w must both be [n_t, b, b]")
+    ip, n_blocks = None, 0
+    if index is not None:
+        idx, ip = _host(index, np.int32)
+        n_blocks = idx.size
+    _check("wush_save_transforms",
+           _lib.wush_save_transforms(os.fsencode(path), tx.shape[1], _enum(TRANSFORMS, kind), tx.shape[0],
+                                     txp, twp, ip, n_blocks))
+
+
+def wush_transforms_file_info(path) -> dict:
+    """Header of a transforms file: block, kind, n_t, n_blocks, has_index."""
+    b, k, hi = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    nt, nb = ctypes.c_int64(), ctypes.c_int64()
+    _check("wush_transforms_file_info",
+           _lib.wush_transforms_file_info(os.fsencode(path), ctypes.byref(b), ctypes.byref(k), ctypes.byref(nt),
+                                          ctypes.byref(nb), ctypes.byref(hi)))
+    return {"block": b.value, "kind": k.value, "n_t": nt.value, "n_blocks": nb.value, "has_index": bool(hi.value)}
+
+
+def wush_load_transforms(path):
+    """(t_x, t_w, index or None, kind) from a file written by wush_save_transforms."""
+    info = wush_transforms_file_info(path)
+    b, nt = info["block"], info["n_t"]
+    tx = np.empty((nt, b, b), np.float32)
+    tw = np.empty_like(tx)
+    index = np.empty(info["n_blocks"], np.int32) if info["has_index"] else None
+    _check("wush_load_transforms",
+           _lib.wush_load_transforms(os.fsencode(path), tx.ctypes.data, tw.ctypes.data, tx.size,
+                                     None if index is None else index.ctypes.data,
+                                     0 if index is None else index.size))
+    return tx, tw, index, info["kind"]
 
 
 def wush_calibrate_shared_from_moments(sigma_x: np.ndarray, sigma_w: np.ndarray, kind, groups: int):

@@ -20,7 +20,7 @@ LIB = os.path.join(HERE, "libwush.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 CU_SOURCES = ["api.cu", "transform_quant.cu", "transform_quant_tc.cu", "qgemm.cu", "qgemm_int4.cu", "itq3_gemv.cu", "itq3_tc.cu"]
-CPP_SOURCES = ["calibrate.cpp", "itq3_host.cpp"]
+CPP_SOURCES = ["calibrate.cpp", "itq3_host.cpp", "transforms_io.cpp"]
 # Files whose rounding decisions must follow the written order of operations exactly.
 NO_FMAD = {"transform_quant.cu", "transform_quant_tc.cu"}
 

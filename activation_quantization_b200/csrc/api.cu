@@ -17,6 +17,7 @@ extern "C" const char* wush_status_string(int status) {
     case WUSH_ERR_CUDA: return "CUDA error";
     case WUSH_ERR_TIMEOUT: return "a bounded device wait gave up";
     case WUSH_ERR_BUFFER_TOO_SMALL: return "buffer too small";
+    case WUSH_ERR_IO: return "file could not be opened, read or written";
     default: return "unknown status";
   }
 }

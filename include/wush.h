@@ -53,7 +53,8 @@ typedef enum {
   WUSH_ERR_NOT_SPD = -3,
   WUSH_ERR_CUDA = -4,
   WUSH_ERR_TIMEOUT = -5,
-  WUSH_ERR_BUFFER_TOO_SMALL = -6
+  WUSH_ERR_BUFFER_TOO_SMALL = -6,
+  WUSH_ERR_IO = -7
 } wush_status;
 
 typedef enum { WUSH_FMT_MXFP4 = 0, WUSH_FMT_NVFP4 = 1, WUSH_FMT_INT4 = 2 } wush_format;
@@ -126,6 +127,39 @@ int wush_calibrate_shared(const float* x_calib, int64_t n_calib, const float* w,
 int wush_calibrate_shared_from_moments(const double* sigma_x, const double* sigma_w, int64_t d_in,
                                        int block, int kind, int groups, float* t_x, float* t_w,
                                        int32_t* index);
+
+/* ---------------------------------------------------------------------------
+ * Checkpointing calibrated transforms (host, no CUDA)
+ *
+ * Calibration runs once, offline, and every block's matrices need storage
+ * (WUSH news article, paragraph 6); these calls write and read its output.  File layout, little-endian: the 8 bytes "WUSHTRF1", u32 version
+ * (1), u32 block size b, u32 kind (wush_transform), u32 has_index, i64 n_t, i64
+ * n_blocks, then fp32 T_X [n_t, b, b], fp32 T_W [n_t, b, b] (row-major per
+ * block) and, when has_index is 1, int32 index [n_blocks] (block j of d_in uses
+ * transform index[j]).  Without an index n_blocks = n_t.
+ *
+ * wush_save_transforms: t_x, t_w host fp32 [n_t, b, b]; index host int32
+ * [n_blocks] or NULL (then n_blocks is ignored).  b a power of two in [2, 256],
+ * kind a wush_transform value, every index entry in [0, n_t): else
+ * WUSH_ERR_INVALID_ARG before the file is opened.  WUSH_ERR_IO when the file
+ * cannot be opened or fully written (a partial file may remain).
+ *
+ * wush_transforms_file_info: reads the header only and returns its fields.
+ *
+ * wush_load_transforms: reads the whole file into t_x and t_w (capacity_floats
+ * floats each, at least n_t * b * b) and, when the file holds an index, into
+ * index (index_capacity entries, at least n_blocks): WUSH_ERR_BUFFER_TOO_SMALL
+ * otherwise, with nothing read.  WUSH_ERR_IO when the file cannot be opened or
+ * its header is cut short; WUSH_ERR_INVALID_ARG for a wrong magic or version, a
+ * header outside the limits above, a body cut short or followed by extra bytes,
+ * or an index entry out of range (the buffers may then hold part of the file).
+ * ------------------------------------------------------------------------- */
+int wush_save_transforms(const char* path, int block, int kind, int64_t n_t, const float* t_x,
+                         const float* t_w, const int32_t* index, int64_t n_blocks);
+int wush_transforms_file_info(const char* path, int* block, int* kind, int64_t* n_t,
+                              int64_t* n_blocks, int* has_index);
+int wush_load_transforms(const char* path, float* t_x, float* t_w, int64_t capacity_floats,
+                         int32_t* index, int64_t index_capacity);
 
 /* ---------------------------------------------------------------------------
  * Output buffer sizes for wush_transform_quant (bytes)
