@@ -34,8 +34,8 @@ _SIGNATURES = {
     "wush_calibrate_from_moments": (_i32, [_vp, _vp, _i64, _i32, _i32, _vp, _vp]),
     "wush_calibrate_shared": (_i32, [_vp, _i64, _vp, _i64, _i64, _i32, _i32, _i32, _vp, _vp, _vp]),
     "wush_calibrate_shared_from_moments": (_i32, [_vp, _vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp]),
-    "wush_save_transforms": (_i32, [ctypes.c_char_p, _i32, _i32, _i64, _vp, _vp, _vp, _i64]),
-    "wush_transforms_file_info": (_i32, [ctypes.c_char_p, _vp, _vp, _vp, _vp, _vp]),
+    "wush_save_transforms": (_i32, [ctypes.c_char_p, _i32, _i32, _i32, _i64, _vp, _vp, _vp, _i64]),
+    "wush_transforms_file_info": (_i32, [ctypes.c_char_p, _vp, _vp, _vp, _vp, _vp, _vp]),
     "wush_load_transforms": (_i32, [ctypes.c_char_p, _vp, _vp, _i64, _vp, _i64]),
     "wush_codes_bytes": (_sz, [_i64, _i64, _i32]),
     "wush_scales_bytes": (_sz, [_i64, _i64, _i32]),
@@ -142,8 +142,14 @@ def wush_calibrate_shared(x_calib: np.ndarray, w: np.ndarray, block: int, kind, 
     return tx, tw, index
 
 
-def wush_save_transforms(path, t_x: np.ndarray, t_w: np.ndarray, kind, index: np.ndarray | None = None):
-    """Write fp32 T_X, T_W [n_t, b, b] (and the block -> transform index, if given) to ``path``."""
+SIGMA_NORMS = {"unknown": 0, "mean": 1}
+
+
+def wush_save_transforms(path, t_x: np.ndarray, t_w: np.ndarray, kind, index: np.ndarray | None = None,
+                         sigma_norm="mean"):
+    """Write fp32 T_X, T_W [n_t, b, b] (and the block -> transform index, if given) to ``path``.
+
+    ``sigma_norm`` "mean" is the normalisation of wush_calibrate*; "unknown" marks other transforms."""
     tx, txp = _host(t_x, np.float32)
     tw, twp = _host(t_w, np.float32)
     if tx.ndim != 3 or tx.shape != tw.shape or tx.shape[1] != tx.shape[2]:
@@ -153,18 +159,19 @@ def wush_save_transforms(path, t_x: np.ndarray, t_w: np.ndarray, kind, index: np
         idx, ip = _host(index, np.int32)
         n_blocks = idx.size
     _check("wush_save_transforms",
-           _lib.wush_save_transforms(os.fsencode(path), tx.shape[1], _enum(TRANSFORMS, kind), tx.shape[0],
-                                     txp, twp, ip, n_blocks))
+           _lib.wush_save_transforms(os.fsencode(path), tx.shape[1], _enum(TRANSFORMS, kind),
+                                     _enum(SIGMA_NORMS, sigma_norm), tx.shape[0], txp, twp, ip, n_blocks))
 
 
 def wush_transforms_file_info(path) -> dict:
-    """Header of a transforms file: block, kind, n_t, n_blocks, has_index."""
-    b, k, hi = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    """Header of a transforms file: block, kind, sigma_norm, n_t, n_blocks, has_index."""
+    b, k, sn, hi = ctypes.c_int(), ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
     nt, nb = ctypes.c_int64(), ctypes.c_int64()
     _check("wush_transforms_file_info",
-           _lib.wush_transforms_file_info(os.fsencode(path), ctypes.byref(b), ctypes.byref(k), ctypes.byref(nt),
-                                          ctypes.byref(nb), ctypes.byref(hi)))
-    return {"block": b.value, "kind": k.value, "n_t": nt.value, "n_blocks": nb.value, "has_index": bool(hi.value)}
+           _lib.wush_transforms_file_info(os.fsencode(path), ctypes.byref(b), ctypes.byref(k), ctypes.byref(sn),
+                                          ctypes.byref(nt), ctypes.byref(nb), ctypes.byref(hi)))
+    return {"block": b.value, "kind": k.value, "sigma_norm": sn.value, "n_t": nt.value, "n_blocks": nb.value,
+            "has_index": bool(hi.value)}
 
 
 def wush_load_transforms(path):

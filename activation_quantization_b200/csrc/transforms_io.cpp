@@ -10,6 +10,9 @@
 //   u32           version (1)
 //   u32           block size b
 //   u32           transform kind (wush_transform)
+//   u32           element type of the matrices (0 = fp32, the only one)
+//   u32           moment normalisation the transforms were calibrated with
+//                 (0 unknown, 1 means: Sigma_X / n_calib, Sigma_W / d_out)
 //   u32           1 if a block -> transform index follows, else 0
 //   i64           n_t, the number of transforms stored
 //   i64           n_blocks, the number of d_in blocks they serve (n_t when no index)
@@ -28,34 +31,39 @@ constexpr uint32_t kVersion = 1;
 
 struct Header {
   char magic[8];
-  uint32_t version, block, kind, has_index;
+  uint32_t version, block, kind, dtype, sigma_norm, has_index;
   int64_t n_t, n_blocks;
 };
-static_assert(sizeof(Header) == 40, "packed header");
+static_assert(sizeof(Header) == 48, "packed header");
 
-bool valid_shape(int block, int kind, int64_t n_t, int64_t n_blocks, bool has_index) {
+constexpr uint32_t kDtypeF32 = 0;
+
+bool valid_shape(int block, int kind, int sigma_norm, int64_t n_t, int64_t n_blocks, bool has_index) {
   if (block < 2 || block > 256 || (block & (block - 1))) return false;
   if (kind < WUSH_T_IDENTITY || kind > WUSH_T_WUSH_DIAG) return false;
+  if (sigma_norm < WUSH_NORM_UNKNOWN || sigma_norm > WUSH_NORM_MEAN) return false;
   if (n_t < 1 || n_blocks < 1 || n_t > (int64_t(1) << 32) || n_blocks > (int64_t(1) << 32)) return false;
   return has_index || n_t == n_blocks;
 }
 
 int read_header(FILE* f, Header* h) {
   if (std::fread(h, sizeof(Header), 1, f) != 1) return WUSH_ERR_IO;
-  if (std::memcmp(h->magic, kMagic, 8) != 0 || h->version != kVersion) return WUSH_ERR_INVALID_ARG;
-  if (!valid_shape(static_cast<int>(h->block), static_cast<int>(h->kind), h->n_t, h->n_blocks, h->has_index != 0))
+  if (std::memcmp(h->magic, kMagic, 8) != 0 || h->version != kVersion || h->dtype != kDtypeF32)
+    return WUSH_ERR_INVALID_ARG;
+  if (h->has_index > 1 || !valid_shape(static_cast<int>(h->block), static_cast<int>(h->kind),
+                                       static_cast<int>(h->sigma_norm), h->n_t, h->n_blocks, h->has_index != 0))
     return WUSH_ERR_INVALID_ARG;
   return WUSH_OK;
 }
 
 }  // namespace
 
-extern "C" int wush_save_transforms(const char* path, int block, int kind, int64_t n_t, const float* t_x,
-                                    const float* t_w, const int32_t* index, int64_t n_blocks) {
+extern "C" int wush_save_transforms(const char* path, int block, int kind, int sigma_norm, int64_t n_t,
+                                    const float* t_x, const float* t_w, const int32_t* index, int64_t n_blocks) {
   if (!path || !t_x || !t_w) return WUSH_ERR_INVALID_ARG;
   const bool has_index = index != nullptr;
   if (!has_index) n_blocks = n_t;
-  if (!valid_shape(block, kind, n_t, n_blocks, has_index)) return WUSH_ERR_INVALID_ARG;
+  if (!valid_shape(block, kind, sigma_norm, n_t, n_blocks, has_index)) return WUSH_ERR_INVALID_ARG;
   if (has_index)
     for (int64_t j = 0; j < n_blocks; ++j)
       if (index[j] < 0 || index[j] >= n_t) return WUSH_ERR_INVALID_ARG;
@@ -66,6 +74,8 @@ extern "C" int wush_save_transforms(const char* path, int block, int kind, int64
   h.version = kVersion;
   h.block = static_cast<uint32_t>(block);
   h.kind = static_cast<uint32_t>(kind);
+  h.dtype = kDtypeF32;
+  h.sigma_norm = static_cast<uint32_t>(sigma_norm);
   h.has_index = has_index ? 1u : 0u;
   h.n_t = n_t;
   h.n_blocks = n_blocks;
@@ -78,9 +88,9 @@ extern "C" int wush_save_transforms(const char* path, int block, int kind, int64
   return ok ? WUSH_OK : WUSH_ERR_IO;
 }
 
-extern "C" int wush_transforms_file_info(const char* path, int* block, int* kind, int64_t* n_t, int64_t* n_blocks,
-                                         int* has_index) {
-  if (!path || !block || !kind || !n_t || !n_blocks || !has_index) return WUSH_ERR_INVALID_ARG;
+extern "C" int wush_transforms_file_info(const char* path, int* block, int* kind, int* sigma_norm, int64_t* n_t,
+                                         int64_t* n_blocks, int* has_index) {
+  if (!path || !block || !kind || !sigma_norm || !n_t || !n_blocks || !has_index) return WUSH_ERR_INVALID_ARG;
   FILE* f = std::fopen(path, "rb");
   if (!f) return WUSH_ERR_IO;
   Header h;
@@ -89,6 +99,7 @@ extern "C" int wush_transforms_file_info(const char* path, int* block, int* kind
   if (st != WUSH_OK) return st;
   *block = static_cast<int>(h.block);
   *kind = static_cast<int>(h.kind);
+  *sigma_norm = static_cast<int>(h.sigma_norm);
   *n_t = h.n_t;
   *n_blocks = h.n_blocks;
   *has_index = static_cast<int>(h.has_index);

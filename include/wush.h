@@ -132,17 +132,26 @@ int wush_calibrate_shared_from_moments(const double* sigma_x, const double* sigm
  * Checkpointing calibrated transforms (host, no CUDA)
  *
  * Calibration runs once, offline, and every block's matrices need storage
- * (WUSH news article, paragraph 6); these calls write and read its output.  File layout, little-endian: the 8 bytes "WUSHTRF1", u32 version
- * (1), u32 block size b, u32 kind (wush_transform), u32 has_index, i64 n_t, i64
- * n_blocks, then fp32 T_X [n_t, b, b], fp32 T_W [n_t, b, b] (row-major per
+ * (WUSH news article, paragraph 6); these calls write and read its output.
+ *
+ * File layout, little-endian, 48 header bytes: the 8 bytes "WUSHTRF1", u32
+ * version (1), u32 block size b, u32 kind (wush_transform), u32 dtype (0 = fp32,
+ * the only one), u32 sigma_norm (wush_sigma_norm), u32 has_index, i64 n_t, i64
+ * n_blocks; then fp32 T_X [n_t, b, b], fp32 T_W [n_t, b, b] (row-major per
  * block) and, when has_index is 1, int32 index [n_blocks] (block j of d_in uses
  * transform index[j]).  Without an index n_blocks = n_t.
  *
+ * sigma_norm records how the second moments were normalised: the transforms
+ * scale with that choice by a factor that is not a power of two, so the codes
+ * depend on it.  wush_calibrate* use WUSH_NORM_MEAN (Sigma_X = X X^T / n_calib,
+ * Sigma_W = W W^T / d_out); WUSH_NORM_UNKNOWN marks transforms from elsewhere.
+ *
  * wush_save_transforms: t_x, t_w host fp32 [n_t, b, b]; index host int32
  * [n_blocks] or NULL (then n_blocks is ignored).  b a power of two in [2, 256],
- * kind a wush_transform value, every index entry in [0, n_t): else
- * WUSH_ERR_INVALID_ARG before the file is opened.  WUSH_ERR_IO when the file
- * cannot be opened or fully written (a partial file may remain).
+ * kind a wush_transform value, sigma_norm a wush_sigma_norm value, every index
+ * entry in [0, n_t): else WUSH_ERR_INVALID_ARG before the file is opened.
+ * WUSH_ERR_IO when the file cannot be opened or fully written (a partial file
+ * may remain).
  *
  * wush_transforms_file_info: reads the header only and returns its fields.
  *
@@ -150,14 +159,17 @@ int wush_calibrate_shared_from_moments(const double* sigma_x, const double* sigm
  * floats each, at least n_t * b * b) and, when the file holds an index, into
  * index (index_capacity entries, at least n_blocks): WUSH_ERR_BUFFER_TOO_SMALL
  * otherwise, with nothing read.  WUSH_ERR_IO when the file cannot be opened or
- * its header is cut short; WUSH_ERR_INVALID_ARG for a wrong magic or version, a
- * header outside the limits above, a body cut short or followed by extra bytes,
- * or an index entry out of range (the buffers may then hold part of the file).
+ * its header is cut short; WUSH_ERR_INVALID_ARG for a wrong magic, version or
+ * dtype, a header outside the limits above, a body cut short or followed by
+ * extra bytes, or an index entry out of range (the buffers may then hold part
+ * of the file).
  * ------------------------------------------------------------------------- */
-int wush_save_transforms(const char* path, int block, int kind, int64_t n_t, const float* t_x,
-                         const float* t_w, const int32_t* index, int64_t n_blocks);
-int wush_transforms_file_info(const char* path, int* block, int* kind, int64_t* n_t,
-                              int64_t* n_blocks, int* has_index);
+typedef enum { WUSH_NORM_UNKNOWN = 0, WUSH_NORM_MEAN = 1 } wush_sigma_norm;
+
+int wush_save_transforms(const char* path, int block, int kind, int sigma_norm, int64_t n_t,
+                         const float* t_x, const float* t_w, const int32_t* index, int64_t n_blocks);
+int wush_transforms_file_info(const char* path, int* block, int* kind, int* sigma_norm,
+                              int64_t* n_t, int64_t* n_blocks, int* has_index);
 int wush_load_transforms(const char* path, float* t_x, float* t_w, int64_t capacity_floats,
                          int32_t* index, int64_t index_capacity);
 

@@ -18,7 +18,7 @@ aq = pytest.importorskip("activation_quantization_b200")
 _lib = ctypes.CDLL(aq.LIB_PATH)
 
 OK, INVALID, TOO_SMALL, IO = 0, -1, -6, -7
-HDR = struct.Struct("<8sIIIIqq")
+HDR = struct.Struct("<8sIIIIIIqq")
 
 
 @pytest.fixture(scope="module")
@@ -32,7 +32,8 @@ def calibrated():
 
 def _parse(path):
     raw = open(path, "rb").read()
-    magic, ver, b, kind, has_index, n_t, n_blocks = HDR.unpack_from(raw, 0)
+    magic, ver, b, kind, dtype, norm, has_index, n_t, n_blocks = HDR.unpack_from(raw, 0)
+    assert HDR.size == 48
     off, m = HDR.size, n_t * b * b
     tx = np.frombuffer(raw, "<f4", m, off).reshape(n_t, b, b)
     tw = np.frombuffer(raw, "<f4", m, off + 4 * m).reshape(n_t, b, b)
@@ -42,7 +43,8 @@ def _parse(path):
         idx = np.frombuffer(raw, "<i4", n_blocks, off)
         off += 4 * n_blocks
     assert off == len(raw)
-    return dict(magic=magic, version=ver, block=b, kind=kind, n_t=n_t, n_blocks=n_blocks), tx, tw, idx
+    return dict(magic=magic, version=ver, block=b, kind=kind, dtype=dtype, sigma_norm=norm, n_t=n_t,
+                n_blocks=n_blocks), tx, tw, idx
 
 
 def test_per_block_round_trip_and_layout(tmp_path, calibrated):
@@ -50,8 +52,8 @@ def test_per_block_round_trip_and_layout(tmp_path, calibrated):
     p = tmp_path / "t.wush"
     aq.wush_save_transforms(p, tx, tw, "wush")
     hdr, fx, fw, fi = _parse(p)
-    assert hdr == dict(magic=b"WUSHTRF1", version=1, block=16, kind=aq.TRANSFORMS["wush"],
-                       n_t=tx.shape[0], n_blocks=tx.shape[0])
+    assert hdr == dict(magic=b"WUSHTRF1", version=1, block=16, kind=aq.TRANSFORMS["wush"], dtype=0,
+                       sigma_norm=1, n_t=tx.shape[0], n_blocks=tx.shape[0])
     assert fi is None and np.array_equal(fx, tx) and np.array_equal(fw, tw)
     lx, lw, li, kind = aq.wush_load_transforms(p)
     assert li is None and kind == aq.TRANSFORMS["wush"]
@@ -63,7 +65,8 @@ def test_shared_round_trip_keeps_index(tmp_path, calibrated):
     p = tmp_path / "s.wush"
     aq.wush_save_transforms(p, sx, sw, "wush", idx)
     info = aq.wush_transforms_file_info(p)
-    assert info == {"block": 16, "kind": aq.TRANSFORMS["wush"], "n_t": 2, "n_blocks": idx.size, "has_index": True}
+    assert info == {"block": 16, "kind": aq.TRANSFORMS["wush"], "sigma_norm": 1, "n_t": 2, "n_blocks": idx.size,
+                    "has_index": True}
     hdr, fx, fw, fi = _parse(p)
     assert np.array_equal(fi, idx)
     lx, lw, li, _ = aq.wush_load_transforms(p)
@@ -75,7 +78,8 @@ def test_special_values_survive(tmp_path):
     t = np.array([0.0, -0.0, np.inf, -np.inf, 1e-45, 3.4e38, np.nan, 1.0], np.float32).reshape(1, 2, 4)
     t = np.concatenate([t, t[:, :, ::-1]], axis=2).reshape(1, 4, 4)
     p = tmp_path / "v.wush"
-    aq.wush_save_transforms(p, t, -t, "identity")
+    aq.wush_save_transforms(p, t, -t, "identity", sigma_norm="unknown")
+    assert aq.wush_transforms_file_info(p)["sigma_norm"] == 0
     lx, lw, _, _ = aq.wush_load_transforms(p)
     assert lx.tobytes() == t.tobytes() and lw.tobytes() == (-t).tobytes()
 
@@ -111,14 +115,17 @@ def test_malformed_files_are_rejected(tmp_path, calibrated):
         "version": (raw[:8] + struct.pack("<I", 2) + raw[12:], INVALID),
         "block_not_pow2": (raw[:12] + struct.pack("<I", 24) + raw[16:], INVALID),
         "kind": (raw[:16] + struct.pack("<I", 9) + raw[20:], INVALID),
-        "n_t_zero": (raw[:24] + struct.pack("<q", 0) + raw[32:], INVALID),
-        "header_short": (raw[:30], IO),
+        "dtype": (raw[:20] + struct.pack("<I", 1) + raw[24:], INVALID),
+        "sigma_norm": (raw[:24] + struct.pack("<I", 2) + raw[28:], INVALID),
+        "has_index_2": (raw[:28] + struct.pack("<I", 2) + raw[32:], INVALID),
+        "n_t_zero": (raw[:32] + struct.pack("<q", 0) + raw[40:], INVALID),
+        "header_short": (raw[:47], IO),
         "body_short": (raw[:-5], INVALID),
         "extra_bytes": (raw + b"\0", INVALID),
         "index_out_of_range": (raw[:-4] + struct.pack("<i", 2), INVALID),
         "index_negative": (raw[:-4] + struct.pack("<i", -1), INVALID),
         # an index that does not cover the blocks: has_index = 0 but n_t != n_blocks
-        "no_index_count_mismatch": (raw[:20] + struct.pack("<I", 0) + raw[24:], INVALID),
+        "no_index_count_mismatch": (raw[:28] + struct.pack("<I", 0) + raw[32:], INVALID),
     }
     for name, (blob, want) in cases.items():
         p = tmp_path / f"{name}.wush"
@@ -141,6 +148,7 @@ def test_save_rejects_bad_arguments_before_writing(tmp_path, calibrated):
     assert _status(aq.wush_save_transforms, p, sx, sw, "wush", bad) == INVALID
     assert _status(aq.wush_save_transforms, p, sx[:, :3, :3], sw[:, :3, :3], "wush") == INVALID
     assert _status(aq.wush_save_transforms, p, tx, tw, 7) == INVALID
+    assert _status(aq.wush_save_transforms, p, tx, tw, "wush", None, 5) == INVALID
     assert not p.exists()
     assert _status(aq.wush_save_transforms, tmp_path / "no_dir" / "x.wush", tx, tw, "wush") == IO
     with pytest.raises(ValueError):
