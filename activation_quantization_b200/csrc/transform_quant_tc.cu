@@ -11,22 +11,28 @@
 //              columns, landing in a 5-stage shared-memory ring;
 //   warp 1     MMA issuer (WUS/WUSH): y = x T^T per b-block as kind::f16 MMAs,
 //              M = 128 rows, K = 16 per instruction.  T is split exactly into three
-//              bf16 parts (hi + mid + lo = the fp32 T).  Per K-step one MMA with
-//              N = 2b multiplies the X slice by [T_hi; T_mid] stacked along N and a
-//              second, N = b, adds x T_lo^T onto the T_hi columns, so X is read
-//              twice rather than three times and two partial products land side
-//              by side in TMEM.  Quarter q (32 columns) of every tile goes to one
-//              of two TMEM slots of warpgroup q, alternating by tile, so the MMAs
-//              of the next tile overlap the epilogue of this one;
+//              bf16 parts (hi + mid + lo = the fp32 T).  Quarter q (32 columns)
+//              of every tile goes to TMEM slot q of an accumulator set; the
+//              epilogue frees a set as soon as its TMEM loads are done, so the
+//              next tile's MMAs overlap this tile's quantisation.
+//                b = 16: per K-step one MMA, N = 3b, against [T_hi; T_mid; T_lo]
+//                stacked along N: three partial products side by side, one
+//                384-column set (8 MMAs per tile).
+//                b = 32: per K-step one MMA, N = 2b, against [T_hi; T_mid] and a
+//                second, N = b, adding x T_lo^T onto the T_hi columns: two partial
+//                products, two 256-column sets alternating by tile (16 MMAs per
+//                tile).  Measured side by side, each form is the faster one for
+//                its block size;
 //   warps 2-17 epilogue, four warpgroups, warpgroup q owning quarter q of every
 //              tile: one thread per row reads the partial products of its row out
-//              of TMEM (tcgen05.ld 32x32b) and adds them, y = (hi + lo) + mid --
+//              of TMEM (tcgen05.ld 32x32b) and adds them -- y = hi + (mid + lo),
+//              or (hi + lo) + mid for b = 32 --
 //              or, for identity and Hadamard, reads X out of the swizzled
 //              shared-memory tile -- and computes absmax, scale and codes in
 //              registers (hardware cvt.rn.satfinite e2m1x2 / e4m3x2), storing
 //              packed codes and scale bytes.  The same warps convert each new
-//              column's fp32 T into the stacked bf16 operand in shared memory,
-//              double-buffered.
+//              column's fp32 T into the stacked bf16 operand in shared memory
+//              (two column buffers).
 // Every mbarrier wait is bounded (see sm100.cuh).
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -51,19 +57,27 @@ constexpr int kStages = 5;
 constexpr int kEpiWarps = 16;
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kEpiGroups = kTileCols / kQuarterCols; // epilogue warpgroups, one quarter each
-constexpr int kSlotCols = 64;                        // TMEM columns of one quarter's partial products
-constexpr int kSets = 2;                             // accumulator sets (whole tiles), double-buffered
-constexpr int kSetCols = kEpiGroups * kSlotCols;     // 256
 constexpr int kThreads = 64 + kEpiThreads;
 constexpr int kStageBytes = kTileRows * kTileCols * 2;  // 32 KB
 constexpr int kBoxBytes = kTileRows * kBoxCols * 2;     // 16 KB
 constexpr int kTBufBytes = 24 * 1024;
-constexpr uint32_t kTmemCols = kSets * kSetCols;   // 512
+constexpr uint32_t kTmemCols = 512;                // allocation: the power of two >= kSets * kSetCols
 constexpr int64_t kDefaultPolls = int64_t(1) << 40;
 constexpr uint64_t kDeadlineNs = 4000000000ull;
 constexpr int kSmemBytes = kStages * kStageBytes + 2 * kTBufBytes + 1024 + 256;
 static_assert(kEpiGroups * 4 == kEpiWarps, "four warps per epilogue warpgroup");
 static_assert(kTmemCols == 512, "TMEM allocation is a power of two of at most 512 columns");
+
+// TMEM accumulator layout per block size (see the file comment).
+template <int B>
+struct AccLayout {
+  static constexpr bool kThree = B == 16;                   // one N = 3b MMA per K-step
+  static constexpr int kParts = kThree ? 3 : 2;             // partial products per block in TMEM
+  static constexpr int kSlotCols = (kQuarterCols / B) * kParts * B;  // one quarter: 96 or 64 columns
+  static constexpr int kSets = kThree ? 1 : 2;              // accumulator sets (whole tiles)
+  static constexpr int kSetCols = kEpiGroups * kSlotCols;   // 384 or 256
+  static_assert(kSets * kSetCols <= static_cast<int>(kTmemCols), "TMEM holds 512 columns");
+};
 
 enum Kind : int { kIdentity = 0, kHadamard = 1, kDense = 2 };
 // kAm: no quantisation; the kernel's only output is max |T x| over the tensor
@@ -229,10 +243,33 @@ __device__ __forceinline__ void tmem_tie(uint32_t (&r)[B]) {
   for (int i = 0; i < B; ++i) asm volatile("" : "+r"(r[i]));
 }
 
-// y = (hi + lo) + mid for one b-block of this thread's row: the MMAs leave
-// x (T_hi + T_lo)^T in TMEM columns taddr + [0, B) and x T_mid^T in [B, 2B).
+// y = hi + (mid + lo) for one b-block of this thread's row (b = 16): the MMA
+// leaves x T_hi^T, x T_mid^T and x T_lo^T in TMEM columns taddr + [0, B),
+// [B, 2B) and [2B, 3B).  The two small parts are added first.
 template <int B>
-__device__ __forceinline__ void tmem_sum_parts(uint32_t taddr, float (&y)[B]) {
+__device__ __forceinline__ void tmem_sum3(uint32_t taddr, float (&y)[B]) {
+  uint32_t h[B], m[B], l[B];
+  tmem_ld_cols<B>(taddr, h);
+  tmem_ld_cols<B>(taddr + B, m);
+  tmem_ld_cols<B>(taddr + 2 * B, l);
+  tmem_ld_wait();
+  tmem_tie<B>(h);
+  tmem_tie<B>(m);
+  tmem_tie<B>(l);
+#pragma unroll
+  for (int i = 0; i < B; i += 2) {
+    float s0 = __uint_as_float(m[i]), s1 = __uint_as_float(m[i + 1]);
+    add2(s0, s1, __uint_as_float(l[i]), __uint_as_float(l[i + 1]));
+    y[i] = __uint_as_float(h[i]);
+    y[i + 1] = __uint_as_float(h[i + 1]);
+    add2(y[i], y[i + 1], s0, s1);
+  }
+}
+
+// y = (hi + lo) + mid for one b-block of this thread's row (b = 32): the MMAs
+// leave x (T_hi + T_lo)^T in TMEM columns taddr + [0, B) and x T_mid^T in [B, 2B).
+template <int B>
+__device__ __forceinline__ void tmem_sum2(uint32_t taddr, float (&y)[B]) {
   uint32_t a[B], c[B];
   tmem_ld_cols<B>(taddr, a);
   tmem_ld_cols<B>(taddr + B, c);
@@ -274,7 +311,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int kBlocks = kTileCols / B;           // b-blocks per tile: 4 or 8
   constexpr int kQBlocks = kQuarterCols / B;       // b-blocks per quarter: 1 or 2
   constexpr int kKSteps = B / 16;                  // K = 16 per MMA
-  constexpr int kN = 2 * B;                        // MMA N: T_hi and T_mid stacked (T_lo adds onto T_hi)
+  using L = AccLayout<B>;
+  constexpr int kN = L::kParts * B;                // N of the stacked MMA: [T_hi; T_mid(; T_lo)]
+  constexpr int kSlotCols = L::kSlotCols, kSets = L::kSets, kSetCols = L::kSetCols;
   constexpr int kChunk = B * 32;                   // bytes of one [B n x 16 k] bf16 operand chunk
   constexpr bool kMma = KIND == kDense;
   static_assert(kQBlocks * kN <= kSlotCols, "a quarter's partial products must fit its TMEM slot");
@@ -298,8 +337,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // Every ring and slot below has consumers that each take its phases in order,
   // so the parity waits are unambiguous for any ring depth: the MMA warp (or all
-  // sixteen epilogue warps) for the X stages, all epilogue warps for the two TMEM
-  // accumulator sets (even and odd tiles).  Epilogue warps poll with lane 0 and
+  // sixteen epilogue warps) for the X stages, all epilogue warps for the TMEM
+  // accumulator set(s).  Epilogue warps poll with lane 0 and
   // release with one arrival per warp.
   const int n_mine = tile_hi - tile_lo;
   const int n_cols = n_mine > 0 ? (tile_hi - 1) / n_row_tiles - col_lo + 1 : 0;
@@ -379,22 +418,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (kMma && elect_one()) {
-      // Tile n goes to accumulator set n & 1; quarter q of it to columns
-      // 256 (n & 1) + 64 q.  Per b-block and K-step two MMAs read the same X slice:
-      // N = 2b against [T_hi; T_mid], then N = b against T_lo, accumulating onto
-      // the T_hi columns.  Descriptors are a per-tile base plus constant offsets.
-      constexpr uint32_t idesc2 = idesc_bf16_f32(kTileRows, kN);
-      constexpr uint32_t idesc1 = idesc_bf16_f32(kTileRows, B);
+      // Tile n goes to accumulator set n % kSets; quarter q of it to columns
+      // kSetCols (n % kSets) + kSlotCols q.  Per b-block and K-step one MMA against
+      // the stacked parts (N = 3b, or N = 2b plus one N = b MMA for T_lo onto the
+      // T_hi columns).  Descriptors are a per-tile base plus constant offsets.
+      constexpr uint32_t idesc_n = idesc_bf16_f32(kTileRows, kN);
+      constexpr uint32_t idesc_lo = idesc_bf16_f32(kTileRows, B);
       bool ok = true;
       int col = col_lo, row_tile = tile_lo % n_row_tiles, k_ready = -1;
       for (int n = 0; n < n_mine; ++n) {
-        const int s = n % kStages, p = n & 1, k = col - col_lo;
+        const int s = n % kStages, p = n % kSets, k = col - col_lo;
         if (k != k_ready) {
           if (!mbar_wait_bounded(&t_full[k & 1], (k >> 1) & 1, max_polls, kDeadlineNs, abort_flag)) { ok = false; break; }
           k_ready = k;
         }
         if (!mbar_wait_bounded(&x_full[s], (n / kStages) & 1, max_polls, kDeadlineNs, abort_flag) ||
-            !mbar_wait_bounded(&acc_empty[p], ((n >> 1) & 1) ^ 1, max_polls, kDeadlineNs, abort_flag)) {
+            !mbar_wait_bounded(&acc_empty[p], ((n / kSets) & 1) ^ 1, max_polls, kDeadlineNs, abort_flag)) {
           ok = false;
           break;
         }
@@ -411,8 +450,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < kKSteps; ++kk) {
             const uint64_t ad = a0 + ((a_off + kk * 32) >> 4);
             const uint32_t b_off = (jj * kKSteps + kk) * 3 * kChunk;
-            mma_bf16(d, ad, b0 + (b_off >> 4), idesc2, kk ? 1u : 0u);
-            mma_bf16(d, ad, b0 + ((b_off + 2 * kChunk) >> 4), idesc1, 1u);
+            mma_bf16(d, ad, b0 + (b_off >> 4), idesc_n, kk ? 1u : 0u);
+            if constexpr (!L::kThree) mma_bf16(d, ad, b0 + ((b_off + 2 * kChunk) >> 4), idesc_lo, 1u);
           }
         }
         tc_commit(&acc_full[p]);
@@ -424,7 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ---------------------------------------------------------------- epilogue
     // Four warpgroups of 4 warps; warpgroup g owns columns [32 g, 32 g + 32) of
-    // every tile (TMEM columns 64 g .. of the tile's accumulator set).  Warp w may read only TMEM lane quarter w % 4, i.e.
+    // every tile (TMEM columns kSlotCols g .. of the tile's accumulator set).  Warp w may read only TMEM lane quarter w % 4, i.e.
     // rows 32 (w % 4) .. + 31, and each thread handles one row of the quarter.
     const int et = threadIdx.x - 64;            // 0..511
     const int g = et / 128;                     // warpgroup = quarter
@@ -509,9 +548,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row0 = (i % n_row_tiles) * kTileRows, col0 = (i / n_row_tiles) * kTileCols;
       const int r = row0 + rloc;
       const bool row_ok = r < rows;
-      const int p = n & 1;
+      const int p = n % kSets;
       uint64_t* full = kMma ? &acc_full[p] : &x_full[s];
-      const uint32_t parity = kMma ? (n >> 1) & 1 : (n / kStages) & 1;
+      const uint32_t parity = kMma ? (n / kSets) & 1 : (n / kStages) & 1;
       // lane 0 polls; once it has seen the phase complete, every lane's own
       // try_wait succeeds at once and gives that lane its acquire
       bool ok = true;
@@ -528,7 +567,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + p * kSetCols + g * kSlotCols;
 #pragma unroll
-        for (int u = 0; u < kQBlocks; ++u) tmem_sum_parts<B>(taddr + u * kN, y[u]);
+        for (int u = 0; u < kQBlocks; ++u) {
+          if constexpr (L::kThree) tmem_sum3<B>(taddr + u * kN, y[u]);
+          else tmem_sum2<B>(taddr + u * kN, y[u]);
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[p]);
