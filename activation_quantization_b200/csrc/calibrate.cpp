@@ -29,6 +29,16 @@ constexpr double kCholJitter = 1e-8;
 
 bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
 
+// Moments, absolute maxima and scale exponents have no meaning for NaN or an
+// infinity, so calibration refuses such inputs before any work.
+template <typename T>
+bool all_finite(const T* p, int64_t n) {
+  bool ok = true;
+#pragma omp parallel for reduction(&& : ok) schedule(static)
+  for (int64_t i = 0; i < n; ++i) ok = ok && std::isfinite(p[i]);
+  return ok;
+}
+
 // Lower Cholesky factor of a (n x n, row-major) into l; false if not positive definite.
 bool cholesky(const double* a, double* l, int n) {
   std::memset(l, 0, sizeof(double) * n * n);
@@ -247,6 +257,8 @@ extern "C" int wush_calibrate_from_moments(const double* sigma_x, const double* 
   if (kind < WUSH_T_IDENTITY || kind > WUSH_T_WUSH_DIAG) return WUSH_ERR_UNSUPPORTED;
   if (kind >= WUSH_T_WUS && (!sigma_x || !sigma_w)) return WUSH_ERR_INVALID_ARG;
   const int64_t nb = d_in / block, bb = static_cast<int64_t>(block) * block;
+  if (kind >= WUSH_T_WUS && (!all_finite(sigma_x, nb * bb) || !all_finite(sigma_w, nb * bb)))
+    return WUSH_ERR_INVALID_ARG;
   int status = WUSH_OK;
 #pragma omp parallel for schedule(dynamic, 1)
   for (int64_t j = 0; j < nb; ++j) {
@@ -269,6 +281,7 @@ extern "C" int wush_calibrate(const float* x_calib, int64_t n_calib, const float
   if (kind == WUSH_T_IDENTITY || kind == WUSH_T_HADAMARD)
     return wush_calibrate_from_moments(nullptr, nullptr, d_in, block, kind, t_x, t_w);
   if (!x_calib || !w || n_calib <= 0 || d_out <= 0) return WUSH_ERR_INVALID_ARG;
+  if (!all_finite(x_calib, n_calib * d_in) || !all_finite(w, d_out * d_in)) return WUSH_ERR_INVALID_ARG;
   const size_t n = static_cast<size_t>(d_in / block) * block * block;
   std::vector<double> sx(n), sw(n);
   block_moments(x_calib, n_calib, d_in, block, sx.data());
@@ -293,6 +306,7 @@ extern "C" int wush_calibrate_shared_from_moments(const double* sigma_x, const d
   if (kind < WUSH_T_WUS || kind > WUSH_T_WUSH_DIAG) return WUSH_ERR_UNSUPPORTED;
   const int64_t nb = d_in / block, bb = static_cast<int64_t>(block) * block, nf = 2 * bb;
   if (groups < 1 || groups > nb) return WUSH_ERR_INVALID_ARG;
+  if (!all_finite(sigma_x, nb * bb) || !all_finite(sigma_w, nb * bb)) return WUSH_ERR_INVALID_ARG;
   std::vector<double> feat(static_cast<size_t>(nb * nf));
   for (int64_t j = 0; j < nb; ++j) {
     for (int m = 0; m < 2; ++m) {
@@ -372,6 +386,7 @@ extern "C" int wush_calibrate_shared(const float* x_calib, int64_t n_calib, cons
   if (!x_calib || !w || n_calib <= 0 || d_out <= 0 || !is_pow2(block) || block < 2 || block > 256 || d_in <= 0 ||
       d_in % block)
     return WUSH_ERR_INVALID_ARG;
+  if (!all_finite(x_calib, n_calib * d_in) || !all_finite(w, d_out * d_in)) return WUSH_ERR_INVALID_ARG;
   const size_t n = static_cast<size_t>(d_in / block) * block * block;
   std::vector<double> sx(n), sw(n);
   block_moments(x_calib, n_calib, d_in, block, sx.data());

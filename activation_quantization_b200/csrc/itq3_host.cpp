@@ -62,6 +62,11 @@ void fwht256(double* x) {
 extern "C" int itq3_quantize_weights(const uint16_t* w_fp16, int64_t d_out, int64_t d_in, uint8_t* codes,
                                      uint16_t* scales_fp16) {
   if (!w_fp16 || !codes || !scales_fp16 || d_out <= 0 || d_in <= 0 || d_in % 256) return WUSH_ERR_INVALID_ARG;
+  // an fp16 with all exponent bits set is an infinity or NaN: no scale exists for its block
+  bool finite = true;
+#pragma omp parallel for reduction(&& : finite) schedule(static)
+  for (int64_t i = 0; i < d_out * d_in; ++i) finite = finite && (w_fp16[i] & 0x7C00u) != 0x7C00u;
+  if (!finite) return WUSH_ERR_INVALID_ARG;
   const int64_t nb = d_in / 256;
   int status = WUSH_OK;
 #pragma omp parallel for schedule(static)

@@ -32,7 +32,9 @@
  *   - Device pointers must be 16-byte aligned.
  *   - ``stream`` is a cudaStream_t passed as void*; NULL is the legacy default
  *     stream.  Work is enqueued in stream order.
- *   - Inputs must be finite; non-finite values give unspecified codes.
+ *   - Inputs must be finite.  The host calls (calibration, ITQ3 weight
+ *     quantisation) check and return WUSH_ERR_INVALID_ARG for NaN or an
+ *     infinity; the device kernels do not check, and give unspecified codes.
  *   - Waits inside kernels are bounded. A kernel that gives up sets a device
  *     error word which wush_check_device_status() reports as WUSH_ERR_TIMEOUT.
  */

@@ -46,6 +46,7 @@ from __future__ import annotations
 
 import numpy as np
 
+from ._checks import require_finite
 from .transforms import normalized_hadamard
 
 KINDS = ("identity", "hadamard", "wus", "wush", "wush_diag")
@@ -60,6 +61,7 @@ def block_moments(x_rows: np.ndarray, b: int) -> np.ndarray:
 
     x_rows: [rows, d_in] -- calibration tokens of X, or the d_out rows of W^T.
     """
+    require_finite("block_moments", x_rows)
     x = np.asarray(x_rows, dtype=np.float64)
     rows, d_in = x.shape
     xb = x.reshape(rows, d_in // b, b)
@@ -123,6 +125,7 @@ def block_transform_pair(sigma_x: np.ndarray, sigma_w: np.ndarray, kind: str):
 
 def transforms_from_moments(sigma_x: np.ndarray, sigma_w: np.ndarray, kind: str):
     """(T_X, T_W) as [d_in/b, b, b] fp64 from per-block moments [d_in/b, b, b]."""
+    require_finite("transforms_from_moments", sigma_x, sigma_w)
     pairs = [block_transform_pair(sx, sw, kind) for sx, sw in zip(sigma_x, sigma_w)]
     return np.stack([p[0] for p in pairs]), np.stack([p[1] for p in pairs])
 
@@ -141,6 +144,7 @@ def nvfp4_global_scale(y_rows: np.ndarray) -> np.float32:
     from the transformed calibration tokens (static), for weights from the
     transformed weight tensor itself.
     """
+    require_finite("nvfp4_global_scale", y_rows)
     amax = float(np.max(np.abs(np.asarray(y_rows, dtype=np.float64))))
     return np.float32(amax / (6.0 * 448.0))
 
@@ -154,6 +158,7 @@ def nvfp4_dynamic_global_scale(y_rows: np.ndarray) -> np.float32:
     the per-batch variant of the same rule.  amax is the exact maximum of the
     fp32 values and the quotient is rounded once to fp32.
     """
+    require_finite("nvfp4_dynamic_global_scale", y_rows)
     amax = np.float32(np.max(np.abs(np.asarray(y_rows, dtype=np.float32)))) if np.size(y_rows) else np.float32(0)
     g = np.float32(np.float64(amax) / 2688.0)
     return g if g >= np.float32(1e-30) else np.float32(1.0)
@@ -170,6 +175,7 @@ def group_blocks(sigma_x: np.ndarray, sigma_w: np.ndarray, groups: int, iters: i
     ties to the lowest group, empty groups keeping their centre, until no block
     changes group (at most ``iters`` rounds).
     """
+    require_finite("group_blocks", sigma_x, sigma_w)
     nb = sigma_x.shape[0]
     if not 1 <= groups <= nb:
         raise ValueError(groups)
@@ -197,6 +203,7 @@ def group_blocks(sigma_x: np.ndarray, sigma_w: np.ndarray, groups: int, iters: i
 def shared_transforms(sigma_x: np.ndarray, sigma_w: np.ndarray, kind: str, groups: int):
     """(T_X [groups, b, b], T_W [groups, b, b], index [nb]) with one transform per
     group of similar blocks, computed from the group's mean moments."""
+    require_finite("shared_transforms", sigma_x, sigma_w)
     index = group_blocks(sigma_x, sigma_w, groups)
     nb = sigma_x.shape[0]
     start = [int(round(g * nb / groups)) for g in range(groups)]

@@ -12,8 +12,11 @@ from __future__ import annotations
 
 import numpy as np
 
+from ._checks import require_finite
+
 
 def gemm_dequantized(a_dq: np.ndarray, b_dq: np.ndarray, alpha: float = 1.0) -> np.ndarray:
+    require_finite("gemm_dequantized", a_dq, b_dq, alpha)
     a = np.asarray(a_dq, dtype=np.float64)
     b = np.asarray(b_dq, dtype=np.float64)
     if a.shape[1] != b.shape[1]:

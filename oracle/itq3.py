@@ -19,12 +19,14 @@ from __future__ import annotations
 
 import numpy as np
 
+from ._checks import require_finite
 from .transforms import fwht
 
 BLOCK = 256
 
 
 def rotate(w_rows: np.ndarray) -> np.ndarray:
+    require_finite("rotate", w_rows)
     w = np.asarray(w_rows, dtype=np.float64)
     d_out, d_in = w.shape
     if d_in % BLOCK:
@@ -62,4 +64,5 @@ def dequantize(codes: np.ndarray, scales16: np.ndarray) -> np.ndarray:
 
 def gemv(codes: np.ndarray, scales16: np.ndarray, x_rows: np.ndarray) -> np.ndarray:
     """y[t, o] = sum_k w_hat[o, k] x[t, k], fp64; x_rows [tokens, d_in]."""
+    require_finite("gemv", scales16, x_rows)
     return np.asarray(x_rows, dtype=np.float64) @ dequantize(codes, scales16).T

@@ -9,11 +9,13 @@ from __future__ import annotations
 
 import numpy as np
 
+from ._checks import require_finite
 from .calibrate import nvfp4_global_scale
 from .quant import transform_quantize
 
 
 def output_loss(y_quant: np.ndarray, y_ref: np.ndarray) -> float:
+    require_finite("output_loss", y_quant, y_ref)
     d = np.asarray(y_quant, dtype=np.float64) - np.asarray(y_ref, dtype=np.float64)
     return float(np.sum(d * d) / d.size)
 
@@ -21,6 +23,7 @@ def output_loss(y_quant: np.ndarray, y_ref: np.ndarray) -> float:
 def layer_loss(x_rows, w_rows, t_x, t_w, fmt: str, x_global_scale=None) -> float:
     """Loss of one quantised linear layer on activations x_rows [tokens, d_in]
     and weights w_rows [d_out, d_in], with transforms t_x, t_w [d_in/b, b, b]."""
+    require_finite("layer_loss", x_rows, w_rows, t_x, t_w)
     w_global = None
     if fmt == "nvfp4":
         from .transforms import apply_block_transform

@@ -35,6 +35,7 @@ from __future__ import annotations
 
 import numpy as np
 
+from ._checks import require_finite
 from .formats import (E2M1_BOUNDARIES, E4M3_MIDPOINTS, INT4_MIDPOINTS, distance_to_boundary,
                       e2m1_code, e2m1_value, e4m3_code_unsigned, e4m3_value, fp16_rne_sat)
 
@@ -52,6 +53,7 @@ def _blocks(y32: np.ndarray, b: int) -> np.ndarray:
 
 
 def quantize_mxfp4(y32: np.ndarray) -> dict:
+    require_finite("quantize_mxfp4", y32)
     yb = _blocks(y32, 32).astype(np.float64)
     amax = np.max(np.abs(yb), axis=2)
     _, p = np.frexp(amax)                       # amax = f * 2^p, f in [0.5, 1)
@@ -73,6 +75,7 @@ def quantize_mxfp4(y32: np.ndarray) -> dict:
 
 
 def quantize_nvfp4(y32: np.ndarray, s_g) -> dict:
+    require_finite("quantize_nvfp4", y32, s_g)
     yb = _blocks(y32, 16)
     s_g = F32(s_g)
     amax = np.max(np.abs(yb), axis=2).astype(F32)
@@ -108,6 +111,7 @@ def _fp16_midpoint_distance(v: np.ndarray) -> np.ndarray:
 
 
 def quantize_int4(y32: np.ndarray) -> dict:
+    require_finite("quantize_int4", y32)
     yb = _blocks(y32, 32)
     amax = np.max(np.abs(yb), axis=2).astype(F32)
     pre = (amax / F32(7.0)).astype(F32)

@@ -11,6 +11,8 @@ from __future__ import annotations
 
 import numpy as np
 
+from ._checks import require_finite
+
 
 def sylvester_hadamard(n: int) -> np.ndarray:
     """The n x n Sylvester Hadamard matrix (entries +-1, H H^T = n I); n a power of 2.
@@ -36,6 +38,7 @@ def fwht(x: np.ndarray) -> np.ndarray:
     log2(n) butterfly stages (a, b) -> (a + b, a - b) with stride 1, 2, 4, ...;
     the result equals sylvester_hadamard(n) @ x for each vector.
     """
+    require_finite("fwht", x)
     y = np.array(x, dtype=np.float64, copy=True)
     n = y.shape[-1]
     if n & (n - 1):
@@ -59,6 +62,7 @@ def apply_block_transform(x_rows: np.ndarray, t: np.ndarray) -> np.ndarray:
     t: [d_in / b, b, b]; block j of a row, x_j = row[j*b:(j+1)*b], becomes
     y_j = t[j] @ x_j.  Returns [rows, d_in] fp64.
     """
+    require_finite("apply_block_transform", x_rows, t)
     x = np.asarray(x_rows, dtype=np.float64)
     nb, b, _ = t.shape
     rows = x.shape[0]
@@ -70,6 +74,7 @@ def apply_block_transform(x_rows: np.ndarray, t: np.ndarray) -> np.ndarray:
 def block_magnitude(x_rows: np.ndarray, t: np.ndarray) -> np.ndarray:
     """sum_k |t[j][i][k] * x_j[k]| for every output element (the size of the terms
     summed to form it); the parity tests measure rounding error against this."""
+    require_finite("block_magnitude", x_rows, t)
     return apply_block_transform(np.abs(x_rows), np.abs(t))
 
 

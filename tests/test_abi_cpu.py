@@ -115,3 +115,33 @@ def test_calibrate_shared_matches_oracle(kind):
         aq.wush_calibrate_shared(xc, wt, 32, kind, 0)
     with pytest.raises(aq.WushError):
         aq.wush_calibrate_shared(xc, wt, 32, kind, 9)      # more groups than blocks
+
+
+@pytest.mark.parametrize("bad", [np.nan, np.inf, -np.inf])
+def test_host_calls_reject_non_finite_inputs(bad):
+    # one planted NaN or infinity anywhere in an input gives WUSH_ERR_INVALID_ARG
+    w = synth.WORKLOADS["tiny"]
+    xc, wt = synth.activations(w, calib=True), synth.weights(w)
+
+    def planted(a):
+        a = np.array(a, copy=True)
+        a.flat[a.size // 3] = bad
+        return a
+
+    def status(fn, *args):
+        with pytest.raises(aq.WushError) as e:
+            fn(*args)
+        return e.value.status
+
+    for kind in ("wus", "wush", "wush_diag"):
+        assert status(aq.wush_calibrate, planted(xc), wt, 32, kind) == -1
+        assert status(aq.wush_calibrate, xc, planted(wt), 32, kind) == -1
+        assert status(aq.wush_calibrate_shared, planted(xc), wt, 32, kind, 2) == -1
+        sx, sw = C.block_moments(xc, 32), C.block_moments(wt, 32)
+        assert status(aq.wush_calibrate_from_moments, planted(sx), sw, kind) == -1
+        assert status(aq.wush_calibrate_shared_from_moments, sx, planted(sw), kind, 2) == -1
+    # identity and Hadamard read no data, so there is nothing to check
+    aq.wush_calibrate(planted(xc), wt, 32, "hadamard")
+    w3 = synth.itq3_weights(4, 512).astype(np.float16)
+    assert status(aq.itq3_quantize_weights, planted(w3)) == -1
+    aq.itq3_quantize_weights(w3)                      # the clean copy is accepted
