@@ -68,10 +68,14 @@ for _name, (_res, _args) in _SIGNATURES.items():
     EXPORTED.append(_name)
 
 
+WUSH_ERR_BUFFER_TOO_SMALL = -6
+
+
 class WushError(RuntimeError):
-    def __init__(self, fn: str, status: int):
+    def __init__(self, fn: str, status: int, detail: str | None = None):
         self.status = status
-        super().__init__(f"{fn}: {_lib.wush_status_string(status).decode()} ({status})")
+        msg = f"{fn}: {_lib.wush_status_string(status).decode()} ({status})"
+        super().__init__(msg + (f": {detail}" if detail else ""))
 
 
 def _check(fn: str, status: int):
@@ -92,6 +96,32 @@ def _ptr(t):
     if not t.is_contiguous():
         raise ValueError("expected a contiguous tensor")
     return t.data_ptr()
+
+
+def _need(fn: str, name: str, t, nbytes: int, dtypes=None):
+    """The C calls take bare pointers, so the binding checks what it can see: the
+    element type (ValueError) and that ``t`` holds at least ``nbytes`` bytes
+    (WushError with WUSH_ERR_BUFFER_TOO_SMALL).  None passes through to the
+    library's own checks."""
+    if t is None:
+        return
+    if dtypes is not None and t.dtype not in dtypes:
+        raise ValueError(f"{fn}: {name} must be {' or '.join(str(d) for d in dtypes)}, got {t.dtype}")
+    have = t.numel() * t.element_size()
+    if have < nbytes:
+        raise WushError(fn, WUSH_ERR_BUFFER_TOO_SMALL, f"{name} holds {have} bytes, needs {nbytes}")
+
+
+def _quant_outputs_ok(fn, rows, d_in, fmt, kind, t, codes, scales, y_debug, n_t=None):
+    import torch
+    f = _enum(FORMATS, fmt)
+    b = _lib.wush_block_size(f)
+    if b > 0 and _enum(TRANSFORMS, kind) >= TRANSFORMS["wus"]:
+        count = n_t if n_t is not None else d_in // b
+        _need(fn, "t", t, count * b * b * 4, (torch.float32,))
+    _need(fn, "codes", codes, wush_codes_bytes(rows, d_in, f))
+    _need(fn, "scales", scales, wush_scales_bytes(rows, d_in, f))
+    _need(fn, "y_debug", y_debug, rows * d_in * 4, (torch.float32,))
 
 
 def _stream(stream):
@@ -250,6 +280,7 @@ def wush_transform_quant(x, t, kind, fmt, codes, scales, global_scale: float = 0
     if x.dtype not in (torch.float32, torch.bfloat16):
         raise ValueError("x must be bf16 or fp32")
     rows, d_in = x.shape
+    _quant_outputs_ok("wush_transform_quant", rows, d_in, fmt, kind, t, codes, scales, y_debug)
     _check("wush_transform_quant",
            _lib.wush_transform_quant(_ptr(x), x_dtype, rows, d_in, _ptr(t), _enum(TRANSFORMS, kind),
                                      _enum(FORMATS, fmt), float(global_scale), _ptr(codes), _ptr(scales),
@@ -264,6 +295,10 @@ def wush_transform_quant_indexed(x, t, t_index, kind, fmt, codes, scales, global
     if x.dtype not in (torch.float32, torch.bfloat16):
         raise ValueError("x must be bf16 or fp32")
     rows, d_in = x.shape
+    b = _lib.wush_block_size(_enum(FORMATS, fmt))
+    _quant_outputs_ok("wush_transform_quant_indexed", rows, d_in, fmt, kind, t, codes, scales, y_debug,
+                      n_t=int(t.shape[0]))
+    _need("wush_transform_quant_indexed", "t_index", t_index, max(d_in // max(b, 1), 0) * 4, (torch.int32,))
     _check("wush_transform_quant_indexed",
            _lib.wush_transform_quant_indexed(_ptr(x), x_dtype, rows, d_in, _ptr(t), _ptr(t_index), int(t.shape[0]),
                                              _enum(TRANSFORMS, kind), _enum(FORMATS, fmt), float(global_scale),
@@ -274,6 +309,9 @@ def wush_transform_amax(x, t, kind, block: int, amax_out, stream=None):
     import torch
     x_dtype = IN_FP32 if x.dtype == torch.float32 else IN_BF16
     rows, d_in = x.shape
+    if _enum(TRANSFORMS, kind) >= TRANSFORMS["wus"] and block > 0:
+        _need("wush_transform_amax", "t", t, (d_in // block) * block * block * 4, (torch.float32,))
+    _need("wush_transform_amax", "amax_out", amax_out, 4, (torch.float32,))
     _check("wush_transform_amax",
            _lib.wush_transform_amax(_ptr(x), x_dtype, rows, d_in, _ptr(t), _enum(TRANSFORMS, kind), block,
                                     _ptr(amax_out), _stream(stream)))
@@ -289,6 +327,10 @@ def wush_transform_quant_nvfp4_dynamic(x, t, kind, amax, codes, scales, global_s
     if x.dtype not in (torch.float32, torch.bfloat16):
         raise ValueError("x must be bf16 or fp32")
     rows, d_in = x.shape
+    fn = "wush_transform_quant_nvfp4_dynamic"
+    _quant_outputs_ok(fn, rows, d_in, "nvfp4", kind, t, codes, scales, y_debug)
+    _need(fn, "amax", amax, 4, (torch.float32,))
+    _need(fn, "global_scale_out", global_scale_out, 4, (torch.float32,))
     _check("wush_transform_quant_nvfp4_dynamic",
            _lib.wush_transform_quant_nvfp4_dynamic(_ptr(x), x_dtype, rows, d_in, _ptr(t), _enum(TRANSFORMS, kind),
                                                    _ptr(amax), _ptr(global_scale_out), _ptr(codes), _ptr(scales),
@@ -298,19 +340,36 @@ def wush_transform_quant_nvfp4_dynamic(x, t, kind, amax, codes, scales, global_s
 def wush_qgemm_nvfp4_dynamic(a_codes, a_scales, b_codes, b_scales, M: int, N: int, K: int, a_global_scale,
                              b_global_scale: float, y, stream=None):
     """NVFP4 GEMM with alpha = *a_global_scale (CUDA fp32 scalar) * b_global_scale, formed on the device."""
+    import torch
+    _gemm_operands_ok("wush_qgemm_nvfp4_dynamic", a_codes, a_scales, b_codes, b_scales, M, N, K, "nvfp4", y)
+    _need("wush_qgemm_nvfp4_dynamic", "a_global_scale", a_global_scale, 4, (torch.float32,))
     _check("wush_qgemm_nvfp4_dynamic",
            _lib.wush_qgemm_nvfp4_dynamic(_ptr(a_codes), _ptr(a_scales), _ptr(b_codes), _ptr(b_scales), M, N, K,
                                          _ptr(a_global_scale), float(b_global_scale), _ptr(y), _stream(stream)))
 
 
+def _gemm_operands_ok(fn, a_codes, a_scales, b_codes, b_scales, M, N, K, fmt, y):
+    import torch
+    if M <= 0 or N <= 0 or K <= 0:
+        return                                      # the library rejects the shape
+    f = _enum(FORMATS, fmt)
+    _need(fn, "a_codes", a_codes, M * K // 2)
+    _need(fn, "b_codes", b_codes, N * K // 2)
+    _need(fn, "a_scales", a_scales, wush_scales_bytes(M, K, f))
+    _need(fn, "b_scales", b_scales, wush_scales_bytes(N, K, f))
+    _need(fn, "y", y, M * N * 4, (torch.float32,))
+
+
 def wush_qgemm(a_codes, a_scales, b_codes, b_scales, M: int, N: int, K: int, fmt, alpha: float, y,
                stream=None):
+    _gemm_operands_ok("wush_qgemm", a_codes, a_scales, b_codes, b_scales, M, N, K, fmt, y)
     _check("wush_qgemm",
            _lib.wush_qgemm(_ptr(a_codes), _ptr(a_scales), _ptr(b_codes), _ptr(b_scales), M, N, K,
                            _enum(FORMATS, fmt), float(alpha), _ptr(y), _stream(stream)))
 
 
 def wush_qgemm_int4(a_codes, a_scales, b_codes, b_scales, M: int, N: int, K: int, y, stream=None):
+    _gemm_operands_ok("wush_qgemm_int4", a_codes, a_scales, b_codes, b_scales, M, N, K, "int4", y)
     _check("wush_qgemm_int4",
            _lib.wush_qgemm_int4(_ptr(a_codes), _ptr(a_scales), _ptr(b_codes), _ptr(b_scales), M, N, K, _ptr(y),
                                 _stream(stream)))
@@ -322,13 +381,27 @@ def wush_qgemm_int4_workspace_bytes(M: int, N: int, K: int) -> int:
 
 def wush_qgemm_int4_ws(a_codes, a_scales, b_codes, b_scales, M: int, N: int, K: int, workspace, y, stream=None):
     """workspace: CUDA tensor of at least wush_qgemm_int4_workspace_bytes(M, N, K) bytes."""
+    _gemm_operands_ok("wush_qgemm_int4_ws", a_codes, a_scales, b_codes, b_scales, M, N, K, "int4", y)
     nbytes = workspace.numel() * workspace.element_size()
     _check("wush_qgemm_int4_ws",
            _lib.wush_qgemm_int4_ws(_ptr(a_codes), _ptr(a_scales), _ptr(b_codes), _ptr(b_scales), M, N, K,
                                    _ptr(workspace), nbytes, _ptr(y), _stream(stream)))
 
+def _itq3_operands_ok(fn, codes, scales, x, d_out, y, workspace=None):
+    import torch
+    tokens, d_in = x.shape
+    _need(fn, "x", x, 0, (torch.float16,))
+    if d_out <= 0 or d_in <= 0:
+        return                                      # the library rejects the shape
+    _need(fn, "codes", codes, d_out * d_in * 3 // 8)
+    _need(fn, "scales", scales, d_out * (d_in // 256) * 2)
+    _need(fn, "y", y, tokens * d_out * 4, (torch.float32,))
+    _need(fn, "workspace", workspace, tokens * d_in * 4, (torch.float32,))
+
+
 def itq3_dequant_gemv(codes, scales, x, d_out: int, mode: int, y, workspace=None, stream=None):
     tokens, d_in = x.shape
+    _itq3_operands_ok("itq3_dequant_gemv", codes, scales, x, d_out, y, workspace if int(mode) == 1 else None)
     _check("itq3_dequant_gemv",
            _lib.itq3_dequant_gemv(_ptr(codes), _ptr(scales), _ptr(x), tokens, d_out, d_in, int(mode),
                                   _ptr(workspace), _ptr(y), _stream(stream)))
@@ -337,6 +410,7 @@ def itq3_dequant_gemv(codes, scales, x, d_out: int, mode: int, y, workspace=None
 def itq3_dequant_gemv_noalloc(codes, scales, x, d_out: int, y, stream=None):
     """Mode-1 ITQ3 GEMV with the library's fixed scratch instead of a workspace."""
     tokens, d_in = x.shape
+    _itq3_operands_ok("itq3_dequant_gemv_noalloc", codes, scales, x, d_out, y)
     _check("itq3_dequant_gemv_noalloc",
            _lib.itq3_dequant_gemv_noalloc(_ptr(codes), _ptr(scales), _ptr(x), tokens, d_out, d_in, _ptr(y),
                                           _stream(stream)))
