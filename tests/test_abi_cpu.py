@@ -145,3 +145,21 @@ def test_host_calls_reject_non_finite_inputs(bad):
     w3 = synth.itq3_weights(4, 512).astype(np.float16)
     assert status(aq.itq3_quantize_weights, planted(w3)) == -1
     aq.itq3_quantize_weights(w3)                      # the clean copy is accepted
+
+
+@pytest.mark.parametrize("b", [2, 4, 8, 64, 128, 256])
+@pytest.mark.parametrize("kind", ["hadamard", "wus", "wush", "wush_diag"])
+def test_calibrate_every_block_size_matches_oracle(kind, b):
+    # the host calibration accepts any power-of-two block up to 256; the device
+    # kernels use 16 and 32, checked above, and here the rest of the range
+    w = synth.WORKLOADS["tiny"]
+    xc, wt = synth.activations(w, calib=True), synth.weights(w)
+    tx, tw = aq.wush_calibrate(xc, wt, b, kind)
+    ox, ow = C.calibrate(xc, wt, b, kind)
+    for got, want in ((tx, ox), (tw, ow)):
+        scale = np.abs(want).max(axis=(1, 2), keepdims=True)
+        assert np.max(np.abs(got - want) / scale) < 1e-6
+    if kind != "hadamard":
+        # the defining property T_W^T T_X = I, in fp32 storage
+        eye = np.einsum("jki,jkl->jil", tw.astype(np.float64), tx.astype(np.float64))
+        assert np.max(np.abs(eye - np.eye(b))) < 1e-4
