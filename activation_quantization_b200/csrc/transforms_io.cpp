@@ -46,6 +46,9 @@ bool valid_shape(int block, int kind, int sigma_norm, int64_t n_t, int64_t n_blo
   return has_index || n_t == n_blocks;
 }
 
+// Reads and checks the header, then checks that the file is exactly as long as the
+// header says (so that a caller can size its buffers from the header safely), and
+// leaves f positioned at the start of the body.
 int read_header(FILE* f, Header* h) {
   if (std::fread(h, sizeof(Header), 1, f) != 1) return WUSH_ERR_IO;
   if (std::memcmp(h->magic, kMagic, 8) != 0 || h->version != kVersion || h->dtype != kDtypeF32)
@@ -53,7 +56,13 @@ int read_header(FILE* f, Header* h) {
   if (h->has_index > 1 || !valid_shape(static_cast<int>(h->block), static_cast<int>(h->kind),
                                        static_cast<int>(h->sigma_norm), h->n_t, h->n_blocks, h->has_index != 0))
     return WUSH_ERR_INVALID_ARG;
-  return WUSH_OK;
+  // at most 48 + 8 * 2^32 * 2^16 + 4 * 2^32 bytes: no overflow in 64 bits
+  const int64_t want = static_cast<int64_t>(sizeof(Header)) + 8 * h->n_t * h->block * h->block +
+                       (h->has_index ? 4 * h->n_blocks : 0);
+  if (std::fseek(f, 0, SEEK_END) != 0) return WUSH_ERR_IO;
+  const long have = std::ftell(f);
+  if (have < 0 || std::fseek(f, static_cast<long>(sizeof(Header)), SEEK_SET) != 0) return WUSH_ERR_IO;
+  return static_cast<int64_t>(have) == want ? WUSH_OK : WUSH_ERR_INVALID_ARG;
 }
 
 }  // namespace

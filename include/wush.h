@@ -155,7 +155,10 @@ int wush_calibrate_shared_from_moments(const double* sigma_x, const double* sigm
  * WUSH_ERR_IO when the file cannot be opened or fully written (a partial file
  * may remain).
  *
- * wush_transforms_file_info: reads the header only and returns its fields.
+ * wush_transforms_file_info: reads the header and returns its fields, after
+ * checking it as wush_load_transforms does, the file's length included (a file
+ * longer or shorter than its header implies gives WUSH_ERR_INVALID_ARG), so that
+ * buffers may be sized from what it returns.
  *
  * wush_load_transforms: reads the whole file into t_x and t_w (capacity_floats
  * floats each, at least n_t * b * b) and, when the file holds an index, into

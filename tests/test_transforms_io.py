@@ -153,3 +153,18 @@ def test_save_rejects_bad_arguments_before_writing(tmp_path, calibrated):
     assert _status(aq.wush_save_transforms, tmp_path / "no_dir" / "x.wush", tx, tw, "wush") == IO
     with pytest.raises(ValueError):
         aq.wush_save_transforms(p, tx, tw[:1], "wush")
+
+
+def test_header_that_overstates_the_body_is_rejected_before_allocation(tmp_path, calibrated):
+    # a header claiming 2^31 transforms over a short body: info refuses it, so the
+    # binding never sizes a buffer from it
+    (tx, tw), _ = calibrated
+    good = tmp_path / "g.wush"
+    aq.wush_save_transforms(good, tx, tw, "wush")
+    raw = good.read_bytes()
+    p = tmp_path / "huge.wush"
+    _write(p, raw[:32] + struct.pack("<qq", 1 << 31, 1 << 31) + raw[48:])
+    assert _status(aq.wush_transforms_file_info, p) == INVALID
+    assert _status(aq.wush_load_transforms, p) == INVALID
+    _write(p, raw + b"\0\0\0\0")
+    assert _status(aq.wush_transforms_file_info, p) == INVALID
