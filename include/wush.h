@@ -130,6 +130,10 @@ int wush_calibrate_shared_from_moments(const double* sigma_x, const double* sigm
                                        int block, int kind, int groups, float* t_x, float* t_w,
                                        int32_t* index);
 
+/* How the second moments behind a set of transforms were normalised (recorded in
+ * the transforms file; see below). */
+typedef enum { WUSH_NORM_UNKNOWN = 0, WUSH_NORM_MEAN = 1 } wush_sigma_norm;
+
 /* ---------------------------------------------------------------------------
  * Checkpointing calibrated transforms (host, no CUDA)
  *
@@ -169,8 +173,6 @@ int wush_calibrate_shared_from_moments(const double* sigma_x, const double* sigm
  * extra bytes, or an index entry out of range (the buffers may then hold part
  * of the file).
  * ------------------------------------------------------------------------- */
-typedef enum { WUSH_NORM_UNKNOWN = 0, WUSH_NORM_MEAN = 1 } wush_sigma_norm;
-
 int wush_save_transforms(const char* path, int block, int kind, int sigma_norm, int64_t n_t,
                          const float* t_x, const float* t_w, const int32_t* index, int64_t n_blocks);
 int wush_transforms_file_info(const char* path, int* block, int* kind, int* sigma_norm,
