@@ -88,6 +88,61 @@ def test_ragged_rows_bf16(lib, fmt, kind):
     P.compare_transform_quant(x, t, fmt, gs, c, s, y)
 
 
+def _run_raw(lib, x, t, kind, fmt, gs):
+    """bf16 x through wush_transform_quant: (codes, raw scale buffer, y) on the host;
+    the scale buffer is poisoned first, so every byte left in it was written."""
+    rows, d_in = x.shape
+    xt = _as_input(x, True).cuda()
+    tt = None if kind in ("identity", "hadamard") else torch.from_numpy(np.ascontiguousarray(t)).cuda()
+    codes, scales = lib.alloc_quant_outputs(rows, d_in, fmt)
+    scales.fill_(0x5A)
+    y = torch.empty((rows, d_in), dtype=torch.float32, device="cuda")
+    lib.wush_transform_quant(xt, tt, kind, fmt, codes, scales, gs, y)
+    torch.cuda.synchronize()
+    assert lib.wush_check_device_status() == 0
+    return P.unpack_nibbles(codes.cpu().numpy(), rows, d_in), scales.cpu().numpy(), y.cpu().numpy()
+
+
+@pytest.mark.parametrize("fmt, d_in", [("mxfp4", 160), ("nvfp4", 176), ("nvfp4", 48), ("int4", 224)])
+@pytest.mark.parametrize("kind", ["identity", "hadamard", "wush"])
+def test_ragged_columns_bf16(lib, fmt, d_in, kind):
+    # d_in not a multiple of the 128-column tile (d_in = 48 is even narrower than
+    # one TMA box): the tensor-core kernel's last tile column reaches past the end of
+    # X, which the TMA fills with zeros.  Blocks are independent, so every real block
+    # must come out bit for bit as in the same rows zero-padded to whole tiles (a
+    # path the other tests check against the oracle); blocks beyond d_in must write
+    # no codes, and the scale atoms' padding must be written as zero.  Identity and
+    # Hadamard, exact on both sides, are also checked against the oracle directly.
+    w = synth.WORKLOADS[FMT_WORKLOAD[fmt]]
+    b = P.Q.BLOCK[fmt]
+    x = np.ascontiguousarray(synth.activations(w, tokens=200)[:, :d_in])
+    rows, nb = x.shape[0], d_in // b
+    d_pad = (d_in + 127) // 128 * 128
+    if kind == "identity":
+        t, t_pad = T.identity_blocks(d_in, b), T.identity_blocks(d_pad, b)
+    elif kind == "hadamard":
+        t, t_pad = T.hadamard_blocks(d_in, b), T.hadamard_blocks(d_pad, b)
+    else:
+        xc, wt = _calib_inputs(w.name, 1024)
+        t = C.calibrate(xc[:, :d_in], wt[:, :d_in], b, kind)[0]
+        t_pad = np.concatenate([t, T.identity_blocks(d_pad - d_in, b)])
+    t, t_pad = t.astype(np.float32), t_pad.astype(np.float32)
+    gs = _global_scale(x, t, fmt)
+    c, raw, y = _run_raw(lib, x, t, kind, fmt, gs)
+    x_pad = np.zeros((rows, d_pad), np.float32)
+    x_pad[:, :d_in] = x
+    c_pad, raw_pad, y_pad = _run_raw(lib, x_pad, t_pad, kind, fmt, gs)
+    assert np.array_equal(c, c_pad[:, :d_in])
+    assert np.array_equal(P.decode_scales(raw, rows, d_in, fmt), P.decode_scales(raw_pad, rows, d_pad, fmt)[:, :nb])
+    assert np.array_equal(y, y_pad[:, :d_in])
+    if fmt != "int4":
+        full = P.unswizzle_scales(raw, (rows + 127) // 128 * 128, (nb + 3) // 4 * 4)
+        assert not full[rows:, :].any() and not full[:, nb:].any()
+    if kind != "wush":
+        P.compare_transform_quant(x, t, fmt, gs if fmt == "nvfp4" else None, c,
+                                  P.decode_scales(raw, rows, d_in, fmt), y)
+
+
 @pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4", "int4"])
 def test_partial_scale_atom_and_special_values(lib, fmt):
     # d_in = 3 blocks (a partial 4-column scale atom), 5 rows; zero blocks, tiny and
