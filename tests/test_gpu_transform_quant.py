@@ -201,6 +201,29 @@ def test_amax_matches_oracle(lib, kind, fmt):
         assert abs(float(out.item()) - want) <= 1e-5 * want, (bf16, float(out.item()), want)
 
 
+@pytest.mark.parametrize("fmt, d_in", [("nvfp4", 176), ("mxfp4", 160), ("nvfp4", 48)])
+@pytest.mark.parametrize("kind", ["hadamard", "wush"])
+def test_amax_ragged_columns(lib, fmt, d_in, kind):
+    # the amax mode over a last tile column that reaches past the end of X (TMA zero
+    # fill), for both kernels
+    w = synth.WORKLOADS[FMT_WORKLOAD[fmt]]
+    b = P.Q.BLOCK[fmt]
+    x = np.ascontiguousarray(synth.activations(w, tokens=200)[:, :d_in])
+    if kind == "hadamard":
+        t = T.hadamard_blocks(d_in, b).astype(np.float32)
+    else:
+        xc, wt = _calib_inputs(w.name, 1024)
+        t = C.calibrate(xc[:, :d_in], wt[:, :d_in], b, kind)[0].astype(np.float32)
+    tt = None if kind == "hadamard" else torch.from_numpy(t).cuda()
+    want = np.max(np.abs(T.apply_block_transform(x, t)))
+    for bf16 in (True, False):
+        out = torch.full((1,), float("nan"), dtype=torch.float32, device="cuda")
+        lib.wush_transform_amax(_as_input(x, bf16).cuda(), tt, kind, b, out)
+        torch.cuda.synchronize()
+        assert lib.wush_check_device_status() == 0
+        assert abs(float(out.item()) - want) <= 1e-5 * want, (bf16, float(out.item()), want)
+
+
 @pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4", "int4"])
 def test_full_size_sampled_rows(lib, fmt):
     # the bench's launch configuration (full workload, WUSH), oracle on sampled rows
