@@ -5,6 +5,8 @@ code, written independently of both the CUDA kernels and the oracle.
 """
 from __future__ import annotations
 
+import os
+
 import numpy as np
 
 from oracle import quant as Q
@@ -21,6 +23,11 @@ Y_TOL = 1e-5
 # needs no excuse and is not counted against the budget).
 MAX_EXEMPT_FRACTION = 1e-4
 GEMM_REL_FRO = 1e-3
+
+# Boundary-window counts of every comparison made in this process: the session
+# report in conftest prints them per test and per format (and writes them as JSON
+# to $WUSH_PARITY_REPORT when that is set).
+WINDOW_LOG: list = []
 
 
 def unpack_nibbles(packed: np.ndarray, rows: int, d_in: int) -> np.ndarray:
@@ -111,5 +118,9 @@ def compare_transform_quant(x_rows, t, fmt, gs, codes_gpu, scales_gpu, y_gpu=Non
     out["in_window"] = int(el_exempt.sum())
     out["exempt"] = int(((ref["codes"] != codes_gpu) & el_exempt).sum())
     out["scale_exempt"] = int(((want_sc != got_sc) & blk_exempt).sum())
+    out["blocks"] = rows * nb
+    out["scale_in_window"] = int(blk_exempt.sum())
+    WINDOW_LOG.append(dict(out, fmt=fmt, rows=rows, d_in=d_in,
+                           test=os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0]))
     assert out["exempt"] <= max(MAX_EXEMPT_FRACTION * out["elements"], 1), out
     return out

@@ -1,5 +1,7 @@
 """Pins for oracle.quant: brute-force scale and code search, grid membership,
 idempotence, special cases and the boundary margins used by the parity tests."""
+from fractions import Fraction
+
 import numpy as np
 import pytest
 
@@ -63,23 +65,76 @@ def test_mxfp4_special_blocks():
     assert q["codes"][0, 33] == 8                      # -1e-3 / 0.25 rounds to -0
 
 
+def _exact_nearest(q, grid, even_key):
+    """Index of the grid value nearest to the rational q >= 0 by exhaustive search;
+    at an exact tie the candidate with even_key(index) == 0 wins; above the last
+    value it saturates."""
+    if q >= grid[-1]:
+        return len(grid) - 1
+    dist = [abs(q - g) for g in grid]
+    best = min(dist)
+    cands = [i for i, dd in enumerate(dist) if dd == best]
+    return min(cands, key=lambda i: (even_key(i), i))
+
+
+_E2M1_EXACT = [Fraction(v) for v in F.E2M1_GRID]
+_E4M3_EXACT = [Fraction(v) for v in F.E4M3_GRID]
+
+
+def _e2m1_exact(y, d):
+    """E2M1 code of the exact quotient y / d (rationals): sign of y, magnitude RNE-sat."""
+    q = abs(Fraction(y)) / d
+    mag = _exact_nearest(q, _E2M1_EXACT, lambda i: i & 1)
+    return (8 if np.signbit(y) else 0) | mag
+
+
+def _nvfp4_exact(yb, s_g):
+    """Scale byte and codes of one NVFP4 block in exact rational arithmetic."""
+    amax = max(abs(Fraction(float(v))) for v in yb)
+    sg = Fraction(float(s_g))
+    sb = _exact_nearest(amax / (6 * sg), _E4M3_EXACT, lambda i: i & 1)
+    if sb == 0 or amax == 0:
+        return sb, [0] * len(yb)
+    d = _E4M3_EXACT[sb] * sg
+    return sb, [_e2m1_exact(float(v), d) for v in yb]
+
+
+def _int4_exact(yb):
+    """fp16 scale and codes of one INT4 block in exact rational arithmetic."""
+    amax = max(abs(Fraction(float(v))) for v in yb)
+    pre = amax / 7
+    # nearest fp16 by search over the two fp16 neighbours of pre, ties to the even significand
+    lo = np.float16(float(pre))
+    cands = {float(lo), float(np.nextafter(lo, np.float16(np.inf))), float(np.nextafter(lo, np.float16(0)))}
+    cands = sorted(c for c in cands if np.isfinite(c))
+    dist = [abs(pre - Fraction(c)) for c in cands]
+    best = min(dist)
+    tied = [c for c, dd in zip(cands, dist) if dd == best]
+    s = min(tied, key=lambda c: int(np.float16(c).view(np.uint16)) & 1)
+    s = min(s, 65504.0)
+    if s == 0:
+        return np.float16(0), [0] * len(yb)
+    sf = Fraction(s)
+    out = []
+    for v in yb:
+        q = Fraction(float(v)) / sf
+        k = int(np.floor(q))
+        frac = q - k
+        r = k + 1 if frac > Fraction(1, 2) or (frac == Fraction(1, 2) and k % 2) else k
+        out.append(max(-7, min(7, r)))
+    return np.float16(s), out
+
+
 def test_nvfp4_brute_force():
     y = _data(2, d=64, spread=False) * F32(3.0)
     s_g = F32(np.max(np.abs(y)) / (6 * 448) * 0.7)      # some blocks saturate the scale
     q = Q.quantize_nvfp4(y, s_g)
     yb = y.reshape(6, 4, 16)
-    grid = F.E4M3_GRID
     for r in range(6):
         for j in range(4):
-            amax = F32(np.max(np.abs(yb[r, j])))
-            t = F32(amax / F32(F32(6) * s_g))
-            dist = np.abs(grid - np.float64(t))
-            cands = np.flatnonzero(dist == dist.min())
-            sb = 126 if t > 448 else min(cands, key=lambda c: (c & 1, c))
+            sb, want = _nvfp4_exact(yb[r, j], s_g)
             assert q["scale_bytes"][r, j] == sb
-            d = F32(F32(grid[sb]) * s_g)
-            want = _nearest_code_brute((yb[r, j] * F32(F32(1) / d)).astype(F32))
-            assert np.array_equal(q["codes"][r, 16 * j:16 * j + 16], want)
+            assert np.array_equal(q["codes"][r, 16 * j:16 * j + 16], np.array(want))
 
 
 def test_int4_brute_force():
@@ -88,16 +143,80 @@ def test_int4_brute_force():
     yb = y.reshape(6, 4, 32)
     for r in range(6):
         for j in range(4):
-            s = np.float16(F32(np.max(np.abs(yb[r, j]))) / F32(7))
-            v = (yb[r, j] * F32(F32(1) / F32(s))).astype(F32)
-            want = []
-            for x in v.astype(np.float64):
-                cands = np.arange(-7, 8)
-                d = np.abs(cands - np.clip(x, -7.5, 7.5))
-                best = cands[d == d.min()]
-                want.append(best[best % 2 == 0][0] if len(best) > 1 else best[0])
-            assert np.array_equal(q["q"][r, 32 * j:32 * j + 32], np.array(want))
+            s, want = _int4_exact(yb[r, j])
             assert q["scale_fp16"][r, j] == s
+            assert np.array_equal(q["q"][r, 32 * j:32 * j + 32], np.array(want))
+
+
+def _near_ties(grid_mid, scale, rng, n):
+    """fp32 values exactly on scale * midpoint, and one fp32 ulp either side of it."""
+    out = []
+    for _ in range(n):
+        m = float(rng.choice(grid_mid))
+        v = F32(m * scale)
+        out += [v, np.nextafter(v, F32(np.inf)), np.nextafter(v, F32(-np.inf))]
+    return np.array(out, F32)
+
+
+def test_nvfp4_codes_at_and_next_to_ties_are_the_exact_quotients():
+    # Element values on, and one fp32 ulp off, every E2M1 midpoint of a block whose
+    # scale is fixed by one element at 6 d: the code must be the rounding of the
+    # real quotient y / d.  A reciprocal-multiply y * fl(1/d) flips some of these.
+    rng = np.random.default_rng(11)
+    s_g = F32(0.0123)
+    flips = 0
+    for sbv in (1.0, 1.125, 3.5, 13.0, 0.6875):
+        d = np.float64(sbv) * np.float64(s_g)
+        for trial in range(6):
+            body = _near_ties(F.E2M1_MIDPOINTS, d, rng, 5)
+            blk = np.concatenate([[F32(6.0 * d)], body])
+            y = blk.reshape(1, 16)
+            q = Q.quantize_nvfp4(y, s_g)
+            sb, want = _nvfp4_exact(y[0], s_g)
+            assert q["scale_bytes"][0, 0] == sb
+            assert np.array_equal(q["codes"][0], np.array(want))
+            rcp = F32(F32(1) / F32(F.e4m3_value(sb) * np.float64(s_g)))
+            flips += int(np.sum(F.e2m1_code((y[0] * rcp).astype(F32).astype(np.float64)) != np.array(want)))
+    assert flips > 0        # the cases do reach the order-of-operations difference
+
+
+def test_int4_codes_at_and_next_to_ties_are_the_exact_quotients():
+    rng = np.random.default_rng(12)
+    flips = 0
+    for s in (np.float16(0.0123), np.float16(1.0), np.float16(3.1e-3), np.float16(517.0)):
+        for trial in range(6):
+            body = _near_ties(F.INT4_MIDPOINTS, np.float64(s), rng, 10)
+            blk = np.concatenate([[F32(7.0 * np.float64(s))], body])
+            y = blk.reshape(1, 31)
+            y = np.concatenate([y, np.zeros((1, 1), F32)], axis=1)
+            q = Q.quantize_int4(y)
+            sc, want = _int4_exact(y[0])
+            assert q["scale_fp16"][0, 0] == sc
+            assert np.array_equal(q["q"][0], np.array(want))
+            rcp = F32(F32(1) / F32(sc))
+            flips += int(np.sum(np.clip(np.rint((y[0] * rcp).astype(F32)), -7, 7) != np.array(want)))
+    assert flips > 0
+
+
+def test_scale_decisions_at_and_next_to_ties_are_exact():
+    # Block amax on, and one fp32 ulp off, a UE4M3 midpoint (times 6 s_g) or an
+    # fp16 midpoint (times 7): the scale is the rounding of the real quotient.
+    s_g = F32(0.37)
+    for mid in F.E4M3_MIDPOINTS[::5]:
+        a = F32(mid * 6.0 * np.float64(s_g))
+        for v in (a, np.nextafter(a, F32(np.inf)), np.nextafter(a, F32(0))):
+            y = np.zeros((1, 16), F32)
+            y[0, 3] = v
+            assert Q.quantize_nvfp4(y, s_g)["scale_bytes"][0, 0] == _nvfp4_exact(y[0], s_g)[0]
+    rng = np.random.default_rng(13)
+    h = np.sort(rng.uniform(1e-3, 6e4, 60)).astype(np.float16)
+    for hv in h:
+        mid = (np.float64(hv) + np.float64(np.nextafter(hv, np.float16(np.inf)))) / 2
+        a = F32(mid * 7.0)
+        for v in (a, np.nextafter(a, F32(np.inf)), np.nextafter(a, F32(0))):
+            y = np.zeros((1, 32), F32)
+            y[0, 9] = -v
+            assert Q.quantize_int4(y)["scale_fp16"][0, 0] == _int4_exact(y[0])[0]
 
 
 @pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4", "int4"])
