@@ -37,6 +37,8 @@ _SIGNATURES = {
     "wush_save_transforms": (_i32, [ctypes.c_char_p, _i32, _i32, _i32, _i64, _vp, _vp, _vp, _i64]),
     "wush_transforms_file_info": (_i32, [ctypes.c_char_p, _vp, _vp, _vp, _vp, _vp, _vp]),
     "wush_load_transforms": (_i32, [ctypes.c_char_p, _vp, _vp, _i64, _vp, _i64]),
+    "wush_nvfp4_global_scale": (_i32, [_f32, _vp]),
+    "wush_nvfp4_alpha": (_i32, [_f32, _f32, _vp]),
     "wush_codes_bytes": (_sz, [_i64, _i64, _i32]),
     "wush_scales_bytes": (_sz, [_i64, _i64, _i32]),
     "wush_transform_quant": (_i32, [_vp, _i32, _i64, _i64, _vp, _i32, _i32, _f32, _vp, _vp, _vp, _vp]),
@@ -255,6 +257,20 @@ def itq3_quantize_weights(w_fp16: np.ndarray):
 
 
 # --------------------------------------------------------------------------- device
+
+def wush_nvfp4_global_scale(amax: float) -> float:
+    """Static NVFP4 per-tensor scale s_g = fp32(amax / 2688) (1 for an all-zero tensor)."""
+    out = ctypes.c_float()
+    _check("wush_nvfp4_global_scale", _lib.wush_nvfp4_global_scale(float(amax), ctypes.byref(out)))
+    return out.value
+
+
+def wush_nvfp4_alpha(s_gx: float, s_gw: float) -> float:
+    """The NVFP4 GEMM's alpha = fp32(s_gx * s_gw)."""
+    out = ctypes.c_float()
+    _check("wush_nvfp4_alpha", _lib.wush_nvfp4_alpha(float(s_gx), float(s_gw), ctypes.byref(out)))
+    return out.value
+
 
 def wush_codes_bytes(rows: int, d_in: int, fmt) -> int:
     return _lib.wush_codes_bytes(rows, d_in, _enum(FORMATS, fmt))

@@ -393,3 +393,19 @@ extern "C" int wush_calibrate_shared(const float* x_calib, int64_t n_calib, cons
   block_moments(w, d_out, d_in, block, sw.data());
   return wush_calibrate_shared_from_moments(sx.data(), sw.data(), d_in, block, kind, groups, t_x, t_w, index);
 }
+
+// Static NVFP4 per-tensor scale and GEMM alpha (see wush.h): plain fp32 IEEE
+// arithmetic, one rounding each.
+extern "C" int wush_nvfp4_global_scale(float amax, float* s_g) {
+  if (!s_g || !std::isfinite(amax) || amax < 0.0f) return WUSH_ERR_INVALID_ARG;
+  const float q = amax / 2688.0f;
+  *s_g = q >= 1e-30f ? q : 1.0f;
+  return WUSH_OK;
+}
+
+extern "C" int wush_nvfp4_alpha(float s_gx, float s_gw, float* alpha) {
+  if (!alpha || !std::isfinite(s_gx) || !std::isfinite(s_gw) || !(s_gx > 0.0f) || !(s_gw > 0.0f))
+    return WUSH_ERR_INVALID_ARG;
+  *alpha = s_gx * s_gw;
+  return WUSH_OK;
+}

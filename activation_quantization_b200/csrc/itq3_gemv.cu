@@ -346,22 +346,62 @@ static __device__ __align__(256) float g_itq3_noalloc_scratch[kNoAllocScratchFlo
 namespace {
 
 constexpr int kMaxDevices = 64;
-float* g_scratch_addr[kMaxDevices] = {};
+
+// Per device: the context the address was looked up in, and the address.
+struct ScratchEntry {
+  unsigned long long ctx_id;
+  float* addr;
+};
+ScratchEntry g_scratch[kMaxDevices] = {};
 std::mutex g_scratch_mutex;
 
-// Device address of the scratch array on the current device, looked up once per
-// device.  (In host code the array's name is only a host-side stand-in, so the
-// kernels must be handed this address, never the name.)
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Unique id of the current CUDA context (ids are never reused within a process,
+// also when a context is destroyed and a new one made at the same handle); 0 when
+// it cannot be had.
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of the scratch array in the current device's context, looked up
+// once per device and context: a device reset makes a new context and module, so
+// the next call looks the address up again.  (In host code the array's name is
+// only a host-side stand-in, so the kernels must be handed this address, never the
+// name.)
 int scratch_for_current_device(float** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return WUSH_ERR_CUDA;
+  const unsigned long long id = current_context_id();
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (!g_scratch_addr[dev]) {
+  ScratchEntry& e = g_scratch[dev];
+  // (no current context yet: id 0, looked up again until a context is current)
+  if (!e.addr || id == 0 || e.ctx_id != id) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_itq3_noalloc_scratch) != cudaSuccess || !p) return WUSH_ERR_CUDA;
-    g_scratch_addr[dev] = static_cast<float*>(p);
+    e.addr = static_cast<float*>(p);
+    e.ctx_id = id;
   }
-  *out = g_scratch_addr[dev];
+  *out = e.addr;
   return WUSH_OK;
 }
 

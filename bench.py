@@ -300,11 +300,11 @@ def run_gpu(args, rank, world):
     if fmt == "nvfp4":
         amax = torch.empty(1, dtype=torch.float32, device=dev)
         aq.wush_transform_amax(torch.from_numpy(xc).to(torch.bfloat16).to(dev), t_x, kind, b, amax)
-        gx = float(np.float32(amax.item() / (6 * 448)))
+        gx = aq.wush_nvfp4_global_scale(amax.item())
         wt_dev = torch.from_numpy(wt).to(torch.bfloat16).to(dev)
         aq.wush_transform_amax(wt_dev, t_w, kind, b, amax)
-        gw = float(np.float32(amax.item() / (6 * 448)))
-    alpha = float(np.float32(gx) * np.float32(gw)) if fmt == "nvfp4" else 1.0
+        gw = aq.wush_nvfp4_global_scale(amax.item())
+    alpha = aq.wush_nvfp4_alpha(gx, gw) if fmt == "nvfp4" else 1.0
     xs = [torch.from_numpy(x).to(torch.bfloat16).to(dev) for _ in range(ROTATIONS)]
     wcodes = []
     for _ in range(ROTATIONS):
@@ -533,11 +533,11 @@ def run_gpu(args, rank, world):
 
 # --------------------------------------------------------------------------- ITQ3 GEMV
 
-def run_itq3(args):
-    """Times itq3_dequant_gemv (both modes) at 1, 4 and 16 tokens; one JSON line each."""
+def measure_itq3(steps: int, warmup: int):
+    """Times itq3_dequant_gemv (both modes) at 1, 4 and 16 tokens; one dict per (tokens, mode)."""
     import torch
     import activation_quantization_b200 as aq
-    dev = torch.device("cuda", 0)
+    dev = torch.device("cuda", torch.cuda.current_device())
     w = synth.itq3_weights()
     d_out, d_in = w.shape
     codes, scales = aq.itq3_quantize_weights(w.astype(np.float16))
@@ -545,6 +545,7 @@ def run_itq3(args):
     cs = [torch.from_numpy(codes).to(dev) for _ in range(copies)]
     ss = [torch.from_numpy(scales).to(dev) for _ in range(copies)]
     peaks = load_peaks()
+    out = []
     for t in synth.ITQ3_TOKENS:
         x = torch.from_numpy(synth.itq3_activations(t).astype(np.float16)).to(dev)
         y = torch.empty((t, d_out), dtype=torch.float32, device=dev)
@@ -562,9 +563,9 @@ def run_itq3(args):
             with torch.cuda.graph(g, stream=stream):
                 for i in range(burst):
                     aq.itq3_dequant_gemv(cs[i % copies], ss[i % copies], x, d_out, mode, y, ws, stream=stream)
-            reps = max(1, args.steps // burst)
+            reps = max(1, steps // burst)
             with torch.cuda.stream(stream):
-                for _ in range(max(1, args.warmup // burst)):
+                for _ in range(max(1, warmup // burst)):
                     g.replay()
             stream.synchronize()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -577,12 +578,166 @@ def run_itq3(args):
             us = e0.elapsed_time(e1) / (reps * burst) * 1e3
             byts = codes.nbytes + scales.nbytes + t * d_in * 2 + t * d_out * 4
             tc = mode == 1 and t >= 3 and d_out % 128 == 0
-            print(json.dumps({"workload": f"itq3 W fp16 [{d_out}, {d_in}] 3-bit, {t} tokens",
-                              "mode": "fused inverse FWHT" if mode == 0 else "activation-side rotation",
-                              "kernel": "itq3_tc_kernel (tcgen05, fp16 levels from TMEM)" if tc
-                              else "itq3_gemv_kernel (CUDA cores)",
-                              "us": us, "GB_s": byts / us / 1e3, "frac_of_hbm": byts / us / 1e3 / peaks["hbm_gbs"],
-                              "bytes_per_call": byts}))
+            out.append({"workload": f"itq3 W fp16 [{d_out}, {d_in}] 3-bit, {t} tokens", "tokens": t,
+                        "mode": "fused inverse FWHT" if mode == 0 else "activation-side rotation",
+                        "kernel": "itq3_tc_kernel (tcgen05, fp16 levels from TMEM)" if tc
+                        else "itq3_gemv_kernel (CUDA cores)",
+                        "us": us, "GB_s": byts / us / 1e3, "frac_of_hbm": byts / us / 1e3 / peaks["hbm_gbs"],
+                        "bytes_per_call": byts})
+            del g
+    return out
+
+
+def run_itq3(args):
+    """Prints one JSON line per (tokens, mode) of the ITQ3 GEMV."""
+    for line in measure_itq3(args.steps, args.warmup):
+        print(json.dumps(line))
+
+
+# --------------------------------------------------------------------------- the other workloads
+
+EXTRA_STEPS = 24          # steps of each other workload: one CUDA graph, replayed after a warm replay
+
+
+def _graph_kernel_times(stream, launches, n_steps, reps=3):
+    """Captures n_steps steps, each the callables ``launches`` (called with the step
+    index), into one CUDA graph with event nodes between them; replays it once warm,
+    then ``reps`` times timed.  Returns (us per step, [us per launch kind])."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(launches) + 1)]
+           for _ in range(n_steps)]
+    with torch.cuda.graph(g, stream=stream):
+        for j in range(n_steps):
+            for i, fn in enumerate(launches):
+                evs[j][i].record(stream)
+                fn(j)
+            evs[j][-1].record(stream)
+    with torch.cuda.stream(stream):
+        g.replay()
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+    stream.synchronize()
+    per_step = 1e3 * e0.elapsed_time(e1) / (reps * n_steps)
+    per_kind = [1e3 * float(np.mean([e[i].elapsed_time(e[i + 1]) for e in evs])) for i in range(len(launches))]
+    del g
+    return per_step, per_kind
+
+
+def measure_layer(dev, stream, inputs, fmt, kind, tokens=None):
+    """The step (transform + quantise of X, then the GEMM) of one workload, timed as
+    a graph of EXTRA_STEPS steps over rotating copies; weights prepared offline."""
+    import torch
+    import activation_quantization_b200 as aq
+    w, x, wt, xc = inputs
+    if tokens:
+        x = x[:tokens]
+    M, N, K, b = x.shape[0], w.d_out, w.d_in, w.block
+    tx, tw = aq.wush_calibrate(xc, wt, b, kind)
+    t_x, t_w = torch.from_numpy(tx).to(dev), torch.from_numpy(tw).to(dev)
+    gx = gw = 0.0
+    alpha = 1.0
+    wt_dev = torch.from_numpy(wt).to(torch.bfloat16).to(dev)
+    if fmt == "nvfp4":
+        amax = torch.zeros(1, dtype=torch.float32, device=dev)
+        aq.wush_transform_amax(torch.from_numpy(xc).to(torch.bfloat16).to(dev), t_x, kind, b, amax)
+        gx = aq.wush_nvfp4_global_scale(amax.item())
+        aq.wush_transform_amax(wt_dev, t_w, kind, b, amax)
+        gw = aq.wush_nvfp4_global_scale(amax.item())
+        alpha = aq.wush_nvfp4_alpha(gx, gw)
+    xs = [torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16).to(dev) for _ in range(ROTATIONS)]
+    bc, bs = aq.alloc_quant_outputs(N, K, fmt, dev)
+    aq.wush_transform_quant(wt_dev, t_w, kind, fmt, bc, bs, gw)
+    del wt_dev
+    wcodes = [(bc, bs)] + [(bc.clone(), bs.clone()) for _ in range(ROTATIONS - 1)]
+    acodes = [aq.alloc_quant_outputs(M, K, fmt, dev) for _ in range(ROTATIONS)]
+    y = torch.empty((M, N), dtype=torch.float32, device=dev)
+    ws = (torch.empty(aq.wush_qgemm_int4_workspace_bytes(M, N, K), dtype=torch.uint8, device=dev)
+          if fmt == "int4" else None)
+
+    def tq(j):
+        r = j % ROTATIONS
+        aq.wush_transform_quant(xs[r], t_x, kind, fmt, acodes[r][0], acodes[r][1], gx, stream=stream)
+
+    def gemm(j):
+        r = j % ROTATIONS
+        (a, sa), (bb, sb) = acodes[r], wcodes[r]
+        if fmt == "int4":
+            aq.wush_qgemm_int4_ws(a, sa, bb, sb, M, N, K, ws, y, stream=stream)
+        else:
+            aq.wush_qgemm(a, sa, bb, sb, M, N, K, fmt, alpha, y, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for j in range(ROTATIONS):
+            tq(j)
+            gemm(j)
+    stream.synchronize()
+    step_us, (tq_us, gm_us) = _graph_kernel_times(stream, [tq, gemm], EXTRA_STEPS)
+    if aq.wush_check_device_status(stream) != 0:
+        raise RuntimeError(f"device status after {w.name} {kind}")
+    peaks = load_peaks()
+    tq_bytes = M * K * 2 + aq.wush_codes_bytes(M, K, fmt) + aq.wush_scales_bytes(M, K, fmt) + (K // b) * b * b * 4
+    flops = 2.0 * M * N * K
+    gemm_peak = peaks["bf16_tflops"] * (FP4_OVER_BF16 if fmt != "int4" else 1.0)
+    gemm_tflops = flops / (gm_us * 1e-6) / 1e12
+    return {"M": M, "N": N, "K": K, "format": fmt, "transform": kind, "step_us": step_us,
+            "TFLOP_s": flops / (step_us * 1e-6) / 1e12,
+            "transform_quant": {"us": tq_us, "GB_s": tq_bytes / (tq_us * 1e-6) / 1e9,
+                                "frac_of_hbm": tq_bytes / (tq_us * 1e-6) / 1e9 / peaks["hbm_gbs"],
+                                "bytes_per_launch": tq_bytes},
+            "gemm": {"kernel": ("int4_dequant_kernel x2 + hgemm_pair_kernel (fp16 MMA)" if fmt == "int4"
+                                else "qgemm_pair_kernel (block-scaled FP4 MMA)"),
+                     "us": gm_us, "TFLOP_s": gemm_tflops, "frac_of_peak": gemm_tflops / gemm_peak,
+                     "peak": gemm_peak}}
+
+
+def tiny_losses(dev):
+    """Loss l = ||y - W^T X||_F^2 / (d_out tokens) of the GPU layer on the tiny workload
+    (MXFP4), for the identity, Hadamard and WUSH transforms."""
+    import torch
+    import activation_quantization_b200 as aq
+    w, x, wt, xc = build_inputs("tiny")
+    M, N, K = w.tokens, w.d_out, w.d_in
+    ref = x.astype(np.float64) @ wt.astype(np.float64).T
+    out = {}
+    for kind in ("identity", "hadamard", "wush"):
+        tx, tw = aq.wush_calibrate(xc, wt, w.block, kind)
+        ac, as_ = aq.alloc_quant_outputs(M, K, "mxfp4", dev)
+        bc, bs = aq.alloc_quant_outputs(N, K, "mxfp4", dev)
+        aq.wush_transform_quant(torch.from_numpy(x).to(dev), torch.from_numpy(tx).to(dev), kind, "mxfp4", ac, as_)
+        aq.wush_transform_quant(torch.from_numpy(wt).to(dev), torch.from_numpy(tw).to(dev), kind, "mxfp4", bc, bs)
+        y = torch.empty((M, N), dtype=torch.float32, device=dev)
+        aq.wush_qgemm(ac, as_, bc, bs, M, N, K, "mxfp4", 1.0, y)
+        d = y.cpu().numpy().astype(np.float64) - ref
+        out[kind] = float(np.sum(d * d) / (N * M))
+    out["workload"] = (f"tiny: X fp32 [{M} tok, {K}] N(0,1) with {w.n_outlier} outlier channels "
+                       f"x{w.outlier_factor:g}; W [{N}, {K}]; MXFP4 b=32 through the GPU path")
+    return out
+
+
+def run_extras(args):
+    """The other workloads' kernels, each measured in this process, for the bench line."""
+    import torch
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.Stream(device=dev)
+    extras = {}
+    inp = build_inputs("down_proj")
+    extras["down_proj"] = {k: measure_layer(dev, stream, inp, "nvfp4", k) for k in ("wus", "wush")}
+    del inp
+    inp = build_inputs("int4")
+    extras["int4_2048"] = measure_layer(dev, stream, inp, "int4", "wush", tokens=2048)
+    extras["int4_8192"] = measure_layer(dev, stream, inp, "int4", "wush")
+    del inp
+    torch.cuda.empty_cache()
+    extras["itq3"] = measure_itq3(max(args.steps, 96), 48)
+    extras["tiny_loss"] = tiny_losses(dev)
+    torch.cuda.empty_cache()
+    return extras
 
 
 # --------------------------------------------------------------------------- main
@@ -598,6 +753,8 @@ def main():
     ap.add_argument("--transform", default=None, choices=["identity", "hadamard", "wus", "wush", "wush_diag"],
                     help="override the workload's block transform (calibrated from the same tokens)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the other workloads' kernel timings (down_proj, int4, itq3, tiny loss)")
     ap.add_argument("--share-groups", type=int, default=0,
                     help="share the dense transforms among this many groups of similar blocks")
     ap.add_argument("--dynamic-scale", action="store_true",
@@ -643,6 +800,8 @@ def main():
     dist_init(world)
     result, ctx = run_gpu(args, rank, world)
     if rank == 0:
+        if world == 1 and not args.no_extras:
+            result.update(run_extras(args))
         if world == 1 and not args.no_cpu_baseline:
             w, x, wt, xc, fmt, kind = ctx
             result["cpu_baseline"] = time_oracle(w, x, wt, xc, fmt, kind, groups=args.share_groups)

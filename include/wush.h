@@ -130,6 +130,24 @@ int wush_calibrate_shared_from_moments(const double* sigma_x, const double* sigm
                                        int block, int kind, int groups, float* t_x, float* t_w,
                                        int32_t* index);
 
+/* Static NVFP4 per-tensor scale (host, no CUDA).  The pages name NVFP4 without
+ * its scale rule (WUSH news article, experiments paragraph); the reading used
+ * throughout is s_g = amax / 2688 with 2688 = 6 * 448 (the largest E2M1 magnitude
+ * times the largest UE4M3 block scale), so the largest value of the tensor maps to
+ * the top of both grids.  ``amax`` is the largest |T x| of the calibration tokens
+ * (activations; e.g. from wush_transform_amax) or of the transformed weights.
+ * *s_g receives fp32(amax / 2688) rounded once to nearest even, or 1 when that is
+ * below 1e-30 (an all-zero tensor, whose codes are 0 whatever the scale): the
+ * same rule the device applies in wush_transform_quant_nvfp4_dynamic.
+ * WUSH_ERR_INVALID_ARG for a negative or non-finite amax or a NULL s_g. */
+int wush_nvfp4_global_scale(float amax, float* s_g);
+
+/* The NVFP4 GEMM's alpha for wush_qgemm: *alpha = fp32(s_gx * s_gw), the product
+ * of the activations' and the weights' per-tensor scales rounded once (the device
+ * forms the same product in wush_qgemm_nvfp4_dynamic).  WUSH_ERR_INVALID_ARG for
+ * a non-positive or non-finite scale or a NULL alpha. */
+int wush_nvfp4_alpha(float s_gx, float s_gw, float* alpha);
+
 /* How the second moments behind a set of transforms were normalised (recorded in
  * the transforms file; see below). */
 typedef enum { WUSH_NORM_UNKNOWN = 0, WUSH_NORM_MEAN = 1 } wush_sigma_norm;
@@ -386,7 +404,9 @@ int itq3_dequant_gemv(const uint8_t* codes, const void* scales_fp16, const void*
  * Arguments as in itq3_dequant_gemv; tokens * d_in must be <= 262,144, else
  * WUSH_ERR_BUFFER_TOO_SMALL and nothing is launched.  Calls no allocating
  * routine.  The first call on a device looks up the array's device address (with
- * that device current); make that first call before any stream capture.  All
+ * that device current); make that first call before any stream capture.  The
+ * address is kept per device and CUDA context: after a device reset (which makes
+ * a new context) the next call looks it up again, so it too is a first call.  All
  * calls on a device share the array: calls whose kernels overlap on the GPU
  * (different streams, no ordering between them) race on it.  Nothing needs to
  * start at zero: every call overwrites the part of the array it reads. */

@@ -163,3 +163,27 @@ def test_calibrate_every_block_size_matches_oracle(kind, b):
         # the defining property T_W^T T_X = I, in fp32 storage
         eye = np.einsum("jki,jkl->jil", tw.astype(np.float64), tx.astype(np.float64))
         assert np.max(np.abs(eye - np.eye(b))) < 1e-4
+
+
+def test_nvfp4_static_scale_and_alpha_match_the_oracle_rule():
+    # s_g = amax / 2688 rounded once to fp32 (the oracle's static rule, which
+    # rounds the fp64 quotient; with 53 >= 2*24 + 2 bits that double rounding is
+    # the correctly rounded fp32 quotient); alpha = fp32(s_gx * s_gw)
+    from oracle import calibrate as C
+    rng = np.random.default_rng(21)
+    amaxes = np.concatenate([np.float32(10.0) ** rng.uniform(-20, 20, 2000),
+                             np.float32([1.0, 2688.0, 448.0 * 6, 1e-3, 3.4e38])]).astype(np.float32)
+    for a in amaxes:
+        want = C.nvfp4_global_scale(np.array([[a]], np.float32))
+        assert np.float32(aq.wush_nvfp4_global_scale(float(a))) == want, a
+    assert aq.wush_nvfp4_global_scale(0.0) == 1.0
+    assert np.float32(aq.wush_nvfp4_global_scale(0.0)) == C.nvfp4_dynamic_global_scale(np.zeros((1, 16), np.float32))
+    for _ in range(500):
+        gx, gw = np.float32(10.0 ** rng.uniform(-8, 2, 2))
+        assert np.float32(aq.wush_nvfp4_alpha(float(gx), float(gw))) == np.float32(np.float64(gx) * np.float64(gw))
+    for bad in (-1.0, float("nan"), float("inf")):
+        with pytest.raises(aq.WushError):
+            aq.wush_nvfp4_global_scale(bad)
+    for bad in ((0.0, 1.0), (1.0, -2.0), (float("nan"), 1.0), (1.0, float("inf"))):
+        with pytest.raises(aq.WushError):
+            aq.wush_nvfp4_alpha(*bad)

@@ -145,6 +145,62 @@ def test_full_size_up_proj_sampled(lib):
     assert _rel_fro(got, want) <= P.GEMM_REL_FRO
 
 
+@pytest.mark.parametrize("fmt, mnk", [("nvfp4", (4096, 4096, 12288)), ("nvfp4", (4096, 4096, 1024)),
+                                      ("mxfp4", (4096, 4096, 1024))])
+def test_gemm_random_codes_many_tiles_per_pair(lib, fmt, mnk):
+    # 16 x 16 = 256 pair tiles of 256 x 256 for 74 CTA pairs: every pair runs three
+    # or four tiles, handing its accumulator back between them; (4096, 4096, 12288)
+    # is the NVFP4 down_proj launch.  The oracle checks 64 sampled rows, all columns.
+    m, n, k = mnk
+    a_c, a_s, a_dq = _random_operand(301 + k, m, k, fmt)
+    b_c, b_s, b_dq = _random_operand(402 + k, n, k, fmt)
+    alpha = 0.37 if fmt == "nvfp4" else 1.0
+    dev = "cuda"
+    y = torch.full((m, n), float("nan"), dtype=torch.float32, device=dev)
+    lib.wush_qgemm(torch.from_numpy(a_c).to(dev), torch.from_numpy(a_s).to(dev), torch.from_numpy(b_c).to(dev),
+                   torch.from_numpy(b_s).to(dev), m, n, k, fmt, alpha, y)
+    assert lib.wush_check_device_status() == 0
+    got = y.cpu().numpy().astype(np.float64)
+    assert np.isfinite(got).all()
+    rows = np.sort(np.random.default_rng(17).choice(m, 64, replace=False))
+    rows[0], rows[-1] = 0, m - 1
+    err = _rel_fro(got[rows], G.gemm_dequantized(a_dq[rows], b_dq, alpha))
+    assert err <= 1e-5, err
+
+
+def test_full_size_down_proj_sampled(lib):
+    # the NVFP4 down_proj launch: M 4096, N 4096, K 12288, WUSH b = 16 with static
+    # per-tensor scales; the oracle checks 48 rows x 256 columns of y
+    w = synth.WORKLOADS["down_proj"]
+    x = synth.activations(w)
+    wt = synth.weights(w)
+    xc = synth.activations(w, tokens=1024, calib=True)
+    tx, tw = C.calibrate(xc, wt[:2048], 16, "wush")
+    tx, tw = tx.astype(np.float32), tw.astype(np.float32)
+    gx = C.nvfp4_global_scale(T.apply_block_transform(xc, tx).astype(np.float32))
+    gw = C.nvfp4_global_scale(T.apply_block_transform(wt, tw).astype(np.float32))
+    alpha = lib.wush_nvfp4_alpha(float(gx), float(gw))
+    dev = "cuda"
+    m, n, k = w.tokens, w.d_out, w.d_in
+    ac, as_ = lib.alloc_quant_outputs(m, k, "nvfp4")
+    bc, bs = lib.alloc_quant_outputs(n, k, "nvfp4")
+    lib.wush_transform_quant(torch.from_numpy(x).to(torch.bfloat16).to(dev), torch.from_numpy(tx).to(dev),
+                             "wush", "nvfp4", ac, as_, float(gx))
+    lib.wush_transform_quant(torch.from_numpy(wt).to(torch.bfloat16).to(dev), torch.from_numpy(tw).to(dev),
+                             "wush", "nvfp4", bc, bs, float(gw))
+    y = torch.empty((m, n), dtype=torch.float32, device=dev)
+    lib.wush_qgemm(ac, as_, bc, bs, m, n, k, "nvfp4", alpha, y)
+    assert lib.wush_check_device_status() == 0
+    rng = np.random.default_rng(19)
+    rows = np.sort(rng.choice(m, 48, replace=False))
+    cols = np.sort(rng.choice(n, 256, replace=False))
+    qa = Q.transform_quantize(x[rows], tx, "nvfp4", gx)
+    qb = Q.transform_quantize(wt[cols], tw, "nvfp4", gw)
+    want = G.gemm_dequantized(qa["dq"] / np.float64(gx), qb["dq"] / np.float64(gw), alpha)
+    got = y.cpu().numpy()[np.ix_(rows, cols)].astype(np.float64)
+    assert _rel_fro(got, want) <= P.GEMM_REL_FRO
+
+
 @pytest.mark.parametrize("m", [128, 256])     # single-CTA kernel, CTA-pair kernel
 def test_bounded_wait_gives_up_and_context_survives(lib, m):
     n, k = 256, 512

@@ -110,10 +110,12 @@ def test_int4_gemm_two_pass_random(lib, mnk):
     assert diff <= 1e-5, diff
 
 
-def test_int4_two_pass_end_to_end_sampled(lib):
-    # the int4 workload at 2048 tokens through the two-pass form, oracle on 40 x 256
+@pytest.mark.parametrize("m", [2048, 8192])
+def test_int4_two_pass_end_to_end_sampled(lib, m):
+    # the int4 workload at 2048 and 8192 tokens (the bench's launches) through the
+    # two-pass form, oracle on 40 x 256
     w = synth.WORKLOADS["int4"]
-    m, n, k = 2048, w.d_out, w.d_in
+    n, k = w.d_out, w.d_in
     x = synth.activations(w, tokens=m)
     wt = synth.weights(w)
     xc = synth.activations(w, tokens=1024, calib=True)
