@@ -378,6 +378,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_sync();                       // both CTAs' barriers exist before either touches the other's
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Launched after another kernel with programmatic stream serialization, the set-up
+  // above overlaps that kernel's tail; no operand is read and no output written
+  // before the wait.
+  pdl_launch_dependents();
+  pdl_wait();
 
   auto give_up = [&]() {
     if (!*abort_flag) {
@@ -612,13 +617,15 @@ int launch_pair(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const ui
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   if (cudaLaunchKernelEx(&cfg, kern, ma, mb, msa, msb, my, static_cast<int>(M), static_cast<int>(N),
                          static_cast<int>(K), alpha, alpha_scale, polls, debug_never) != cudaSuccess)
     return WUSH_ERR_CUDA;

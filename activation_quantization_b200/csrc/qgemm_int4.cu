@@ -338,17 +338,17 @@ constexpr uint32_t kTmemCols = 512;                  // two 256-column accumulat
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 }  // namespace hp
 
-// Tile order of the fp16 pair GEMM: groups of kGroupRows 256-row blocks of A, N
-// fastest inside a group, so the tiles in flight at once share a few row blocks of
-// A and a few of B (each group reads A's rows once and B once) instead of sweeping
-// all of A for every column of tiles.
-constexpr int kGroupRows = 8;
-
-__device__ __forceinline__ void pair_tile_coords(int pt, int mt, int nt, int& pm, int& pn) {
-  const int g = pt / (kGroupRows * nt);
-  const int rows = min(kGroupRows, mt - g * kGroupRows);
-  const int w = pt - g * kGroupRows * nt;
-  pm = g * kGroupRows + w % rows;
+// Tile order of the fp16 pair GEMM: groups of ``group`` 256-row blocks of A, the
+// row blocks fastest inside a group, so the tiles in flight at once share one or
+// two 256-row blocks of B while the group's rows of A stay in L2 (their loads are
+// marked evict-last, y's stores evict-first) for the whole sweep over N: each
+// group reads its rows of A once and B once.  The host sizes the group so its rows
+// of A fill at most about two thirds of L2 (all of A when it fits).
+__device__ __forceinline__ void pair_tile_coords(int pt, int mt, int nt, int group, int& pm, int& pn) {
+  const int g = pt / (group * nt);
+  const int rows = min(group, mt - g * group);
+  const int w = pt - g * group * nt;
+  pm = g * group + w % rows;
   pn = w / rows;
 }
 
@@ -371,7 +371,8 @@ __device__ __forceinline__ void mma_f16_pair(uint32_t tmem_d, uint64_t adesc, ui
 //               then 128-byte-swizzled shared chunks -> TMA stores of y.
 __global__ void __launch_bounds__(hp::kThreads, 1)
     hgemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                      const __grid_constant__ CUtensorMap tmap_y, int M, int N, int K, int64_t max_polls) {
+                      const __grid_constant__ CUtensorMap tmap_y, int M, int N, int K, int group,
+                      int64_t max_polls) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* epi_smem = smem + hp::kStages * hp::kStageBytes;
@@ -421,11 +422,12 @@ __global__ void __launch_bounds__(hp::kThreads, 1)
 
   if (warp == 0) {
     if (elect_one()) {
+      const uint64_t keep_a = l2_policy_evict_last();
       int it = 0;
       bool ok = true;
       for (int pt = pair; ok && pt < n_ptiles; pt += n_pairs) {
         int pm, pn;
-        pair_tile_coords(pt, mt, nt, pm, pn);
+        pair_tile_coords(pt, mt, nt, group, pm, pn);
         const int arow = pm * 256 + static_cast<int>(rank) * 128;   // this CTA's A rows
         const int brow = pn * 256 + static_cast<int>(rank) * 128;   // this CTA's half of the B rows
         for (int kt = 0; kt < k_tiles; ++kt, ++it) {
@@ -437,7 +439,7 @@ __global__ void __launch_bounds__(hp::kThreads, 1)
           }
           uint8_t* sa = smem + s * hp::kStageBytes;
           if (leader) mbar_arrive_expect_tx(&full[s], 2 * hp::kStageBytes);
-          tma_load_2d_pair(sa, &tmap_a, kt * hp::kRowBytes, arow, &full[s]);
+          tma_load_2d_pair_hint(sa, &tmap_a, kt * hp::kRowBytes, arow, &full[s], keep_a);
           tma_load_2d_pair(sa + hp::kABytes, &tmap_b, kt * hp::kRowBytes, brow, &full[s]);
         }
       }
@@ -477,11 +479,12 @@ __global__ void __launch_bounds__(hp::kThreads, 1)
   } else {
     const int ew = warp - 2, q = warp & 3, half = ew / 4;
     uint8_t* buf = epi_smem + ew * hp::kEpiChunk;
+    const uint64_t stream_y = l2_policy_evict_first();
     int tcount = 0;
     for (int pt = pair; pt < n_ptiles; pt += n_pairs, ++tcount) {
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
       int pm, pn;
-      pair_tile_coords(pt, mt, nt, pm, pn);
+      pair_tile_coords(pt, mt, nt, group, pm, pn);
       const int a = tcount & 1;
       bool ok = mbar_wait_bounded(&acc_full[a], (tcount >> 1) & 1, max_polls, kDeadlineNs, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
@@ -506,7 +509,8 @@ __global__ void __launch_bounds__(hp::kThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(&tmap_y, buf, pn * 256 + half * 128 + 32 * c, pm * 256 + static_cast<int>(rank) * 128 + q * 32);
+          tma_store_2d_hint(&tmap_y, buf, pn * 256 + half * 128 + 32 * c, pm * 256 + static_cast<int>(rank) * 128 + q * 32,
+                            stream_y);
           bulk_commit_group();
         }
       }
@@ -593,6 +597,12 @@ int launch_hgemm_pair(const __half* a, const __half* b, int64_t M, int64_t N, in
     return WUSH_ERR_CUDA;
   const int64_t n_ptiles = (M / 256) * (N / 256);
   const int pairs = static_cast<int>(n_ptiles < sms / 2 ? n_ptiles : sms / 2);
+  // row blocks of A per group: as many 256-row blocks as fit in about two thirds of
+  // L2 (fp16, K wide), at least 8
+  int l2 = 0;
+  if (cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess || l2 <= 0) return WUSH_ERR_CUDA;
+  const int64_t fit = (static_cast<int64_t>(l2) * 2 / 3) / (256 * K * 2);
+  const int group = static_cast<int>(fit < 8 ? 8 : (fit > M / 256 ? M / 256 : fit));
   const int64_t polls = g_wait_limit_override > 0 ? g_wait_limit_override : kDefaultPolls;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
@@ -607,7 +617,7 @@ int launch_hgemm_pair(const __half* a, const __half* b, int64_t M, int64_t N, in
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, hgemm_pair_kernel, ma, mb, my, static_cast<int>(M), static_cast<int>(N),
-                         static_cast<int>(K), polls) != cudaSuccess)
+                         static_cast<int>(K), group, polls) != cudaSuccess)
     return WUSH_ERR_CUDA;
   return launch_status();
 }
@@ -669,8 +679,9 @@ extern "C" int wush_qgemm_int4_ws(const uint8_t* a_codes, const void* a_scales, 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   __half* wa = static_cast<__half*>(workspace);
   __half* wb = wa + M * K;
-  int status = launch_dequant(a_codes, a_scales, M, K, wa, st);
-  if (status == WUSH_OK) status = launch_dequant(b_codes, b_scales, N, K, wb, st);
+  // B first: A's fp16 copy, which the GEMM keeps in L2, is then the most recently written
+  int status = launch_dequant(b_codes, b_scales, N, K, wb, st);
+  if (status == WUSH_OK) status = launch_dequant(a_codes, a_scales, M, K, wa, st);
   if (status == WUSH_OK) status = launch_hgemm_pair(wa, wb, M, N, K, y, st);
   return status;
 }

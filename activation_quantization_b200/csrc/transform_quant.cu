@@ -16,6 +16,7 @@
 #include <cuda_fp16.h>
 
 #include "common.cuh"
+#include "quant_decide.cuh"
 
 namespace wush {
 namespace {
@@ -25,42 +26,6 @@ constexpr int kBlocksPerCta = 4;
 
 enum Kind : int { kIdentity = 0, kHadamard = 1, kDense = 2 };
 enum Fmt : int { kMx = 0, kNv = 1, kI4 = 2, kAmax = 3 };
-
-__device__ __forceinline__ float exp2i(int k) {  // exact 2^k for k in [-149, 127]
-  return k >= -126 ? __uint_as_float(static_cast<uint32_t>(k + 127) << 23)
-                   : __uint_as_float(1u << (k + 149));
-}
-
-__device__ __forceinline__ int floor_log2(float a) {  // a > 0, finite
-  const uint32_t b = __float_as_uint(a);
-  const int e = (b >> 23) & 0xFF;
-  return e ? e - 127 : (31 - __clz(b & 0x7FFFFFu)) - 149;
-}
-
-// E2M1 code of v: nearest of {0, .5, 1, 1.5, 2, 3, 4, 6}, ties to the even code,
-// saturating at 6; the sign bit is v's sign bit.
-__device__ __forceinline__ uint32_t e2m1_rne(float v) {
-  const float a = fabsf(v);
-  const uint32_t m = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) + (a > 2.5f) +
-                     (a >= 3.5f) + (a > 5.0f);
-  return m | ((__float_as_uint(v) >> 28) & 8u);
-}
-
-// UE4M3 code of t >= 0: round to nearest, ties to even, saturating at 448 (code 126).
-__device__ __forceinline__ uint32_t ue4m3_rne(float t) {
-  if (!(t < 448.0f)) return 126u;
-  if (t == 0.0f) return 0u;
-  int e = floor_log2(t);
-  if (e < -6) return static_cast<uint32_t>(rintf(t * 512.0f));  // subnormal step 2^-9; 8 = 2^-6
-  float q = rintf(t * exp2i(3 - e));                              // in [8, 16]
-  if (q >= 16.0f) { q = 8.0f; ++e; }
-  return (static_cast<uint32_t>(e + 7) << 3) | (static_cast<uint32_t>(q) - 8u);
-}
-
-__device__ __forceinline__ float ue4m3_value(uint32_t c) {
-  const uint32_t e = c >> 3, m = c & 7u;
-  return e == 0 ? static_cast<float>(m) * 0.001953125f : static_cast<float>(8u + m) * exp2i(static_cast<int>(e) - 10);
-}
 
 template <int B, bool XF32>
 __device__ __forceinline__ void load_block(const void* x, int64_t off, float (&v)[B]) {
@@ -190,43 +155,30 @@ __global__ void __launch_bounds__(kRowsPerCta) transform_quant_kernel(
         continue;
       }
 
-      uint32_t c[B];
+      // every decision is the round-to-nearest-even of the exact quotient (quant_decide.cuh)
+      uint32_t wv[B / 8];
       if constexpr (FMT == kMx) {
         int e = amax > 0.f ? floor_log2(amax) - 2 : -127;
         e = e < -127 ? -127 : (e > 127 ? 127 : e);
         const float inv = exp2i(-e);  // y * 2^-e is exact
 #pragma unroll
-        for (int i = 0; i < B; ++i) c[i] = amax > 0.f ? e2m1_rne(y[i] * inv) : 0u;
+        for (int w = 0; w < B / 8; ++w) wv[w] = amax > 0.f ? e2m1x8_times(y + 8 * w, inv) : 0u;
         s_sf[(tid & 31) * 16 + (tid >> 5) * 4 + jj] = static_cast<uint8_t>(e + 127);
       } else if constexpr (FMT == kNv) {
-        const float den = 6.0f * gscale;
-        const uint32_t sb = ue4m3_rne(__fdiv_rn(amax, den));
-        const float d = __fmul_rn(ue4m3_value(sb), gscale);
+        const uint32_t sb = nvfp4_scale_byte(amax, gscale, __frcp_rn(__fmul_rn(6.0f, gscale)));
+        const float sbv = ue4m3_val(sb);
         const bool live = sb != 0u && amax > 0.f;
-        const float rd = live ? __fdiv_rn(1.0f, d) : 0.f;
+        const float rd = live ? __frcp_rn(__fmul_rn(sbv, gscale)) : 0.f;
 #pragma unroll
-        for (int i = 0; i < B; ++i) c[i] = live ? e2m1_rne(y[i] * rd) : 0u;
+        for (int w = 0; w < B / 8; ++w) wv[w] = live ? nvfp4_codes8(y + 8 * w, rd, sbv, gscale) : 0u;
         s_sf[(tid & 31) * 16 + (tid >> 5) * 4 + jj] = static_cast<uint8_t>(sb);
       } else {  // INT4
-        const float pre = fminf(__fdiv_rn(amax, 7.0f), 65504.0f);
-        const __half s16 = __float2half_rn(pre);
+        const __half s16 = int4_scale(amax);
         const float s = __half2float(s16);
-        const float rs = s > 0.f ? __fdiv_rn(1.0f, s) : 0.f;
+        const float rs = s > 0.f ? __frcp_rn(s) : 0.f;
 #pragma unroll
-        for (int i = 0; i < B; ++i) {
-          float q = s > 0.f ? rintf(y[i] * rs) : 0.f;
-          q = fminf(fmaxf(q, -7.0f), 7.0f);
-          c[i] = static_cast<uint32_t>(static_cast<int>(q)) & 0xFu;
-        }
+        for (int w = 0; w < B / 8; ++w) wv[w] = s > 0.f ? int4_codes8(y + 8 * w, rs, s) : 0u;
         reinterpret_cast<__half*>(scales)[r * nb + j] = s16;
-      }
-      uint32_t wv[B / 8];
-#pragma unroll
-      for (int w = 0; w < B / 8; ++w) {
-        uint32_t acc = 0;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) acc |= c[8 * w + q] << (4 * q);
-        wv[w] = acc;
       }
       uint8_t* cp = codes + r * (d_in / 2) + j * (B / 2);
       if constexpr (B == 32) {

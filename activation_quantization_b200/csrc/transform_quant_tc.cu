@@ -42,6 +42,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "quant_decide.cuh"
 #include "sm100.cuh"
 
 namespace wush {
@@ -85,69 +86,6 @@ enum Fmt : int { kMx = 0, kNv = 1, kI4 = 2, kAm = 3 };
 
 __device__ int g_tq_error = 0;
 
-__device__ __forceinline__ float exp2i(int k) {
-  return k >= -126 ? __uint_as_float(static_cast<uint32_t>(k + 127) << 23) : __uint_as_float(1u << (k + 149));
-}
-
-__device__ __forceinline__ int floor_log2(float a) {
-  const uint32_t b = __float_as_uint(a);
-  const int e = (b >> 23) & 0xFF;
-  return e ? e - 127 : (31 - __clz(b & 0x7FFFFFu)) - 149;
-}
-
-// UE4M3 scale byte of t >= 0: round to nearest even, saturating at 448 (the
-// hardware conversion with .satfinite; the sign bit of a non-negative input is 0).
-__device__ __forceinline__ uint32_t ue4m3_rne(float t) {
-  uint16_t h;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(0.0f), "f"(t));
-  return h & 0xFFu;
-}
-
-// Value of a UE4M3 byte (exact through fp16).
-__device__ __forceinline__ float ue4m3_value(uint32_t c) {
-  uint32_t h2;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>(c)));
-  return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
-}
-
-// (a, b) * s as one packed f32x2 multiply, each lane rounded to nearest like FMUL.
-__device__ __forceinline__ void mul2(float a, float b, float s, float& pa, float& pb) {
-  unsigned long long x, y, z;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a), "f"(b));
-  asm("mov.b64 %0, {%1, %1};" : "=l"(y) : "f"(s));
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(z) : "l"(x), "l"(y));
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(pa), "=f"(pb) : "l"(z));
-}
-
-// Eight values -> eight E2M1 codes, element 0 in the low nibble (RNE, satfinite).
-__device__ __forceinline__ uint32_t e2m1x8(float v0, float v1, float v2, float v3, float v4, float v5, float v6,
-                                           float v7) {
-  uint32_t out;
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
-      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
-      : "=r"(out)
-      : "f"(v0), "f"(v1), "f"(v2), "f"(v3), "f"(v4), "f"(v5), "f"(v6), "f"(v7));
-  return out;
-}
-
-// Eight values times s -> eight E2M1 codes, element 0 in the low nibble (RNE, satfinite).
-__device__ __forceinline__ uint32_t e2m1x8_scaled(const float* v, float s) {
-  float p[8];
-#pragma unroll
-  for (int i = 0; i < 8; i += 2) mul2(v[i], v[i + 1], s, p[i], p[i + 1]);
-  return e2m1x8(p[0], p[1], p[2], p[3], p[4], p[5], p[6], p[7]);
-}
-
-__device__ __forceinline__ uint32_t int4_nibble(float v) {
-  int q = __float2int_rn(v);
-  q = q < -7 ? -7 : (q > 7 ? 7 : q);
-  return static_cast<uint32_t>(q) & 0xFu;
-}
-
 // max |y_i| as a pairwise tree (max is exact, so the order is free): depth log2 B
 // instead of a B-long dependent chain.
 template <int B>
@@ -163,40 +101,33 @@ __device__ __forceinline__ float block_amax(const float (&y)[B]) {
 }
 
 // Quantise one block of B fp32 values held by this thread.  Writes B/8 code
-// words and returns the scale (byte for MXFP4/NVFP4, fp16 bits for INT4).
+// words and returns the scale (byte for MXFP4/NVFP4, fp16 bits for INT4).  Every
+// decision is the round-to-nearest-even of the exact quotient (quant_decide.cuh).
 template <int B, int FMT>
-__device__ __forceinline__ uint32_t quantize_block(const float (&y)[B], float gscale, float den, uint32_t (&w)[B / 8]) {
+__device__ __forceinline__ uint32_t quantize_block(const float (&y)[B], float gscale, float inv_den,
+                                                  uint32_t (&w)[B / 8]) {
   const float amax = block_amax<B>(y);
   if constexpr (FMT == kMx) {
     int e = amax > 0.f ? floor_log2(amax) - 2 : -127;
     e = e < -127 ? -127 : (e > 127 ? 127 : e);
-    const float inv = exp2i(-e);
+    const float inv = exp2i(-e);                 // y * 2^-e is exact
 #pragma unroll
-    for (int q = 0; q < B / 8; ++q) w[q] = amax > 0.f ? e2m1x8_scaled(y + 8 * q, inv) : 0u;
+    for (int q = 0; q < B / 8; ++q) w[q] = amax > 0.f ? e2m1x8_times(y + 8 * q, inv) : 0u;
     return static_cast<uint32_t>(e + 127);
   } else if constexpr (FMT == kNv) {
-    const uint32_t sb = ue4m3_rne(__fdiv_rn(amax, den));
-    const float d = __fmul_rn(ue4m3_value(sb), gscale);
+    const uint32_t sb = nvfp4_scale_byte(amax, gscale, inv_den);
+    const float sbv = ue4m3_val(sb);
     const bool live = sb != 0u && amax > 0.f;
-    const float r = live ? __frcp_rn(d) : 0.f;
+    const float r = live ? __frcp_rn(__fmul_rn(sbv, gscale)) : 0.f;
 #pragma unroll
-    for (int q = 0; q < B / 8; ++q) w[q] = live ? e2m1x8_scaled(y + 8 * q, r) : 0u;
+    for (int q = 0; q < B / 8; ++q) w[q] = live ? nvfp4_codes8(y + 8 * q, r, sbv, gscale) : 0u;
     return sb;
   } else {
-    const float pre = fminf(__fdiv_rn(amax, 7.0f), 65504.0f);
-    const __half s16 = __float2half_rn(pre);
+    const __half s16 = int4_scale(amax);
     const float s = __half2float(s16);
     const float r = s > 0.f ? __frcp_rn(s) : 0.f;
 #pragma unroll
-    for (int q = 0; q < B / 8; ++q) {
-      float p[8];
-#pragma unroll
-      for (int k = 0; k < 8; k += 2) mul2(y[8 * q + k], y[8 * q + k + 1], r, p[k], p[k + 1]);
-      uint32_t acc = 0;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) acc |= int4_nibble(p[k]) << (4 * k);
-      w[q] = s > 0.f ? acc : 0u;
-    }
+    for (int q = 0; q < B / 8; ++q) w[q] = s > 0.f ? int4_codes8(y + 8 * q, r, s) : 0u;
     return static_cast<uint32_t>(__half_as_ushort(s16));
   }
 }
@@ -357,18 +288,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     return t + static_cast<int64_t>(jt) * B * B;
   };
-  float4 t_pre[2][kTPer];
-  if (kMma && threadIdx.x >= 64) {
-#pragma unroll
-    for (int c = 0; c < 2; ++c)
-#pragma unroll
-      for (int p = 0; p < kTPer; ++p) {
-        const int e0 = 4 * (static_cast<int>(threadIdx.x) - 64 + p * kEpiThreads);
-        const int j = (col_lo + c) * kBlocks + e0 / (B * B);
-        t_pre[c][p] = (c < n_cols && j < nb) ? __ldg(reinterpret_cast<const float4*>(t_block(j) + e0 % (B * B)))
-                                             : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-  }
   auto issue_load = [&](int n) {
     const int i = tile_lo + n, s = n % kStages;
     const int row0 = (i % n_row_tiles) * kTileRows, col0 = (i / n_row_tiles) * kTileCols;
@@ -390,10 +309,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tmap(&tmap_x);
-    // the ring starts empty: the first loads go out before the rest of the setup
-    for (int n = 0; n < kStages && n < n_mine; ++n) issue_load(n);
   }
   if (warp == 1 && kMma) tmem_alloc(tmem_slot, kTmemCols);
+  // Launched after another kernel with programmatic stream serialization, the set-up
+  // above overlaps that kernel's tail; no global input is read and no output written
+  // before the wait.
+  pdl_launch_dependents();
+  pdl_wait();
+  // the ring starts empty: the first loads go out before the rest of the set-up
+  if (threadIdx.x == 0)
+    for (int n = 0; n < kStages && n < n_mine; ++n) issue_load(n);
+  float4 t_pre[2][kTPer];
+  if (kMma && threadIdx.x >= 64) {
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+#pragma unroll
+      for (int p = 0; p < kTPer; ++p) {
+        const int e0 = 4 * (static_cast<int>(threadIdx.x) - 64 + p * kEpiThreads);
+        const int j = (col_lo + c) * kBlocks + e0 / (B * B);
+        t_pre[c][p] = (c < n_cols && j < nb) ? __ldg(reinterpret_cast<const float4*>(t_block(j) + e0 % (B * B)))
+                                             : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -475,7 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       gscale = nvfp4_dynamic_scale(__ldg(gs_amax));
       if (gs_out && blockIdx.x == 0 && et == 0) *gs_out = gscale;
     }
-    const float den = 6.0f * gscale;
+    const float inv_den = __frcp_rn(__fmul_rn(6.0f, gscale));   // 1 / (6 s_g), for the scale bracket
     const int n_atom_cols = (nb + 3) / 4;
 
     // Four fp32 values of T (group gi of a column: block jj, output row nrow,
@@ -620,7 +557,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         } else {
           uint32_t cw[B / 8];
-          const uint32_t sc = quantize_block<B, FMT>(y[u], gscale, den, cw);
+          const uint32_t sc = quantize_block<B, FMT>(y[u], gscale, inv_den, cw);
           if (blk_ok) {
             uint8_t* cp = codes + static_cast<int64_t>(r) * (d_in / 2) + static_cast<int64_t>(j) * (B / 2);
             if constexpr (B == 32) *reinterpret_cast<uint4*>(cp) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
@@ -721,9 +658,19 @@ int launch_tc(const void* x, int64_t rows, int64_t d_in, const float* t, const i
   if (sms <= 0) return WUSH_ERR_CUDA;
   const int grid = n_tiles < sms ? n_tiles : sms;
   const int64_t polls = g_wait_limit_override > 0 ? g_wait_limit_override : kDefaultPolls;
-  kern<<<grid, kThreads, kSmemBytes, st>>>(map, t, t_index, n_t, gscale, gs_amax, gs_out, codes, scales, ydbg,
-                                           static_cast<int>(rows),
-                                           static_cast<int>(d_in), n_row_tiles, n_tiles, polls);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, map, t, t_index, n_t, gscale, gs_amax, gs_out, codes, scales, ydbg,
+                         static_cast<int>(rows), static_cast<int>(d_in), n_row_tiles, n_tiles, polls) != cudaSuccess)
+    return WUSH_ERR_CUDA;
   return launch_status();
 }
 

@@ -363,22 +363,30 @@ def run_gpu(args, rank, world):
             gemm(r)
     stream.synchronize()
 
-    def capture(n_steps, start=0):
+    def capture(n_steps, start=0, events=True):
+        """A graph of n_steps steps; with ``events`` an event node sits between the
+        kernels (for per-kernel times), without them consecutive kernels are adjacent,
+        so each may start its set-up under the previous one's tail (programmatic
+        dependent launch)."""
         g = torch.cuda.CUDAGraph()
         evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(n_steps)]
         with torch.cuda.graph(g, stream=stream):
             for j in range(n_steps):
                 r = (start + j) % ROTATIONS
-                evs[j][0].record(stream)
+                if events:
+                    evs[j][0].record(stream)
                 tq(r)
-                evs[j][1].record(stream)
+                if events:
+                    evs[j][1].record(stream)
                 gemm(r)
-                evs[j][2].record(stream)
+                if events:
+                    evs[j][2].record(stream)
         return g, evs
 
-    g_main, ev_main = capture(STEPS_PER_GRAPH)
+    g_main, _ = capture(STEPS_PER_GRAPH, events=False)
     n_rem = args.steps % STEPS_PER_GRAPH
-    g_rem, ev_rem = capture(n_rem) if n_rem else (None, [])
+    g_rem, _ = capture(n_rem, events=False) if n_rem else (None, [])
+    g_ev, ev_main = capture(STEPS_PER_GRAPH)
     # a graph's event nodes refer to its Event objects: keep every (graph, events) pair alive
     g_one = [capture(1, r) for r in range(ROTATIONS)]
     if aq.wush_check_device_status(stream) != 0:
@@ -398,11 +406,14 @@ def run_gpu(args, rank, world):
         torch.cuda.synchronize()
         barrier(world)
         total_ms = e_start.elapsed_time(e_end)
-        # per-kernel device times from the event nodes of the last replay
-        evs = ev_main if steps >= STEPS_PER_GRAPH else ev_rem
-        tq_ms = [e[0].elapsed_time(e[1]) for e in evs]
-        gm_ms = [e[1].elapsed_time(e[2]) for e in evs]
-        return total_ms, tq_ms, gm_ms
+        return total_ms
+
+    def kernel_times():
+        """Per-kernel device times from the event nodes of one replay of the evented graph."""
+        with torch.cuda.stream(stream):
+            g_ev.replay()
+        stream.synchronize()
+        return ([e[0].elapsed_time(e[1]) for e in ev_main], [e[1].elapsed_time(e[2]) for e in ev_main])
 
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
@@ -412,9 +423,10 @@ def run_gpu(args, rank, world):
     for attempt in range(2):
         sampler = ClockSampler(dev.index)
         with sampler:
-            total_ms, tq_ms, gm_ms = timed(args.steps)
+            total_ms = timed(args.steps)
         if not sampler.rejected():
             break
+    tq_ms, gm_ms = kernel_times()
     status = aq.wush_check_device_status(stream)
     if status != 0:
         raise RuntimeError(f"device status {status}")
@@ -601,31 +613,38 @@ EXTRA_STEPS = 24          # steps of each other workload: one CUDA graph, replay
 
 def _graph_kernel_times(stream, launches, n_steps, reps=3):
     """Captures n_steps steps, each the callables ``launches`` (called with the step
-    index), into one CUDA graph with event nodes between them; replays it once warm,
-    then ``reps`` times timed.  Returns (us per step, [us per launch kind])."""
+    index), into two CUDA graphs: one with event nodes between the kernels (per-kernel
+    times), one without (the step time, kernels adjacent as in the headline step).
+    Each is replayed once warm, then timed.  Returns (us per step, [us per launch kind])."""
     import torch
-    g = torch.cuda.CUDAGraph()
+    g_plain, g_ev = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
     evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(launches) + 1)]
            for _ in range(n_steps)]
-    with torch.cuda.graph(g, stream=stream):
+    with torch.cuda.graph(g_plain, stream=stream):
+        for j in range(n_steps):
+            for fn in launches:
+                fn(j)
+    with torch.cuda.graph(g_ev, stream=stream):
         for j in range(n_steps):
             for i, fn in enumerate(launches):
                 evs[j][i].record(stream)
                 fn(j)
             evs[j][-1].record(stream)
     with torch.cuda.stream(stream):
-        g.replay()
+        g_plain.replay()
+        g_ev.replay()
     stream.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         e0.record(stream)
         for _ in range(reps):
-            g.replay()
+            g_plain.replay()
         e1.record(stream)
+        g_ev.replay()
     stream.synchronize()
     per_step = 1e3 * e0.elapsed_time(e1) / (reps * n_steps)
     per_kind = [1e3 * float(np.mean([e[i].elapsed_time(e[i + 1]) for e in evs])) for i in range(len(launches))]
-    del g
+    del g_plain, g_ev
     return per_step, per_kind
 
 

@@ -71,11 +71,13 @@ def magnitude(x_rows: np.ndarray, t: np.ndarray) -> np.ndarray:
     return T.block_magnitude(x_rows, t)
 
 
-def compare_transform_quant(x_rows, t, fmt, gs, codes_gpu, scales_gpu, y_gpu=None, rows_sel=None):
+def compare_transform_quant(x_rows, t, fmt, gs, codes_gpu, scales_gpu, y_gpu=None, rows_sel=None, strict=False):
     """Compare GPU outputs for rows ``rows_sel`` (all if None) of x_rows against the oracle.
 
     Returns a dict of counts; raises AssertionError on any non-exempt mismatch.
     codes_gpu/scales_gpu/y_gpu are already decoded to [rows, d_in] / [rows, nb] / [rows, d_in].
+    ``strict``: every code and scale must equal the oracle's (for inputs whose
+    transformed values are exact in fp32 on both sides, e.g. the identity transform).
     """
     x = np.asarray(x_rows, dtype=np.float64)
     if rows_sel is not None:
@@ -123,4 +125,6 @@ def compare_transform_quant(x_rows, t, fmt, gs, codes_gpu, scales_gpu, y_gpu=Non
     WINDOW_LOG.append(dict(out, fmt=fmt, rows=rows, d_in=d_in,
                            test=os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0]))
     assert out["exempt"] <= max(MAX_EXEMPT_FRACTION * out["elements"], 1), out
+    if strict:
+        assert out["exempt"] == 0 and out["scale_exempt"] == 0, out
     return out

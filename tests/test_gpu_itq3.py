@@ -19,7 +19,7 @@ def pack_codes(c):
 
 
 @pytest.mark.parametrize("shape", [(256, 1024), (4096, 4096)])
-@pytest.mark.parametrize("tokens", [1, 3, 4, 16])
+@pytest.mark.parametrize("tokens", [1, 2, 3, 4, 16])
 @pytest.mark.parametrize("mode", [0, 1])
 def test_itq3_gemv(lib, shape, tokens, mode):
     d_out, d_in = shape
@@ -48,3 +48,22 @@ def test_itq3_library_quantiser_feeds_gemv(lib):
                           torch.from_numpy(x.astype(np.float16)).cuda(), 512, 0, y)
     err = np.linalg.norm(y.cpu().numpy() - want) / np.linalg.norm(want)
     assert err <= 1e-5
+
+
+@pytest.mark.parametrize("tokens, d_in", [(1, 40960), (2, 10240), (2, 12288), (1, 43008)])
+def test_itq3_mode1_rotation_inside_or_outside_the_gemv(lib, tokens, d_in):
+    # one or two tokens rotate x inside the GEMV kernel while a token chunk of x
+    # fits shared memory (1 x 40960 and 2 x 10240 are the largest such); beyond
+    # that the call rotates into the workspace first.  Both forms against the oracle.
+    d_out = 64
+    w = synth.itq3_weights(d_out, d_in)
+    x = synth.itq3_activations(tokens, d_in).astype(np.float16)
+    c, s = I.quantize(w)
+    want = I.gemv(c, s, x.astype(np.float64))
+    y = torch.full((tokens, d_out), float("nan"), dtype=torch.float32, device="cuda")
+    ws = torch.empty((tokens, d_in), dtype=torch.float32, device="cuda")
+    lib.itq3_dequant_gemv(torch.from_numpy(pack_codes(c)).cuda(), torch.from_numpy(s).cuda(),
+                          torch.from_numpy(x).cuda(), d_out, 1, y, ws)
+    assert lib.wush_check_device_status() == 0
+    got = y.cpu().numpy().astype(np.float64)
+    assert np.linalg.norm(got - want) / np.linalg.norm(want) <= 1e-5

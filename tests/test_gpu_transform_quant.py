@@ -310,3 +310,60 @@ def test_indexed_transform_rejects_non_dense_kinds(lib):
     for kind in ("identity", "hadamard"):
         with pytest.raises(lib.WushError):
             lib.wush_transform_quant_indexed(xt, t, idx, kind, "mxfp4", codes, scales)
+
+
+def _near_tie_rows(fmt, rng, rows=64):
+    """fp32 rows whose quotients sit on, and one fp32 ulp either side of, element
+    and scale rounding boundaries (the cases where a reciprocal-multiply order would
+    round differently from the exact quotient); with the identity transform both
+    sides see the same fp32 values, so every code and scale must match exactly."""
+    from oracle import formats as F
+    b = P.Q.BLOCK[fmt]
+    out = np.zeros((rows, 4 * b), np.float32)
+    gs = np.float32(0.0123)
+    for r in range(rows):
+        for j in range(4):
+            if fmt == "nvfp4":
+                sbv = float(rng.choice(F.E4M3_GRID[40:110]))
+                d = sbv * float(gs)
+                mids = (F.E2M1_GRID[:-1] + F.E2M1_GRID[1:]) / 2
+                blk = [np.float32(6.0 * d)]
+            else:
+                s = float(np.float16(rng.uniform(1e-3, 50)))
+                d = s
+                mids = np.arange(7) + 0.5
+                blk = [np.float32(7.0 * d)]
+            while len(blk) < b:
+                v = np.float32(float(rng.choice(mids)) * d * (1 if rng.random() < 0.5 else -1))
+                k = rng.integers(0, 3)
+                v = v if k == 0 else np.nextafter(v, np.float32(np.inf if k == 1 else -np.inf))
+                blk.append(v)
+            out[r, j * b:(j + 1) * b] = blk
+    return out, float(gs)
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4"])
+def test_exact_decisions_next_to_ties_fp32(lib, fmt):
+    # one-row-per-thread kernel (fp32 input), identity transform: bit-exact against
+    # the oracle's exact-quotient rule with no boundary window
+    rng = np.random.default_rng(31)
+    x, gs = _near_tie_rows(fmt, rng)
+    t = T.identity_blocks(x.shape[1], P.Q.BLOCK[fmt]).astype(np.float32)
+    c, s, y = run_gpu_t(lib, _as_input(x, False), t, "identity", fmt, gs if fmt == "nvfp4" else 0.0)
+    P.compare_transform_quant(x, t, fmt, gs if fmt == "nvfp4" else None, c, s, y, strict=True)
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4", "int4"])
+@pytest.mark.parametrize("kind", ["identity", "hadamard"])
+def test_exact_decisions_structured_bf16(lib, fmt, kind):
+    # tensor-core kernel, bf16 input with 8-bit significands and a per-tensor scale
+    # derived from a bf16 amax (amax / 2688 = amax / (2^7 * 21)): many quotients fall
+    # on or within an fp32 ulp of a boundary.  The identity transform is exact in
+    # fp32 on both sides, so its codes and scales must match the oracle exactly;
+    # Hadamard's fp32 butterflies may round, so it gets the boundary window.
+    w = synth.WORKLOADS[FMT_WORKLOAD[fmt]]
+    x = synth.activations(w, tokens=256)[:, :1024]
+    t = (T.identity_blocks if kind == "identity" else T.hadamard_blocks)(1024, P.Q.BLOCK[fmt]).astype(np.float32)
+    gs = _global_scale(x, t, fmt)
+    c, s, y = run_gpu_t(lib, _as_input(x, True), t, kind, fmt, gs)
+    P.compare_transform_quant(x, t, fmt, gs if fmt == "nvfp4" else None, c, s, y, strict=kind == "identity")
