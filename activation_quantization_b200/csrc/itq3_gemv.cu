@@ -17,9 +17,6 @@
 //   symmetric and orthogonal, so w_hat . x = ((c - 3.5) s) . (H x / 16).  A
 //   first kernel rotates each 256-block of x once into the caller's fp32
 //   workspace; the GEMV then uses the levels (c - 3.5) s with no transform.
-//   For one or two tokens the rotation runs inside the GEMV instead (mode 2
-//   below): each CTA rotates the x blocks into shared memory while its first
-//   code words are in flight, so the call is one launch.
 #include <cuda_fp16.h>
 
 #include <mutex>
@@ -66,8 +63,14 @@ __device__ __forceinline__ void decode_levels(uint32_t word, int lane, float s, 
   const uint32_t hi = __shfl_sync(0xffffffffu, word, w0 + 1 < 24 ? w0 + 1 : 23);
   const uint32_t bits = __funnelshift_r(lo, hi, bit & 31);
   const float m = -3.5f * s;
+  // code c as a float without an integer-to-float conversion: the bits 2^23 + c
+  // minus 2^23 (both exact); (c - 3.5) s then needs at most 15 significant bits,
+  // so the FMA is exact too
 #pragma unroll
-  for (int i = 0; i < 8; ++i) v[i] = fmaf(static_cast<float>((bits >> (3 * i)) & 7u), s, m);
+  for (int i = 0; i < 8; ++i) {
+    const float c = __fsub_rn(__uint_as_float(0x4B000000u | ((bits >> (3 * i)) & 7u)), 8388608.0f);
+    v[i] = fmaf(c, s, m);
+  }
 }
 
 // In-place unnormalised 256-point FWHT of a warp-distributed vector whose index
@@ -105,8 +108,7 @@ __device__ __forceinline__ void warp_fwht256(float (&v)[8], int lane) {
 // so the block loop waits on shared-memory latency rather than L2.
 // MODE 0: x is fp16 and the inverse FWHT runs on every weight block (the
 // article's fused design).  MODE 1: x is the fp32 rotated activation (H x / 16)
-// and the weights are used as their levels (c - 3.5) s.  MODE 2: as MODE 1, but x
-// is fp16 and the CTA rotates it into shared memory itself (STAGE only).
+// and the weights are used as their levels (c - 3.5) s.
 template <int R, int W, int TC, int MODE, bool STAGE>
 __global__ void __launch_bounds__(kWarps * 32) itq3_gemv_kernel(const uint32_t* __restrict__ codes,
                                                                 const __half* __restrict__ scales,
@@ -117,32 +119,10 @@ __global__ void __launch_bounds__(kWarps * 32) itq3_gemv_kernel(const uint32_t* 
   const int row0 = (blockIdx.x * kWarps + (threadIdx.x >> 5)) * R;
   if (!STAGE && row0 >= d_out) return;             // with STAGE every warp joins the barriers
   const int nb = d_in / 256;
-  static_assert(MODE != 2 || STAGE, "mode 2 rotates x into shared memory");
   // Copies tokens tc0 .. tc0 + TC - 1 of x into shared memory as fp32 (zeros past
-  // the last token); every warp of the CTA takes part.  MODE 2 stores H x / 16 of
-  // every 256-block instead, one warp per (token, block).
+  // the last token); every warp of the CTA takes part.
   auto stage_x = [&](int tc0) {
     __syncthreads();                               // the previous chunk is no longer read
-    if constexpr (MODE == 2) {
-      for (int item = threadIdx.x >> 5; item < TC * nb; item += kWarps) {
-        const int tt = item / nb, blk = item - tt * nb, t = tc0 + tt;
-        float v[8];
-        if (t < tokens) {
-          const __half* xr = static_cast<const __half*>(xin) + static_cast<int64_t>(t) * d_in + blk * 256 + lane;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) v[i] = __half2float(xr[32 * i]);
-          warp_fwht256(v, lane);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) v[i] = 0.f;
-        }
-        float* out = sx + tt * d_in + blk * 256 + lane;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) out[32 * i] = v[i] * 0.0625f;
-      }
-      __syncthreads();
-      return;
-    }
     for (int i = threadIdx.x * 4; i < TC * d_in; i += kWarps * 32 * 4) {
       const int tt = i / d_in, e = i - tt * d_in, t = tc0 + tt;
       float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -153,7 +133,7 @@ __global__ void __launch_bounds__(kWarps * 32) itq3_gemv_kernel(const uint32_t* 
           const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&h.x));
           const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&h.y));
           v = make_float4(a.x, a.y, b.x, b.y);
-        } else if constexpr (MODE == 1) {
+        } else {
           v = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(xin) + xo));
         }
       }
@@ -277,10 +257,8 @@ int launch_one(const uint32_t* c32, const __half* sc, const void* x, int t, int 
   const size_t smem = static_cast<size_t>(TC) * k * 4;
   // a single token's x is read through L1 well enough; staging pays off once a
   // chunk of several tokens is reused by every row of the CTA
-  // (mode 2 always stages: the caller checks that the chunk fits)
-  const bool stage = MODE == 2 || (TC > 1 && smem <= 160 * 1024);
-  auto kern = stage ? itq3_gemv_kernel<R, W, TC, MODE, true>
-                    : itq3_gemv_kernel<R, W, TC, MODE, MODE == 2>;
+  const bool stage = TC > 1 && smem <= 160 * 1024;
+  auto kern = stage ? itq3_gemv_kernel<R, W, TC, MODE, true> : itq3_gemv_kernel<R, W, TC, MODE, false>;
   if (stage) {
     static std::atomic<uint64_t> attr_done{0};     // the limit is raised to the 160 KB cap once
     if (smem > 48 * 1024 && set_smem_once(kern, 160 * 1024, attr_done) != WUSH_OK) return WUSH_ERR_CUDA;
@@ -310,15 +288,6 @@ int launch_gemv(const uint32_t* c32, const __half* sc, const void* x, int t, int
   if (t == 1) return launch_one<1, 16, 1, MODE>(c32, sc, x, t, n, k, y, st);
   if (t <= 4) return launch_one<4, 4, 4, MODE>(c32, sc, x, t, n, k, y, st);
   return launch_one<4, 4, 8, MODE>(c32, sc, x, t, n, k, y, st);
-}
-
-// Mode 1 for one or two tokens whose x fits shared memory: one launch that rotates
-// x inside each CTA (mode 2 of the kernel); WUSH_ERR_UNSUPPORTED otherwise.
-int gemv_rotating(const uint32_t* c32, const __half* sc, const __half* x, int t, int n, int k, float* y,
-                  cudaStream_t st) {
-  if (t == 1 && k <= 40960) return launch_one<1, 16, 1, 2>(c32, sc, x, t, n, k, y, st);
-  if (t == 2 && k <= 10240) return launch_one<4, 4, 4, 2>(c32, sc, x, t, n, k, y, st);
-  return WUSH_ERR_UNSUPPORTED;
 }
 
 // Mode 1 after the rotation: the tensor-core kernel (itq3_tc.cu) where the shape
@@ -353,10 +322,6 @@ extern "C" int itq3_dequant_gemv(const uint8_t* codes, const void* scales_fp16, 
   const auto* xh = static_cast<const __half*>(x_fp16);
   const int t = static_cast<int>(tokens), n = static_cast<int>(d_out), k = static_cast<int>(d_in);
   if (mode == 0) return launch_gemv<0>(c32, sc, xh, t, n, k, y, st);
-  if (t <= 2) {
-    const int r = gemv_rotating(c32, sc, xh, t, n, k, y, st);
-    if (r != WUSH_ERR_UNSUPPORTED) return r;
-  }
   const dim3 block(kWarps * 32);
   const int items = t * (k / 256);
   itq3_rotate_x_kernel<<<(items + kWarps - 1) / kWarps, block, 0, st>>>(xh, t, k, workspace);

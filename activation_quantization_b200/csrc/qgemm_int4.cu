@@ -343,7 +343,7 @@ static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 // two 256-row blocks of B while the group's rows of A stay in L2 (their loads are
 // marked evict-last, y's stores evict-first) for the whole sweep over N: each
 // group reads its rows of A once and B once.  The host sizes the group so its rows
-// of A fill at most about two thirds of L2 (all of A when it fits).
+// of A fill at most about a third of L2.
 __device__ __forceinline__ void pair_tile_coords(int pt, int mt, int nt, int group, int& pm, int& pn) {
   const int g = pt / (group * nt);
   const int rows = min(group, mt - g * group);
@@ -597,11 +597,13 @@ int launch_hgemm_pair(const __half* a, const __half* b, int64_t M, int64_t N, in
     return WUSH_ERR_CUDA;
   const int64_t n_ptiles = (M / 256) * (N / 256);
   const int pairs = static_cast<int>(n_ptiles < sms / 2 ? n_ptiles : sms / 2);
-  // row blocks of A per group: as many 256-row blocks as fit in about two thirds of
-  // L2 (fp16, K wide), at least 8
+  // row blocks of A per group: as many 256-row blocks as fit in a third of L2 (fp16,
+  // K wide), at least 8.  (Measured at 8192 x 17408 x 5120: a group holding all of A,
+  // 84 MB, did not stay in L2 and read 2.4 GB from DRAM per launch; 16 row blocks,
+  // 42 MB, ran fastest.)
   int l2 = 0;
   if (cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess || l2 <= 0) return WUSH_ERR_CUDA;
-  const int64_t fit = (static_cast<int64_t>(l2) * 2 / 3) / (256 * K * 2);
+  const int64_t fit = (static_cast<int64_t>(l2) / 3) / (256 * K * 2);
   const int group = static_cast<int>(fit < 8 ? 8 : (fit > M / 256 ? M / 256 : fit));
   const int64_t polls = g_wait_limit_override > 0 ? g_wait_limit_override : kDefaultPolls;
   cudaLaunchConfig_t cfg = {};

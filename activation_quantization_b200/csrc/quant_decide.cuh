@@ -127,12 +127,16 @@ __device__ __forceinline__ __half int4_scale(float amax) {
   return amax > m7 ? hi : (amax < m7 ? lo : ((__half_as_ushort(lo) & 1u) ? hi : lo));
 }
 
-// clamp(RNE(v), -7, 7) as a two's-complement nibble, without a float-to-integer
-// conversion: adding 1.5 * 2^23 rounds a value of magnitude below 2^22 to an
-// integer (round to nearest even, the ulp there being 1) in the low mantissa bits.
-__device__ __forceinline__ uint32_t int4_nibble_rn(float v) {
-  const float c = fminf(fmaxf(v, -7.0f), 7.0f);
-  return __float_as_uint(__fadd_rn(c, 12582912.0f)) & 15u;
+// RNE(v) of |v| < 2^22 without a float-to-integer conversion: adding 1.5 * 2^23
+// rounds to an integer (the ulp there is 1) held in the low mantissa bits, whose
+// low four bits are the two's-complement nibble of the result.
+__device__ __forceinline__ uint32_t rne_bits(float v) { return __float_as_uint(__fadd_rn(v, 12582912.0f)); }
+
+// Insert the low four bits of src into w at bit position pos.
+__device__ __forceinline__ uint32_t put_nibble(uint32_t w, uint32_t src, uint32_t pos) {
+  uint32_t out;
+  asm("bfi.b32 %0, %1, %2, %3, 4;" : "=r"(out) : "r"(src), "r"(w), "r"(pos));
+  return out;
 }
 
 __device__ __forceinline__ int int4_from_nibble(uint32_t n) {
@@ -141,16 +145,25 @@ __device__ __forceinline__ int int4_from_nibble(uint32_t n) {
 
 // Eight INT4 codes (two's-complement nibbles) of v[0..7] with scale s > 0 and
 // r = fp32(1 / s).  Exact: equal to clamp(RNE(v / s), -7, 7).
+// When s is a normal fp16 below 65504 (s = fp16_RNE(amax / 7) within 2^-11), no
+// |v / s| exceeds 7 (1 + 2^-10) < 7.5, so no value needs the clamp.
 __device__ __forceinline__ uint32_t int4_codes8(const float* v, float r, float s) {
   const float ra = __fmul_rn(r, kBracketLo), rb = __fmul_rn(r, kBracketHi);
+  const bool in_range = s >= 6.103515625e-05f && s < 65504.0f;
   uint32_t wa = 0, wb = 0;
 #pragma unroll
   for (int i = 0; i < 8; i += 2) {
     float a0, a1, b0, b1;
     mul2_rn(v[i], v[i + 1], ra, a0, a1);
     mul2_rn(v[i], v[i + 1], rb, b0, b1);
-    wa |= (int4_nibble_rn(a0) << (4 * i)) | (int4_nibble_rn(a1) << (4 * i + 4));
-    wb |= (int4_nibble_rn(b0) << (4 * i)) | (int4_nibble_rn(b1) << (4 * i + 4));
+    if (!in_range) {
+      a0 = fminf(fmaxf(a0, -7.0f), 7.0f);
+      a1 = fminf(fmaxf(a1, -7.0f), 7.0f);
+      b0 = fminf(fmaxf(b0, -7.0f), 7.0f);
+      b1 = fminf(fmaxf(b1, -7.0f), 7.0f);
+    }
+    wa = put_nibble(put_nibble(wa, rne_bits(a0), 4 * i), rne_bits(a1), 4 * i + 4);
+    wb = put_nibble(put_nibble(wb, rne_bits(b0), 4 * i), rne_bits(b1), 4 * i + 4);
   }
   if (wa == wb) return wa;
   uint32_t w = wa;
@@ -161,7 +174,7 @@ __device__ __forceinline__ uint32_t int4_codes8(const float* v, float r, float s
     const int lo = min(qa, qb), hi = max(qa, qb);
     const float p = (static_cast<float>(lo) + 0.5f) * s;     // at most 15 significant bits: exact
     const int q = v[i] > p ? hi : (v[i] < p ? lo : ((lo & 1) ? hi : lo));
-    w = (w & ~(15u << (4 * i))) | ((static_cast<uint32_t>(q) & 15u) << (4 * i));
+    w = put_nibble(w, static_cast<uint32_t>(q), 4 * i);
   }
   return w;
 }

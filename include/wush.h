@@ -386,9 +386,6 @@ int itq3_quantize_weights(const uint16_t* w_fp16, int64_t d_out, int64_t d_in, u
  *         c - 3.5 are exact fp16 MMA operands and each block of rotated x is
  *         split exactly enough (hi + lo fp16 after a power-of-two scale) that
  *         only the fp32 accumulation rounds; otherwise CUDA cores run it.
- *         For one token (d_in <= 40960) or two (d_in <= 10240) the rotation
- *         runs inside the GEMV kernel, one launch per call, and ``workspace``
- *         is not touched.
  * workspace may be NULL for mode 0.  Requirements: 1 <= tokens <= 16,
  * d_in % 256 == 0, d_out % 8 == 0, codes, scales, x_fp16 and workspace 16-byte
  * aligned; WUSH_ERR_INVALID_ARG otherwise, before any launch. */
