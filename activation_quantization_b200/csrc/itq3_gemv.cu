@@ -42,9 +42,17 @@ namespace {
 
 constexpr int kWarps = 8;
 
-// Programmatic dependent launch: the rotation kernel lets the GEMV that follows it
-// start early, and the GEMV waits for the rotation's results only where it first
-// reads them (a no-op when it was launched without the attribute).
+// Programmatic dependent launch, so that the launch latency of each kernel hides
+// under the previous one:
+//  * the rotation kernel waits for the kernel before it before it reads x, and only
+//    then lets the GEMV that follows it start;
+//  * the GEMV issues its code-word loads at once (no kernel still running can be
+//    writing them: the rotation has passed its wait), and waits for the rotation's
+//    results only where it first reads them;
+//  * every GEMV lets the next call's first kernel start early (mode 1 at entry,
+//    mode 0 once its work is done); that kernel waits for the GEMV to finish
+//    before it touches memory.
+// Both instructions are no-ops in a kernel launched without the attribute.
 __device__ __forceinline__ void allow_dependent_launch() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
@@ -115,6 +123,13 @@ __global__ void __launch_bounds__(kWarps * 32) itq3_gemv_kernel(const uint32_t* 
                                                                 const void* __restrict__ xin, int tokens,
                                                                 int d_out, int d_in, float* __restrict__ y) {
   extern __shared__ __align__(16) float sx[];      // STAGE: [TC][d_in] fp32
+  // Mode 1 (memory-bound) lets the next kernel launch at once.  Mode 0 is bound by
+  // its arithmetic, and a next kernel whose CTAs wait beside it on the same SMs
+  // measured up to 1.6x slower, so it lets the next kernel launch only once its
+  // own work is done; as the call's only kernel it reads nothing global before the
+  // kernel launched before it has finished.
+  if constexpr (MODE == 1) allow_dependent_launch();
+  if constexpr (MODE == 0) wait_for_prerequisite_grid();
   const int lane = threadIdx.x & 31;
   const int row0 = (blockIdx.x * kWarps + (threadIdx.x >> 5)) * R;
   if (!STAGE && row0 >= d_out) return;             // with STAGE every warp joins the barriers
@@ -217,6 +232,9 @@ __global__ void __launch_bounds__(kWarps * 32) itq3_gemv_kernel(const uint32_t* 
         }
       }
     }
+    if constexpr (MODE == 0) {
+      if (tc0 + TC >= tokens) allow_dependent_launch();
+    }
 #pragma unroll
     for (int rr = 0; rr < R; ++rr)
 #pragma unroll
@@ -233,6 +251,7 @@ __global__ void __launch_bounds__(kWarps * 32) itq3_gemv_kernel(const uint32_t* 
 // x_rot[t, blk*256 + e] = (H_256 x[t, blk*256 : +256])[e] / 16; one warp per (t, blk).
 __global__ void __launch_bounds__(kWarps * 32) itq3_rotate_x_kernel(const __half* __restrict__ x, int tokens,
                                                                      int d_in, float* __restrict__ x_rot) {
+  wait_for_prerequisite_grid();
   allow_dependent_launch();
   const int lane = threadIdx.x & 31;
   const int item = blockIdx.x * kWarps + (threadIdx.x >> 5);
@@ -247,6 +266,23 @@ __global__ void __launch_bounds__(kWarps * 32) itq3_rotate_x_kernel(const __half
   float* out = x_rot + static_cast<int64_t>(t) * d_in + blk * 256 + lane;
 #pragma unroll
   for (int i = 0; i < 8; ++i) out[32 * i] = v[i] * 0.0625f;
+}
+
+// Rotation of every 256-block of x into x_rot, launched with programmatic stream
+// serialization (see above).
+int launch_rotation(const __half* x, int t, int k, float* x_rot, cudaStream_t st) {
+  const int items = t * (k / 256);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((items + kWarps - 1) / kWarps));
+  cfg.blockDim = dim3(kWarps * 32);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, itq3_rotate_x_kernel, x, t, k, x_rot) != cudaSuccess) return WUSH_ERR_CUDA;
+  return launch_status();
 }
 
 // Rows per warp, blocks per load window and tokens per pass by token count: one
@@ -272,7 +308,7 @@ int launch_one(const uint32_t* c32, const __half* sc, const void* x, int t, int 
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = MODE == 1 ? 1 : 0;             // mode 1 follows the rotation kernel
+  cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, kern, c32, sc, x, t, n, k, y) != cudaSuccess) return WUSH_ERR_CUDA;
   return launch_status();
 }
@@ -322,10 +358,7 @@ extern "C" int itq3_dequant_gemv(const uint8_t* codes, const void* scales_fp16, 
   const auto* xh = static_cast<const __half*>(x_fp16);
   const int t = static_cast<int>(tokens), n = static_cast<int>(d_out), k = static_cast<int>(d_in);
   if (mode == 0) return launch_gemv<0>(c32, sc, xh, t, n, k, y, st);
-  const dim3 block(kWarps * 32);
-  const int items = t * (k / 256);
-  itq3_rotate_x_kernel<<<(items + kWarps - 1) / kWarps, block, 0, st>>>(xh, t, k, workspace);
-  if (launch_status() != WUSH_OK) return WUSH_ERR_CUDA;
+  if (launch_rotation(xh, t, k, workspace, st) != WUSH_OK) return WUSH_ERR_CUDA;
   return gemv_rotated(codes, scales_fp16, workspace, t, n, k, y, st);
 }
 
@@ -429,9 +462,6 @@ extern "C" int itq3_dequant_gemv_noalloc(const uint8_t* codes, const void* scale
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const auto* xh = static_cast<const __half*>(x_fp16);
   const int t = static_cast<int>(tokens), n = static_cast<int>(d_out), k = static_cast<int>(d_in);
-  const dim3 block(kWarps * 32);
-  const int items = t * (k / 256);
-  itq3_rotate_x_kernel<<<(items + kWarps - 1) / kWarps, block, 0, s>>>(xh, t, k, scratch);
-  if (launch_status() != WUSH_OK) return WUSH_ERR_CUDA;
+  if (launch_rotation(xh, t, k, scratch, s) != WUSH_OK) return WUSH_ERR_CUDA;
   return gemv_rotated(codes, scales_fp16, scratch, t, n, k, y, s);
 }

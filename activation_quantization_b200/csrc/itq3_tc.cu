@@ -146,6 +146,9 @@ __device__ __forceinline__ void tmem_ld_wait_regs(uint32_t (&r)[N]) {
 __device__ __forceinline__ void wait_for_prerequisite_grid() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
+__device__ __forceinline__ void allow_dependent_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 __device__ __forceinline__ void st_shared_cluster_f32(uint32_t addr, float v) {
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
@@ -184,6 +187,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                    float* __restrict__ y, int64_t max_polls) {
   using C_ = Cfg<NT>;
   constexpr int kSlots = C_::kSlots;
+  // the next call's first kernel may start early; it waits for this one to finish
+  // before it touches memory
+  allow_dependent_launch();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* bst = smem;                                              // two B stages

@@ -86,10 +86,10 @@ def max_over_ranks(value: float, world: int) -> float:
 
 
 def source_sha(source_file: str) -> str:
-    """Hash of a kernel's source file together with the device headers it includes."""
+    """Hash of a kernel's source file together with the library's device headers."""
     csrc = os.path.dirname(source_file)
     h = hashlib.sha1()
-    for f in [source_file] + [os.path.join(csrc, n) for n in ("sm100.cuh", "common.cuh")]:
+    for f in [source_file] + sorted(os.path.join(csrc, n) for n in os.listdir(csrc) if n.endswith(".cuh")):
         h.update(open(f, "rb").read())
     return h.hexdigest()[:12]
 
@@ -447,6 +447,39 @@ def run_gpu(args, rank, world):
     torch.cuda.synchronize()
     tq_burst_us = 1e3 * b0.elapsed_time(b1) / (8 * STEPS_PER_GRAPH)
 
+    # Batches pipelined over two streams: the transform of batch j runs on a second
+    # stream as soon as its output buffer is free again (the GEMM of batch j - 3 has
+    # read it), so it overlaps the GEMM of batch j - 1, its tail and its y write-back.
+    # Same work per step; reported beside the serial step, not as the headline.
+    pipe_us = None
+    if not dynamic:
+        side = torch.cuda.Stream(device=dev)
+        ev_tq = [torch.cuda.Event() for _ in range(STEPS_PER_GRAPH)]
+        ev_gm = [torch.cuda.Event() for _ in range(STEPS_PER_GRAPH)]
+        g_pipe = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_pipe, stream=stream):
+            side.wait_stream(stream)
+            for j in range(STEPS_PER_GRAPH):
+                r = j % ROTATIONS
+                if j >= ROTATIONS:
+                    side.wait_event(ev_gm[j - ROTATIONS])
+                quant(xs[r], t_x, t_xs if groups else None, fmt, acodes[r][0], acodes[r][1], gx, side)
+                ev_tq[j].record(side)
+                stream.wait_event(ev_tq[j])
+                gemm(r)
+                ev_gm[j].record(stream)
+            stream.wait_stream(side)
+        with torch.cuda.stream(stream):
+            g_pipe.replay()
+            p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            p0.record(stream)
+            for _ in range(8):
+                g_pipe.replay()
+            p1.record(stream)
+        torch.cuda.synchronize()
+        pipe_us = 1e3 * p0.elapsed_time(p1) / (8 * STEPS_PER_GRAPH)
+        del g_pipe
+
     total_ms = max_over_ranks(total_ms, world)
 
     flops_step = 2.0 * M * N * K
@@ -534,6 +567,10 @@ def run_gpu(args, rank, world):
                                 "burst_us": tq_burst_us,
                                 "burst_frac_of_hbm": tq_bytes / (tq_burst_us * 1e-6) / 1e9 / peaks["hbm_gbs"]},
             "qgemm": {"us": gm_us, "TFLOP_s": gemm_tflops, "frac_of_peak": gemm_tflops / fp4_peak},
+            "pipelined_step": None if pipe_us is None else {
+                "us": pipe_us, "TFLOP_s": flops_step / (pipe_us * 1e-6) / 1e12,
+                "how": "transform of batch j on a second stream, overlapping the GEMM of batch j - 1 "
+                       f"({ROTATIONS} rotating code buffers); graph bursts of {STEPS_PER_GRAPH} steps"},
             "roofline": {"kernel": gemm_kernel, "bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak,
                          "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak, "traffic": traffic,
                          "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']:.1f} TFLOP/s, {gemm_peak_src}"},
