@@ -479,10 +479,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     float run_max = 0.f;                        // kAm: this thread's max |y|
+    // tile i = (column col, row tile row_tile), advanced incrementally: no division
+    // by the runtime row-tile count inside the loop
+    int col = col_lo, row_tile = tile_lo - col_lo * n_row_tiles;
     for (int i = tile_lo; i < tile_hi; ++i) {
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
       const int n = i - tile_lo, s = n % kStages;
-      const int row0 = (i % n_row_tiles) * kTileRows, col0 = (i / n_row_tiles) * kTileCols;
+      const int row0 = row_tile * kTileRows, col0 = col * kTileCols;
       const int r = row0 + rloc;
       const bool row_ok = r < rows;
       const int p = n % kSets;
@@ -578,10 +581,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         // commit covers every MMA issued before it: after the last tile of column k,
         // no MMA reads that column's T buffer any more, so it refills it with k + 2.
         if (g == kEpiGroups - 1) {
-          const int k = i / n_row_tiles - col_lo;
-          const bool last_of_col = (i + 1 == tile_hi) || ((i + 1) / n_row_tiles != i / n_row_tiles);
+          const int k = col - col_lo;
+          const bool last_of_col = (i + 1 == tile_hi) || (row_tile + 1 == n_row_tiles);
           if (last_of_col && k + 2 < n_cols) convert_t(k + 2, et - g * 128, 128, 2 + g);
         }
+      }
+      if (++row_tile == n_row_tiles) {
+        row_tile = 0;
+        ++col;
       }
     }
     if constexpr (FMT == kAm) {
