@@ -110,6 +110,27 @@ def test_int4_gemm_two_pass_random(lib, mnk):
     assert diff <= 1e-5, diff
 
 
+def test_int4_two_pass_random_full_size_sampled(lib):
+    # the int4 workload's launch (8192 x 17408 x 5120) on seeded random codes: the pair
+    # GEMM walks its tiles in groups of row blocks sized to L2, so every group, every
+    # tile of a column and the last, partial group are reached; the oracle checks 64
+    # sampled rows (the first and the last included) against all 17408 columns
+    m, n, k = 8192, 17408, 5120
+    a_c, a_s, a_dq = _random_int4(51, m, k)
+    b_c, b_s, b_dq = _random_int4(52, n, k)
+    dev = "cuda"
+    args = [torch.from_numpy(v).to(dev) for v in (a_c, a_s, b_c, b_s)]
+    y = torch.full((m, n), float("nan"), dtype=torch.float32, device=dev)
+    _run_ws(lib, *args, m, n, k, y)
+    assert lib.wush_check_device_status() == 0
+    rows = np.sort(np.random.default_rng(53).choice(m, 64, replace=False))
+    rows[0], rows[-1] = 0, m - 1
+    got = y[torch.from_numpy(rows).to(dev)].cpu().numpy().astype(np.float64)
+    assert np.isfinite(got).all()
+    err = _rel(got, G.gemm_dequantized(a_dq[rows], b_dq))
+    assert err <= 5e-4, err
+
+
 @pytest.mark.parametrize("m", [2048, 8192])
 def test_int4_two_pass_end_to_end_sampled(lib, m):
     # the int4 workload at 2048 and 8192 tokens (the bench's launches) through the
