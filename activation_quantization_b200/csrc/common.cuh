@@ -43,9 +43,6 @@ extern int g_gemm_variant;
 // [tokens, d_in]); WUSH_ERR_UNSUPPORTED, before any launch, for shapes it does not take.
 int itq3_gemv_tc(const uint8_t* codes, const void* scales_fp16, const float* x_rot, int tokens, int d_out, int d_in,
                  float* y, cudaStream_t st);
-// The token count and shape for which itq3_gemv_tc launches (it may still decline a
-// shape whose blocks exceed its shared memory).
-bool itq3_tc_shape_ok(int tokens, int d_out, int d_in);
 
 // ITQ3 mode-1 kernel choice (see wush_debug_set_itq3_variant).
 extern int g_itq3_variant;

@@ -44,13 +44,11 @@ constexpr int kWarps = 8;
 
 // Programmatic dependent launch, so that the launch latency of each kernel hides
 // under the previous one:
-//  * the rotation kernel waits for the kernel before it before it reads x.  Before
-//    the CUDA-core GEMV it lets the GEMV start only after that wait, so the GEMV may
-//    issue its code-word loads at once (no kernel still running can be writing
-//    them) and waits for the rotation's results only where it first reads them.
-//    Before the tensor-core kernel it lets the next kernel start at entry, and that
-//    kernel waits before it reads anything (measured faster at 3-16 tokens:
-//    10.8 -> 9.1 us at 4 tokens; slower for the CUDA-core GEMV at 1-2 tokens);
+//  * the rotation kernel waits for the kernel before it before it reads x, and only
+//    then lets the GEMV that follows it start;
+//  * the GEMV issues its code-word loads at once (no kernel still running can be
+//    writing them: the rotation has passed its wait), and waits for the rotation's
+//    results only where it first reads them;
 //  * every GEMV lets the next call's first kernel start early (mode 1 at entry,
 //    mode 0 once its work is done); that kernel waits for the GEMV to finish
 //    before it touches memory.
@@ -123,8 +121,7 @@ template <int R, int W, int TC, int MODE, bool STAGE>
 __global__ void __launch_bounds__(kWarps * 32) itq3_gemv_kernel(const uint32_t* __restrict__ codes,
                                                                 const __half* __restrict__ scales,
                                                                 const void* __restrict__ xin, int tokens,
-                                                                int d_out, int d_in, float* __restrict__ y,
-                                                                int wait_first) {
+                                                                int d_out, int d_in, float* __restrict__ y) {
   extern __shared__ __align__(16) float sx[];      // STAGE: [TC][d_in] fp32
   // Mode 1 (memory-bound) lets the next kernel launch at once.  Mode 0 is bound by
   // its arithmetic, and a next kernel whose CTAs wait beside it on the same SMs
@@ -132,8 +129,7 @@ __global__ void __launch_bounds__(kWarps * 32) itq3_gemv_kernel(const uint32_t* 
   // own work is done; as the call's only kernel it reads nothing global before the
   // kernel launched before it has finished.
   if constexpr (MODE == 1) allow_dependent_launch();
-  // (mode 1 after a rotation that let it launch before its own wait: wait_first)
-  if (MODE == 0 || wait_first) wait_for_prerequisite_grid();
+  if constexpr (MODE == 0) wait_for_prerequisite_grid();
   const int lane = threadIdx.x & 31;
   const int row0 = (blockIdx.x * kWarps + (threadIdx.x >> 5)) * R;
   if (!STAGE && row0 >= d_out) return;             // with STAGE every warp joins the barriers
@@ -254,11 +250,9 @@ __global__ void __launch_bounds__(kWarps * 32) itq3_gemv_kernel(const uint32_t* 
 
 // x_rot[t, blk*256 + e] = (H_256 x[t, blk*256 : +256])[e] / 16; one warp per (t, blk).
 __global__ void __launch_bounds__(kWarps * 32) itq3_rotate_x_kernel(const __half* __restrict__ x, int tokens,
-                                                                     int d_in, float* __restrict__ x_rot,
-                                                                     int signal_first) {
-  if (signal_first) allow_dependent_launch();
+                                                                     int d_in, float* __restrict__ x_rot) {
   wait_for_prerequisite_grid();
-  if (!signal_first) allow_dependent_launch();
+  allow_dependent_launch();
   const int lane = threadIdx.x & 31;
   const int item = blockIdx.x * kWarps + (threadIdx.x >> 5);
   const int nb = d_in / 256;
@@ -276,7 +270,7 @@ __global__ void __launch_bounds__(kWarps * 32) itq3_rotate_x_kernel(const __half
 
 // Rotation of every 256-block of x into x_rot, launched with programmatic stream
 // serialization (see above).
-int launch_rotation(const __half* x, int t, int k, float* x_rot, bool signal_first, cudaStream_t st) {
+int launch_rotation(const __half* x, int t, int k, float* x_rot, cudaStream_t st) {
   const int items = t * (k / 256);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>((items + kWarps - 1) / kWarps));
@@ -287,8 +281,7 @@ int launch_rotation(const __half* x, int t, int k, float* x_rot, bool signal_fir
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, itq3_rotate_x_kernel, x, t, k, x_rot, signal_first ? 1 : 0) != cudaSuccess)
-    return WUSH_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, itq3_rotate_x_kernel, x, t, k, x_rot) != cudaSuccess) return WUSH_ERR_CUDA;
   return launch_status();
 }
 
@@ -296,8 +289,7 @@ int launch_rotation(const __half* x, int t, int k, float* x_rot, bool signal_fir
 // row and all 16 blocks of a 4096-wide row in flight per warp for a single token
 // (memory-bound), more rows sharing each x load as the token count grows.
 template <int R, int W, int TC, int MODE>
-int launch_one(const uint32_t* c32, const __half* sc, const void* x, int t, int n, int k, float* y, bool wait_first,
-               cudaStream_t st) {
+int launch_one(const uint32_t* c32, const __half* sc, const void* x, int t, int n, int k, float* y, cudaStream_t st) {
   const size_t smem = static_cast<size_t>(TC) * k * 4;
   // a single token's x is read through L1 well enough; staging pays off once a
   // chunk of several tokens is reused by every row of the CTA
@@ -317,7 +309,7 @@ int launch_one(const uint32_t* c32, const __half* sc, const void* x, int t, int 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, c32, sc, x, t, n, k, y, wait_first ? 1 : 0) != cudaSuccess) return WUSH_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kern, c32, sc, x, t, n, k, y) != cudaSuccess) return WUSH_ERR_CUDA;
   return launch_status();
 }
 
@@ -328,27 +320,22 @@ int launch_one(const uint32_t* c32, const __half* sc, const void* x, int t, int 
 // chunk of it fits.
 template <int MODE>
 int launch_gemv(const uint32_t* c32, const __half* sc, const void* x, int t, int n, int k, float* y,
-                bool wait_first, cudaStream_t st) {
-  if (t == 1) return launch_one<1, 16, 1, MODE>(c32, sc, x, t, n, k, y, wait_first, st);
-  if (t <= 4) return launch_one<4, 4, 4, MODE>(c32, sc, x, t, n, k, y, wait_first, st);
-  return launch_one<4, 4, 8, MODE>(c32, sc, x, t, n, k, y, wait_first, st);
+                cudaStream_t st) {
+  if (t == 1) return launch_one<1, 16, 1, MODE>(c32, sc, x, t, n, k, y, st);
+  if (t <= 4) return launch_one<4, 4, 4, MODE>(c32, sc, x, t, n, k, y, st);
+  return launch_one<4, 4, 8, MODE>(c32, sc, x, t, n, k, y, st);
 }
 
-// Mode 1: rotation of x into x_rot, then the tensor-core kernel (itq3_tc.cu) where
-// the shape allows it and the CUDA-core kernel above otherwise.  When the
-// tensor-core kernel is expected the rotation lets it launch at once (it waits
-// before reading anything); should it then decline the shape, the CUDA-core kernel
-// runs with wait_first, so it too reads nothing before the rotation has finished.
-int rotate_and_gemv(const uint8_t* codes, const void* scales_fp16, const __half* x, float* x_rot, int t, int n,
-                    int k, float* y, cudaStream_t st) {
-  const bool tc_expected = g_itq3_variant == 0 && itq3_tc_shape_ok(t, n, k);
-  if (launch_rotation(x, t, k, x_rot, tc_expected, st) != WUSH_OK) return WUSH_ERR_CUDA;
-  if (tc_expected) {
+// Mode 1 after the rotation: the tensor-core kernel (itq3_tc.cu) where the shape
+// allows it and the CUDA-core kernel above otherwise.
+int gemv_rotated(const uint8_t* codes, const void* scales_fp16, const float* x_rot, int t, int n, int k, float* y,
+                 cudaStream_t st) {
+  if (g_itq3_variant == 0) {
     const int r = itq3_gemv_tc(codes, scales_fp16, x_rot, t, n, k, y, st);
     if (r != WUSH_ERR_UNSUPPORTED) return r;
   }
   return launch_gemv<1>(reinterpret_cast<const uint32_t*>(codes), static_cast<const __half*>(scales_fp16), x_rot, t,
-                        n, k, y, tc_expected, st);
+                        n, k, y, st);
 }
 
 }  // namespace
@@ -370,8 +357,9 @@ extern "C" int itq3_dequant_gemv(const uint8_t* codes, const void* scales_fp16, 
   const auto* sc = static_cast<const __half*>(scales_fp16);
   const auto* xh = static_cast<const __half*>(x_fp16);
   const int t = static_cast<int>(tokens), n = static_cast<int>(d_out), k = static_cast<int>(d_in);
-  if (mode == 0) return launch_gemv<0>(c32, sc, xh, t, n, k, y, false, st);
-  return rotate_and_gemv(codes, scales_fp16, xh, workspace, t, n, k, y, st);
+  if (mode == 0) return launch_gemv<0>(c32, sc, xh, t, n, k, y, st);
+  if (launch_rotation(xh, t, k, workspace, st) != WUSH_OK) return WUSH_ERR_CUDA;
+  return gemv_rotated(codes, scales_fp16, workspace, t, n, k, y, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -474,5 +462,6 @@ extern "C" int itq3_dequant_gemv_noalloc(const uint8_t* codes, const void* scale
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const auto* xh = static_cast<const __half*>(x_fp16);
   const int t = static_cast<int>(tokens), n = static_cast<int>(d_out), k = static_cast<int>(d_in);
-  return rotate_and_gemv(codes, scales_fp16, xh, scratch, t, n, k, y, s);
+  if (launch_rotation(xh, t, k, scratch, s) != WUSH_OK) return WUSH_ERR_CUDA;
+  return gemv_rotated(codes, scales_fp16, scratch, t, n, k, y, s);
 }

@@ -187,11 +187,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                    float* __restrict__ y, int64_t max_polls) {
   using C_ = Cfg<NT>;
   constexpr int kSlots = C_::kSlots;
-  // The next call's first kernel may start early; it waits for this one to finish
-  // before it touches memory.  The rotation before this kernel let it launch at its
-  // own entry, so nothing global is read here before the rotation has finished.
+  // the next call's first kernel may start early; it waits for this one to finish
+  // before it touches memory
   allow_dependent_launch();
-  wait_for_prerequisite_grid();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* bst = smem;                                              // two B stages
@@ -557,15 +555,12 @@ int launch_tc(const uint8_t* codes, const __half* scales, const float* xrot, int
 
 }  // namespace
 
-bool itq3_tc_shape_ok(int tokens, int d_out, int d_in) {
-  // One or two tokens: the decode, not the multiply, is the work, and the CUDA-core
-  // kernel (no TMEM round trip, no cluster reduction) is faster on B200.
-  return tokens >= kMinTokens && tokens <= 16 && d_out > 0 && d_out % kRows == 0 && d_in > 0 && d_in % 256 == 0;
-}
-
 int itq3_gemv_tc(const uint8_t* codes, const void* scales_fp16, const float* x_rot, int tokens, int d_out, int d_in,
                  float* y, cudaStream_t st) {
-  if (!itq3_tc_shape_ok(tokens, d_out, d_in)) return WUSH_ERR_UNSUPPORTED;
+  // One or two tokens: the decode, not the multiply, is the work, and the CUDA-core
+  // kernel (no TMEM round trip, no cluster reduction) is faster on B200.
+  if (tokens < kMinTokens || tokens > 16 || d_out <= 0 || d_out % kRows || d_in <= 0 || d_in % 256)
+    return WUSH_ERR_UNSUPPORTED;
   const auto* sc = static_cast<const __half*>(scales_fp16);
   const int nb = d_in / 256;
   if (tokens <= 8) return launch_tc<16>(codes, sc, x_rot, tokens, d_out, nb, y, st);

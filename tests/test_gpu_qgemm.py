@@ -146,11 +146,12 @@ def test_full_size_up_proj_sampled(lib):
 
 
 @pytest.mark.parametrize("fmt, mnk", [("nvfp4", (4096, 4096, 12288)), ("nvfp4", (4096, 4096, 1024)),
-                                      ("mxfp4", (4096, 4096, 1024))])
+                                      ("mxfp4", (4096, 4096, 1024)), ("mxfp4", (4096, 12288, 4096))])
 def test_gemm_random_codes_many_tiles_per_pair(lib, fmt, mnk):
     # 16 x 16 = 256 pair tiles of 256 x 256 for 74 CTA pairs: every pair runs three
-    # or four tiles, handing its accumulator back between them; (4096, 4096, 12288)
-    # is the NVFP4 down_proj launch.  The oracle checks 64 sampled rows, all columns.
+    # or four tiles, handing its accumulator back between them; (4096, 4096, 12288) is
+    # the NVFP4 down_proj launch and (4096, 12288, 4096) the MXFP4 up_proj launch (10
+    # or 11 tiles per pair).  The oracle checks 64 sampled rows, all columns.
     m, n, k = mnk
     a_c, a_s, a_dq = _random_operand(301 + k, m, k, fmt)
     b_c, b_s, b_dq = _random_operand(402 + k, n, k, fmt)
