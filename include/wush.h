@@ -225,15 +225,18 @@ size_t wush_scales_bytes(int64_t rows, int64_t d_in, int fmt);
  *   MXFP4: amax = max|y| over 32; e = clamp(floor(log2 amax) - 2, -127, 127)
  *          (e = -127 for amax 0); scale byte e + 127; code = E2M1 RNE-satfinite
  *          of y / 2^e.
- *   NVFP4: t = amax / fp32(6 * global_scale); s_b = UE4M3 RNE-satfinite(t);
- *          d = fp32(s_b * global_scale); r = fp32(1 / d);
- *          code = E2M1 RNE-satfinite(fp32(y * r)); codes 0 when s_b = 0.
+ *   NVFP4: s_b = UE4M3 RNE-satfinite(amax / (6 global_scale));
+ *          code = E2M1 RNE-satfinite(y / (s_b global_scale)); codes 0 when s_b = 0.
  *          global_scale is the per-tensor fp32 scale, in [1e-30, 1e30).
- *   INT4:  s = fp16 RNE(amax / 7); r = fp32(1 / s);
- *          q = clamp(rint(fp32(y * r)), -7, 7) (0 if s = 0);
+ *   INT4:  s = fp16 RNE(amax / 7) (saturating at 65504);
+ *          q = clamp(RNE(y / s), -7, 7) (0 if s = 0);
  *          code = q & 0xF (two's complement nibble).
- *   All decisions in fp32 with round-to-nearest-even. E2M1 codes carry the
- *   sign of y even when the magnitude rounds to 0; an all-zero block gives +0.
+ *   y is the fp32 transformed value.  Every decision is the round-to-nearest-even
+ *   (ties to even) of the exact quotient, as written, of that fp32 value: the
+ *   kernels multiply by reciprocals nudged 2^-20 below and above the scale's, and
+ *   settle the rare values whose two results differ with an exact comparison
+ *   against the boundary.  E2M1 codes carry the sign of y even when the magnitude
+ *   rounds to 0; an all-zero block gives +0.
  *
  * x:       device [rows, d_in], bf16 (x_dtype = WUSH_IN_BF16) or fp32.
  * t:       device fp32 [d_in/b, b, b] for WUS/WUSH/WUSH_DIAG; ignored (may be NULL) for
