@@ -197,6 +197,44 @@ __device__ __forceinline__ void tmem_sum3(uint32_t taddr, float (&y)[B]) {
   }
 }
 
+// tmem_sum3 for both b = 16 blocks of a quarter: columns [0, 48) hold block 0's
+// hi, mid and lo, [48, 96) block 1's.  Block 1's loads are issued before block 0's
+// sums are formed, so their latency overlaps that arithmetic.
+__device__ __forceinline__ void tmem_sum3_pair16(uint32_t taddr, float (&y0)[16], float (&y1)[16]) {
+  uint32_t h[16], m[16], l[16];
+  tmem_ld_cols<16>(taddr, h);
+  tmem_ld_cols<16>(taddr + 16, m);
+  tmem_ld_cols<16>(taddr + 32, l);
+  tmem_ld_wait();
+  tmem_tie<16>(h);
+  tmem_tie<16>(m);
+  tmem_tie<16>(l);
+  uint32_t h1[16], m1[16], l1[16];
+  tmem_ld_cols<16>(taddr + 48, h1);
+  tmem_ld_cols<16>(taddr + 64, m1);
+  tmem_ld_cols<16>(taddr + 80, l1);
+#pragma unroll
+  for (int i = 0; i < 16; i += 2) {
+    float s0 = __uint_as_float(m[i]), s1 = __uint_as_float(m[i + 1]);
+    add2(s0, s1, __uint_as_float(l[i]), __uint_as_float(l[i + 1]));
+    y0[i] = __uint_as_float(h[i]);
+    y0[i + 1] = __uint_as_float(h[i + 1]);
+    add2(y0[i], y0[i + 1], s0, s1);
+  }
+  tmem_ld_wait();
+  tmem_tie<16>(h1);
+  tmem_tie<16>(m1);
+  tmem_tie<16>(l1);
+#pragma unroll
+  for (int i = 0; i < 16; i += 2) {
+    float s0 = __uint_as_float(m1[i]), s1 = __uint_as_float(m1[i + 1]);
+    add2(s0, s1, __uint_as_float(l1[i]), __uint_as_float(l1[i + 1]));
+    y1[i] = __uint_as_float(h1[i]);
+    y1[i + 1] = __uint_as_float(h1[i + 1]);
+    add2(y1[i], y1[i + 1], s0, s1);
+  }
+}
+
 // y = (hi + lo) + mid for one b-block of this thread's row (b = 32): the MMAs
 // leave x (T_hi + T_lo)^T in TMEM columns taddr + [0, B) and x T_mid^T in [B, 2B).
 template <int B>
@@ -506,10 +544,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (kMma) {
         tc_fence_after();
         const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + p * kSetCols + g * kSlotCols;
+        if constexpr (L::kThree && kQBlocks == 2 && B == 16) {
+          // both blocks' three partial products (96 contiguous columns) in one round
+          // trip: three loads, one wait
+          tmem_sum3_pair16(taddr, y[0], y[1]);
+        } else {
 #pragma unroll
-        for (int u = 0; u < kQBlocks; ++u) {
-          if constexpr (L::kThree) tmem_sum3<B>(taddr + u * kN, y[u]);
-          else tmem_sum2<B>(taddr + u * kN, y[u]);
+          for (int u = 0; u < kQBlocks; ++u) {
+            if constexpr (L::kThree) tmem_sum3<B>(taddr + u * kN, y[u]);
+            else tmem_sum2<B>(taddr + u * kN, y[u]);
+          }
         }
         tc_fence_before();
         __syncwarp();
