@@ -46,7 +46,7 @@ extern "C" int wush_debug_set_wait_limit(int64_t max_polls) {
 }
 
 extern "C" int wush_debug_set_itq3_variant(int variant) {
-  if (variant < 0 || variant > 1) return WUSH_ERR_INVALID_ARG;
+  if (variant < 0 || variant > 3) return WUSH_ERR_INVALID_ARG;
   wush::g_itq3_variant = variant;
   return WUSH_OK;
 }

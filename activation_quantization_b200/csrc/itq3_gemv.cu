@@ -16,7 +16,9 @@
 // mode 1 (algebraically identical, cheaper per weight on B200): H/16 is
 //   symmetric and orthogonal, so w_hat . x = ((c - 3.5) s) . (H x / 16).  A
 //   first kernel rotates each 256-block of x once into the caller's fp32
-//   workspace; the GEMV then uses the levels (c - 3.5) s with no transform.
+//   workspace; the GEMV then uses the levels (c - 3.5) s with no transform.  For
+//   one or two tokens the call is a single kernel instead (itq3_gemv_rot_kernel):
+//   every CTA rotates the tokens of x into its shared memory.
 #include <cuda_fp16.h>
 
 #include <mutex>
@@ -248,6 +250,223 @@ __global__ void __launch_bounds__(kWarps * 32) itq3_gemv_kernel(const uint32_t* 
   }
 }
 
+// Levels c - 3.5 of the lane's eight elements, as four packed f32x2 pairs.  Code i
+// (bits 3i .. 3i + 2 of the lane's 24 bits) is moved to mantissa bits 20 .. 22 of
+// 1.0f, giving exactly f = 1 + c / 8, and 8 f - 11.5 = c - 3.5 exactly (one packed
+// FMA per pair).  The move is an integer multiply by 2^(20 - 3i) + 2^31 (the 2^31
+// term only reaches bit 31, which the mask drops; it keeps the multiply off the
+// shift unit, which the masks already keep busy), and a right shift by one for
+// i = 7.  Bits past the lane's 24 are masked off.
+__device__ __forceinline__ void levels8(uint32_t word, int lane, uint64_t (&lv)[4]) {
+  const int bit = 24 * lane;
+  const int w0 = bit >> 5;
+  const uint32_t lo = __shfl_sync(0xffffffffu, word, w0);
+  const uint32_t hi = __shfl_sync(0xffffffffu, word, w0 + 1 < 24 ? w0 + 1 : 23);
+  const uint32_t bits = __funnelshift_r(lo, hi, bit & 31);
+  const uint64_t eight = (static_cast<uint64_t>(__float_as_uint(8.0f)) << 32) | __float_as_uint(8.0f);
+  const uint64_t off = (static_cast<uint64_t>(__float_as_uint(-11.5f)) << 32) | __float_as_uint(-11.5f);
+  uint32_t e[8];
+#pragma unroll
+  for (int i = 0; i < 7; ++i) {
+    uint32_t t;
+    asm("mul.lo.u32 %0, %1, %2;" : "=r"(t) : "r"(bits), "r"((1u << (20 - 3 * i)) | 0x80000000u));
+    e[i] = (t & 0x00700000u) | 0x3F800000u;
+  }
+  e[7] = ((bits >> 1) & 0x00700000u) | 0x3F800000u;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    asm("mov.b64 %0, {%1, %2};" : "=l"(lv[i]) : "r"(e[2 * i]), "r"(e[2 * i + 1]));
+    asm("fma.rn.f32x2 %0, %0, %1, %2;" : "+l"(lv[i]) : "l"(eight), "l"(off));
+  }
+}
+
+// Sum of the eight products level * x, in two packed partial sums.
+__device__ __forceinline__ float dot8(const uint64_t (&lv)[4], const float4& xa, const float4& xb) {
+  const float x8[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+  uint64_t acc = 0;                                                 // (+0, +0)
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint64_t xx;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(xx) : "f"(x8[2 * i]), "f"(x8[2 * i + 1]));
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(lv[i]), "l"(xx));
+  }
+  float a0, a1;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(acc));
+  return a0 + a1;
+}
+
+// Mode 1 for up to T tokens in one launch.  A call of two dependent kernels pays two
+// launch-to-launch hand-overs for about 1 us of memory traffic; here each CTA
+// rotates the tokens of x itself (a warp per 256-block and token, x read from L2)
+// into shared memory, so the call is one kernel and needs no workspace.
+//  * Before it waits for the kernel launched before it, every thread asks L2 for one
+//    128-byte line of the CTA's code words and scales.  A prefetch writes no
+//    register, so a kernel still writing them is no hazard: the loads after the wait
+//    read what it wrote, now from L2 instead of DRAM.
+//  * After the wait each warp rotates its blocks of x, the CTA meets at a barrier,
+//    and each warp then loads its code words from L2 for the dot products.
+//  * Each warp owns R rows; the CTA's WARPS * R rows share the rotated x.  A row's
+//    levels are decoded once per block and meet every token.
+template <int WARPS, int R, int W, int T>
+__global__ void __launch_bounds__(WARPS * 32) itq3_gemv_rot_kernel(const uint32_t* __restrict__ codes,
+                                                                    const __half* __restrict__ scales,
+                                                                    const __half* __restrict__ x, int tokens,
+                                                                    int d_out, int d_in, float* __restrict__ y) {
+  extern __shared__ __align__(16) float sx[];      // H x / 16, [tokens][d_in] fp32
+  allow_dependent_launch();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nb = d_in / 256;
+  const int row_cta = blockIdx.x * WARPS * R;
+  {
+    const int rows = min(WARPS * R, d_out - row_cta);
+    const char* cb = reinterpret_cast<const char*>(codes) + static_cast<int64_t>(row_cta) * nb * 96;
+    const int64_t c_bytes = static_cast<int64_t>(rows) * nb * 96;
+    for (int64_t off = static_cast<int64_t>(threadIdx.x) * 128; off < c_bytes; off += WARPS * 32 * 128)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(cb + off));
+    const char* sb = reinterpret_cast<const char*>(scales + static_cast<int64_t>(row_cta) * nb);
+    const int64_t s_bytes = static_cast<int64_t>(rows) * nb * 2;
+    for (int64_t off = static_cast<int64_t>(threadIdx.x) * 128; off < s_bytes; off += WARPS * 32 * 128)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(sb + off));
+  }
+  wait_for_prerequisite_grid();
+  // x first: it is small and stays in L2; the code words (prefetched into L2 above)
+  // are loaded once x is rotated, so that no x load queues behind them
+  for (int item = warp; item < tokens * nb; item += WARPS) {
+    const int64_t base = (T == 1 ? item * 256 : static_cast<int64_t>(item / nb) * d_in + (item % nb) * 256) + lane;
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __half2float(x[base + 32 * i]);
+    warp_fwht256(v, lane);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) sx[base + 32 * i] = v[i] * 0.0625f;
+  }
+  __syncthreads();
+  const int row0 = row_cta + warp * R;
+  // the scales stay fp16 in registers until they are used
+  uint32_t word[R][W];
+  __half sc[R][W];
+  // a full window of a row's scales is W * 2 contiguous bytes, 16-byte aligned when
+  // nb % 8 == 0: then it is read with W / 8 vector loads
+  const bool vec_scales = (nb & 7) == 0 && (W & 7) == 0;
+  float acc[R][T];
+#pragma unroll
+  for (int rr = 0; rr < R; ++rr)
+#pragma unroll
+    for (int tt = 0; tt < T; ++tt) acc[rr][tt] = 0.f;
+  for (int b0 = 0; b0 < nb; b0 += W) {
+#pragma unroll
+    for (int rr = 0; rr < R; ++rr) {
+      const int row = row0 + rr;
+      const uint32_t* crow = codes + (static_cast<int64_t>(row) * nb + b0) * 24 + lane;
+      const __half* srow = scales + static_cast<int64_t>(row) * nb + b0;
+#pragma unroll
+      for (int w = 0; w < W; ++w) {
+        const bool live = row < d_out && b0 + w < nb;
+        word[rr][w] = (live && lane < 24) ? __ldg(crow + 24 * w) : 0u;
+      }
+      if (vec_scales && row < d_out && b0 + W <= nb) {
+#pragma unroll
+        for (int w = 0; w < W; w += 8) {
+          const uint4 q = __ldg(reinterpret_cast<const uint4*>(srow + w));
+          const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+          for (int h = 0; h < 8; ++h)
+            sc[rr][w + h] = __ushort_as_half(static_cast<unsigned short>(qw[h / 2] >> (16 * (h & 1))));
+        }
+      } else {
+#pragma unroll
+        for (int w = 0; w < W; ++w)
+          sc[rr][w] = (row < d_out && b0 + w < nb) ? srow[w] : __ushort_as_half(0);
+      }
+    }
+#pragma unroll
+    for (int w = 0; w < W; ++w) {
+      const int blk = b0 + w;
+      if (blk >= nb) break;
+      if constexpr (T == 1) {
+        // one token: each row's levels go straight into its products
+        const float* xs = sx + blk * 256 + 8 * lane;
+        const float4 xa = *reinterpret_cast<const float4*>(xs);
+        const float4 xb = *reinterpret_cast<const float4*>(xs + 4);
+#pragma unroll
+        for (int rr = 0; rr < R; ++rr) {
+          uint64_t lv[4];
+          levels8(word[rr][w], lane, lv);
+          acc[rr][0] = fmaf(__half2float(sc[rr][w]), dot8(lv, xa, xb), acc[rr][0]);
+        }
+        continue;
+      }
+      uint64_t lv[R][4];
+#pragma unroll
+      for (int rr = 0; rr < R; ++rr) levels8(word[rr][w], lane, lv[rr]);
+#pragma unroll
+      for (int tt = 0; tt < T; ++tt) {
+        if (tt >= tokens) break;
+        const float* xs = sx + static_cast<int64_t>(tt) * d_in + blk * 256 + 8 * lane;
+        const float4 xa = *reinterpret_cast<const float4*>(xs);
+        const float4 xb = *reinterpret_cast<const float4*>(xs + 4);
+#pragma unroll
+        for (int rr = 0; rr < R; ++rr)
+          acc[rr][tt] = fmaf(__half2float(sc[rr][w]), dot8(lv[rr], xa, xb), acc[rr][tt]);
+      }
+    }
+  }
+#pragma unroll
+  for (int rr = 0; rr < R; ++rr)
+#pragma unroll
+    for (int tt = 0; tt < T; ++tt) {
+      const int row = row0 + rr;
+      float a = acc[rr][tt];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
+      if (lane == 0 && row < d_out && tt < tokens) y[static_cast<int64_t>(tt) * d_out + row] = a;
+    }
+}
+
+// Largest token-chunk of rotated x (tokens * d_in fp32) the one-launch kernel keeps in
+// shared memory.
+constexpr int64_t kRotSmemFloats = 40960;
+
+template <int T>
+int launch_rot_t(const uint32_t* c32, const __half* sc, const __half* x, int t, int n, int k, float* y,
+                 cudaStream_t st) {
+  constexpr int kW = 16, kR = 2, kWin = 16;
+  auto kern = itq3_gemv_rot_kernel<kW, kR, kWin, T>;
+  const size_t smem = static_cast<size_t>(t) * k * 4;
+  if (smem > 48 * 1024) {
+    static std::atomic<uint64_t> attr_done{0};
+    if (set_smem_once(kern, kRotSmemFloats * 4, attr_done) != WUSH_OK) return WUSH_ERR_CUDA;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((n + kW * kR - 1) / (kW * kR)));
+  cfg.blockDim = dim3(kW * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, c32, sc, x, t, n, k, y) != cudaSuccess) return WUSH_ERR_CUDA;
+  return launch_status();
+}
+
+int launch_rot(const uint32_t* c32, const __half* sc, const __half* x, int t, int n, int k, float* y,
+               cudaStream_t st) {
+  if (t == 1) return launch_rot_t<1>(c32, sc, x, t, n, k, y, st);
+  if (t == 2) return launch_rot_t<2>(c32, sc, x, t, n, k, y, st);
+  if (t <= 4) return launch_rot_t<4>(c32, sc, x, t, n, k, y, st);
+  return launch_rot_t<8>(c32, sc, x, t, n, k, y, st);
+}
+
+// Whether a mode-1 call runs as the one-launch kernel (see wush_debug_set_itq3_variant):
+// by default for one and two tokens, whose rotated x fits shared memory.
+bool use_rot(int t, int k) {
+  if (static_cast<int64_t>(t) * k > kRotSmemFloats || t > 8) return false;
+  if (g_itq3_variant == 3) return true;
+  return t <= 2 && g_itq3_variant != 2;
+}
+
 // x_rot[t, blk*256 + e] = (H_256 x[t, blk*256 : +256])[e] / 16; one warp per (t, blk).
 __global__ void __launch_bounds__(kWarps * 32) itq3_rotate_x_kernel(const __half* __restrict__ x, int tokens,
                                                                      int d_in, float* __restrict__ x_rot) {
@@ -358,6 +577,7 @@ extern "C" int itq3_dequant_gemv(const uint8_t* codes, const void* scales_fp16, 
   const auto* xh = static_cast<const __half*>(x_fp16);
   const int t = static_cast<int>(tokens), n = static_cast<int>(d_out), k = static_cast<int>(d_in);
   if (mode == 0) return launch_gemv<0>(c32, sc, xh, t, n, k, y, st);
+  if (use_rot(t, k)) return launch_rot(c32, sc, xh, t, n, k, y, st);
   if (launch_rotation(xh, t, k, workspace, st) != WUSH_OK) return WUSH_ERR_CUDA;
   return gemv_rotated(codes, scales_fp16, workspace, t, n, k, y, st);
 }
@@ -454,14 +674,17 @@ extern "C" int itq3_dequant_gemv_noalloc(const uint8_t* codes, const void* scale
   if (d_out > (int64_t(1) << 30)) return WUSH_ERR_UNSUPPORTED;
   if (!codes || !scales_fp16 || !x_fp16 || !y || !aligned16(codes) || !aligned16(scales_fp16) || !aligned16(x_fp16))
     return WUSH_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const auto* xh = static_cast<const __half*>(x_fp16);
+  const int t = static_cast<int>(tokens), n = static_cast<int>(d_out), k = static_cast<int>(d_in);
+  if (use_rot(t, k))
+    return launch_rot(reinterpret_cast<const uint32_t*>(codes), static_cast<const __half*>(scales_fp16), xh, t, n, k,
+                      y, s);
   float* scratch = nullptr;
   const int st = scratch_for_current_device(&scratch);
   if (st != WUSH_OK) return st;
   // The rotation kernel writes every scratch element the GEMV then reads, so
   // nothing left there by an earlier call needs clearing.
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const auto* xh = static_cast<const __half*>(x_fp16);
-  const int t = static_cast<int>(tokens), n = static_cast<int>(d_out), k = static_cast<int>(d_in);
   if (launch_rotation(xh, t, k, scratch, s) != WUSH_OK) return WUSH_ERR_CUDA;
   return gemv_rotated(codes, scales_fp16, scratch, t, n, k, y, s);
 }

@@ -389,6 +389,9 @@ int itq3_quantize_weights(const uint16_t* w_fp16, int64_t d_out, int64_t d_in, u
  *         c - 3.5 are exact fp16 MMA operands and each block of rotated x is
  *         split exactly enough (hi + lo fp16 after a power-of-two scale) that
  *         only the fp32 accumulation rounds; otherwise CUDA cores run it.
+ *         For one or two tokens with tokens * d_in <= 40960 the call is a
+ *         single kernel in which every CTA rotates x into its own shared
+ *         memory; the workspace is then not touched.
  * workspace may be NULL for mode 0.  Requirements: 1 <= tokens <= 16,
  * d_in % 256 == 0, d_out % 8 == 0, codes, scales, x_fp16 and workspace 16-byte
  * aligned; WUSH_ERR_INVALID_ARG otherwise, before any launch. */
@@ -412,7 +415,9 @@ int itq3_dequant_gemv(const uint8_t* codes, const void* scales_fp16, const void*
  * a new context) the next call looks it up again, so it too is a first call.  All
  * calls on a device share the array: calls whose kernels overlap on the GPU
  * (different streams, no ordering between them) race on it.  Nothing needs to
- * start at zero: every call overwrites the part of the array it reads. */
+ * start at zero: every call overwrites the part of the array it reads.  One or two
+ * tokens with tokens * d_in <= 40960 do not use the array (the single-kernel form
+ * above). */
 int itq3_dequant_gemv_noalloc(const uint8_t* codes, const void* scales_fp16, const void* x_fp16,
                               int64_t tokens, int64_t d_out, int64_t d_in, float* y, void* stream);
 
@@ -437,11 +442,14 @@ int wush_debug_set_wait_limit(int64_t max_polls);
 int wush_debug_set_gemm_variant(int variant);
 
 /* Test hook: 0 (default) lets itq3_dequant_gemv mode 1 and
- * itq3_dequant_gemv_noalloc run the tensor-core kernel when tokens >= 3,
+ * itq3_dequant_gemv_noalloc run the single-kernel form when tokens <= 2 and
+ * tokens * d_in <= 40960, and the tensor-core kernel when tokens >= 3,
  * d_out % 128 == 0 and no CTA gets more than 64 of the 256-blocks (always so for
- * d_in <= 16384); 1
- * always uses the CUDA-core kernel, so that the two can be checked against each
- * other.  WUSH_ERR_INVALID_ARG for other values. */
+ * d_in <= 16384); 1 always uses the CUDA-core kernel from 3 tokens on; 2 uses the
+ * rotation kernel followed by the CUDA-core kernel for every token count; 3 uses
+ * the single-kernel form for up to 8 tokens whenever tokens * d_in <= 40960.  So
+ * the forms can be checked against each other.  WUSH_ERR_INVALID_ARG for other
+ * values. */
 int wush_debug_set_itq3_variant(int variant);
 
 #ifdef __cplusplus

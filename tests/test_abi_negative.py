@@ -126,7 +126,7 @@ def test_itq3_gemv():
 
 def test_debug_hooks_reject_out_of_range_values():
     assert lib.wush_debug_set_gemm_variant(3) == INVALID and lib.wush_debug_set_gemm_variant(-1) == INVALID
-    assert lib.wush_debug_set_itq3_variant(2) == INVALID
+    assert lib.wush_debug_set_itq3_variant(4) == INVALID
     assert lib.wush_debug_set_wait_limit(-5) == INVALID
     assert lib.wush_status_string(-7) == b"file could not be opened, read or written"
     assert lib.wush_status_string(-99) == b"unknown status"

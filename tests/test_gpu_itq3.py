@@ -50,11 +50,15 @@ def test_itq3_library_quantiser_feeds_gemv(lib):
     assert err <= 1e-5
 
 
-@pytest.mark.parametrize("tokens, d_in", [(1, 40960), (2, 10240), (2, 12288), (1, 43008)])
-def test_itq3_mode1_rotation_inside_or_outside_the_gemv(lib, tokens, d_in):
-    # one or two tokens rotate x inside the GEMV kernel while a token chunk of x
-    # fits shared memory (1 x 40960 and 2 x 10240 are the largest such); beyond
-    # that the call rotates into the workspace first.  Both forms against the oracle.
+@pytest.mark.parametrize("tokens, d_in", [(1, 40960), (2, 20480), (2, 24576), (1, 43008), (1, 256), (3, 4096),
+                                          (8, 4096), (5, 1024)])
+@pytest.mark.parametrize("variant", [0, 2, 3])
+def test_itq3_mode1_rotation_inside_or_outside_the_gemv(lib, tokens, d_in, variant):
+    # the single-kernel form rotates x inside the GEMV while the tokens' rotated x
+    # fits shared memory (tokens * d_in <= 40960): by default for one and two
+    # tokens, for up to eight as variant 3.  Otherwise, and for every call as variant
+    # 2, the call rotates into the workspace first and then runs the GEMV (the
+    # tensor-core kernel from 3 tokens when d_out % 128 == 0).  Against the oracle.
     d_out = 64
     w = synth.itq3_weights(d_out, d_in)
     x = synth.itq3_activations(tokens, d_in).astype(np.float16)
@@ -62,8 +66,12 @@ def test_itq3_mode1_rotation_inside_or_outside_the_gemv(lib, tokens, d_in):
     want = I.gemv(c, s, x.astype(np.float64))
     y = torch.full((tokens, d_out), float("nan"), dtype=torch.float32, device="cuda")
     ws = torch.empty((tokens, d_in), dtype=torch.float32, device="cuda")
-    lib.itq3_dequant_gemv(torch.from_numpy(pack_codes(c)).cuda(), torch.from_numpy(s).cuda(),
-                          torch.from_numpy(x).cuda(), d_out, 1, y, ws)
-    assert lib.wush_check_device_status() == 0
+    lib.wush_debug_set_itq3_variant(variant)
+    try:
+        lib.itq3_dequant_gemv(torch.from_numpy(pack_codes(c)).cuda(), torch.from_numpy(s).cuda(),
+                              torch.from_numpy(x).cuda(), d_out, 1, y, ws)
+        assert lib.wush_check_device_status() == 0
+    finally:
+        lib.wush_debug_set_itq3_variant(0)
     got = y.cpu().numpy().astype(np.float64)
     assert np.linalg.norm(got - want) / np.linalg.norm(want) <= 1e-5

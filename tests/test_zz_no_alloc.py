@@ -36,9 +36,10 @@ def _rel(got, want):
     return np.linalg.norm(got - want) / np.linalg.norm(want)
 
 
-# tokens 1-2 run the CUDA-core GEMV, 3 and 16 the tensor-core one; the last case
-# fills the fixed array exactly (16 x 16384 floats)
-@pytest.mark.parametrize("tokens, d_out, d_in", [(1, 1024, 4096), (2, 1024, 4096), (3, 1024, 4096),
+# tokens 1-2 with tokens * d_in <= 40960 run the single-kernel form, which does not
+# touch the array; 2 x 32768 rotates into the array and runs the CUDA-core GEMV, 3
+# and 16 the tensor-core one; the last case fills the array exactly (16 x 16384)
+@pytest.mark.parametrize("tokens, d_out, d_in", [(1, 1024, 4096), (2, 1024, 4096), (2, 64, 32768), (3, 1024, 4096),
                                                  (16, 1024, 4096), (16, 256, 16384)])
 def test_noalloc_matches_oracle_and_workspace_form_on_consecutive_calls(lib, tokens, d_out, d_in):
     assert tokens * d_in <= SCRATCH_FLOATS
