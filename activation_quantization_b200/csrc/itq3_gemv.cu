@@ -65,21 +65,25 @@ __device__ __forceinline__ void wait_for_prerequisite_grid() {
 // Levels (c - 3.5) s of the eight elements 8 lane .. 8 lane + 7 of one 256-block.
 // Lane j < 24 holds word j of the block's 96 packed bytes (3-bit codes,
 // little-endian, element e at bits 3e .. 3e + 2); this lane's 24 bits start at bit
-// 24 lane, inside words (24 lane) / 32 and the one after it.
+// 24 lane, inside words (24 lane) / 32 and the one after it.  Code i goes into
+// mantissa bits 20 .. 22 of 1.0f (see levels8 below), giving f = 1 + c / 8 exactly,
+// and (c - 3.5) s = f (8 s) - 11.5 s: 8 s and 11.5 s are exact, and so is the FMA,
+// since (c - 3.5) s needs at most 15 significant bits.
 __device__ __forceinline__ void decode_levels(uint32_t word, int lane, float s, float (&v)[8]) {
   const int bit = 24 * lane;
   const int w0 = bit >> 5;
   const uint32_t lo = __shfl_sync(0xffffffffu, word, w0);
   const uint32_t hi = __shfl_sync(0xffffffffu, word, w0 + 1 < 24 ? w0 + 1 : 23);
   const uint32_t bits = __funnelshift_r(lo, hi, bit & 31);
-  const float m = -3.5f * s;
-  // code c as a float without an integer-to-float conversion: the bits 2^23 + c
-  // minus 2^23 (both exact); (c - 3.5) s then needs at most 15 significant bits,
-  // so the FMA is exact too
+  const float s8 = 8.0f * s, m = -11.5f * s;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float c = __fsub_rn(__uint_as_float(0x4B000000u | ((bits >> (3 * i)) & 7u)), 8388608.0f);
-    v[i] = fmaf(c, s, m);
+    uint32_t t;
+    if (i < 7)
+      asm("mul.lo.u32 %0, %1, %2;" : "=r"(t) : "r"(bits), "r"((1u << (20 - 3 * (i < 7 ? i : 0))) | 0x80000000u));
+    else
+      t = bits >> 1;
+    v[i] = fmaf(__uint_as_float((t & 0x00700000u) | 0x3F800000u), s8, m);
   }
 }
 
