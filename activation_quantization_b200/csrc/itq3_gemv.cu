@@ -6,9 +6,9 @@
 // the exact inverse transform is applied as the weights are loaded for the
 // matmul.  Here one warp owns one to four output rows; lane l holds elements
 // 8*l .. 8*l + 7 of each 256-block, whose codes are the 24 contiguous bits at bit
-// 24*l of the block's packed 96 bytes, so a lane decodes its eight weights with
-// one funnel shift and one bit-field extract and one FMA each, and reads its x
-// values with 16-byte loads.
+// 24*l of the block's packed 96 bytes, so a lane gathers its bits with one funnel
+// shift, decodes each weight with an integer multiply, a mask and one FMA, and
+// reads its x values with 16-byte loads.
 //
 // mode 0 (the article's design): the 256-point inverse FWHT of each weight
 //   block runs in registers -- index bits 0..2 inside the lane, bits 3..7 across
