@@ -143,14 +143,37 @@ __device__ __forceinline__ int int4_from_nibble(uint32_t n) {
   return static_cast<int>(n << 28) >> 28;
 }
 
+// (a0, a1) + (b0, b1) and (a0, a1) * (b0, b1) + (c0, c1) as packed f32x2 operations,
+// each lane rounded to nearest like FADD / FFMA.
+__device__ __forceinline__ void pk_add(float a0, float a1, float b0, float b1, float& o0, float& o1) {
+  unsigned long long x, y, z;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(y) : "f"(b0), "f"(b1));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(z) : "l"(x), "l"(y));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(o0), "=f"(o1) : "l"(z));
+}
+__device__ __forceinline__ void pk_fma(float a0, float a1, float b0, float b1, float& c0, float& c1) {
+  unsigned long long x, y, z;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(y) : "f"(b0), "f"(b1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(z) : "f"(c0), "f"(c1));
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(z) : "l"(x), "l"(y));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(c0), "=f"(c1) : "l"(z));
+}
+
 // Eight INT4 codes (two's-complement nibbles) of v[0..7] with scale s > 0 and
 // r = fp32(1 / s).  Exact: equal to clamp(RNE(v / s), -7, 7).
 // When s is a normal fp16 below 65504 (s = fp16_RNE(amax / 7) within 2^-11), no
 // |v / s| exceeds 7 (1 + 2^-10) < 7.5, so no value needs the clamp.
+// Both brackets are rounded with packed adds of 1.5 * 2^23; only the low one is
+// packed into nibbles.  The two agree everywhere exactly when the sum of the squared
+// differences of their rounded values (each 0 or 1, all exact) is zero.
 __device__ __forceinline__ uint32_t int4_codes8(const float* v, float r, float s) {
+  constexpr float kBias = 12582912.0f;                         // 1.5 * 2^23
   const float ra = __fmul_rn(r, kBracketLo), rb = __fmul_rn(r, kBracketHi);
   const bool in_range = s >= 6.103515625e-05f && s < 65504.0f;
-  uint32_t wa = 0, wb = 0;
+  uint32_t wa = 0;
+  float dd0 = 0.f, dd1 = 0.f;
 #pragma unroll
   for (int i = 0; i < 8; i += 2) {
     float a0, a1, b0, b1;
@@ -162,14 +185,19 @@ __device__ __forceinline__ uint32_t int4_codes8(const float* v, float r, float s
       b0 = fminf(fmaxf(b0, -7.0f), 7.0f);
       b1 = fminf(fmaxf(b1, -7.0f), 7.0f);
     }
-    wa = put_nibble(put_nibble(wa, rne_bits(a0), 4 * i), rne_bits(a1), 4 * i + 4);
-    wb = put_nibble(put_nibble(wb, rne_bits(b0), 4 * i), rne_bits(b1), 4 * i + 4);
+    pk_add(a0, a1, kBias, kBias, a0, a1);
+    pk_add(b0, b1, kBias, kBias, b0, b1);
+    wa = put_nibble(put_nibble(wa, __float_as_uint(a0), 4 * i), __float_as_uint(a1), 4 * i + 4);
+    pk_add(b0, b1, -a0, -a1, b0, b1);                           // 0 or +-1, exact
+    pk_fma(b0, b1, b0, b1, dd0, dd1);
   }
-  if (wa == wb) return wa;
+  if (dd0 + dd1 == 0.f) return wa;
   uint32_t w = wa;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const int qa = int4_from_nibble((wa >> (4 * i)) & 15u), qb = int4_from_nibble((wb >> (4 * i)) & 15u);
+    float b = __fmul_rn(v[i], rb);
+    if (!in_range) b = fminf(fmaxf(b, -7.0f), 7.0f);
+    const int qa = int4_from_nibble((wa >> (4 * i)) & 15u), qb = int4_from_nibble(rne_bits(b) & 15u);
     if (qa == qb) continue;
     const int lo = min(qa, qb), hi = max(qa, qb);
     const float p = (static_cast<float>(lo) + 0.5f) * s;     // at most 15 significant bits: exact
