@@ -75,3 +75,22 @@ def test_itq3_mode1_rotation_inside_or_outside_the_gemv(lib, tokens, d_in, varia
         lib.wush_debug_set_itq3_variant(0)
     got = y.cpu().numpy().astype(np.float64)
     assert np.linalg.norm(got - want) / np.linalg.norm(want) <= 1e-5
+
+
+@pytest.mark.parametrize("d_out", [8, 40, 72, 1000])
+@pytest.mark.parametrize("tokens, d_in", [(1, 256), (1, 2048), (2, 2048)])
+def test_itq3_one_launch_ragged_rows(lib, d_out, tokens, d_in):
+    # the one-launch form gives each CTA 32 rows: row counts that leave the last CTA
+    # partly empty (and a single CTA of 8 rows) against the oracle
+    w = synth.itq3_weights(d_out, d_in)
+    x = synth.itq3_activations(tokens, d_in).astype(np.float16)
+    c, s = I.quantize(w)
+    want = I.gemv(c, s, x.astype(np.float64))
+    y = torch.full((tokens, d_out), float("nan"), dtype=torch.float32, device="cuda")
+    ws = torch.empty((tokens, d_in), dtype=torch.float32, device="cuda")
+    lib.itq3_dequant_gemv(torch.from_numpy(pack_codes(c)).cuda(), torch.from_numpy(s).cuda(),
+                          torch.from_numpy(x).cuda(), d_out, 1, y, ws)
+    assert lib.wush_check_device_status() == 0
+    got = y.cpu().numpy().astype(np.float64)
+    assert np.isfinite(got).all()
+    assert np.linalg.norm(got - want) / np.linalg.norm(want) <= 1e-5
