@@ -20,6 +20,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -86,10 +87,27 @@ def max_over_ranks(value: float, world: int) -> float:
 
 
 def source_sha(source_file: str) -> str:
-    """Hash of a kernel's source file together with the library's device headers."""
-    csrc = os.path.dirname(source_file)
+    """Hash of a kernel's source file together with the device headers it includes
+    (quoted includes found beside it, followed recursively; the public C header, which
+    holds declarations only, is left out)."""
+    dirs = [os.path.dirname(source_file)]
+    seen, order, todo = set(), [], [source_file]
+    while todo:
+        f = todo.pop(0)
+        if f in seen:
+            continue
+        seen.add(f)
+        order.append(f)
+        for line in open(f, encoding="utf-8", errors="replace"):
+            m = re.match(r'\s*#\s*include\s+"([^"]+)"', line)
+            if m:
+                for d in dirs:
+                    cand = os.path.join(d, m.group(1))
+                    if os.path.exists(cand):
+                        todo.append(cand)
+                        break
     h = hashlib.sha1()
-    for f in [source_file] + sorted(os.path.join(csrc, n) for n in os.listdir(csrc) if n.endswith(".cuh")):
+    for f in [order[0]] + sorted(order[1:]):
         h.update(open(f, "rb").read())
     return h.hexdigest()[:12]
 
