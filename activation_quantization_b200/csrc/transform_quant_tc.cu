@@ -311,8 +311,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // release with one arrival per warp.
   const int n_mine = tile_hi - tile_lo;
   const int n_cols = n_mine > 0 ? (tile_hi - 1) / n_row_tiles - col_lo + 1 : 0;
-  // The epilogue threads fetch the fp32 T of this CTA's first two columns before
-  // anything else, so those reads do not queue behind the X tiles in DRAM.
+  // Right after the launch wait, thread 0 sends the first X loads and the epilogue
+  // threads then fetch the fp32 T of this CTA's first two columns, ahead of the rest
+  // of the X tiles.
   constexpr int kTGroups = kBlocks * B * B / 4;    // float4 groups of T per column
   constexpr int kTPer = kTGroups / kEpiThreads;    // per epilogue thread: 2 or 1
   static_assert(kTPer * kEpiThreads == kTGroups, "T column splits evenly over the epilogue threads");
