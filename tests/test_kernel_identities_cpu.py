@@ -73,3 +73,51 @@ def test_int4_agreement_test_is_exact():
             a, b = base + F32(qa), base + F32(qa + d)
             diff = b - a
             assert float(diff) == d and float(diff * diff) == d
+
+
+def _significant_bits(x):
+    x = abs(float(x))
+    if x == 0:
+        return 0
+    num, den = x.as_integer_ratio()
+    while num % 2 == 0:
+        num //= 2
+    return num.bit_length()
+
+
+def _ue4m3_values():
+    vals = []
+    for code in range(0x7F):                      # 0x7F is NaN
+        e, m = code >> 3, code & 7
+        vals.append(m / 8 * 2.0 ** -6 if e == 0 else (1 + m / 8) * 2.0 ** (e - 7))
+    return vals
+
+
+def test_nvfp4_scale_midpoints_are_exact_with_few_bits():
+    # between adjacent UE4M3 codes the decision compares amax with 6 m s_g, m their
+    # midpoint: 6 m = 3 (v_lo + v_hi) has at most 7 significant bits, so it is exact
+    # in fp32 and one FMA gives the sign of amax - 6 m s_g exactly
+    v = _ue4m3_values()
+    for lo, hi in zip(v[:-1], v[1:]):
+        m6 = 3.0 * (lo + hi)
+        assert float(F32(m6)) == m6 and _significant_bits(m6) <= 7
+
+
+def test_e2m1_midpoints_times_scales_are_exact():
+    # code decision: |v| against m * s_b * s_g with m the E2M1 midpoint (at most 3
+    # significant bits) and s_b a UE4M3 value (4): m * s_b is exact in fp32
+    mags = [0, 0.5, 1, 1.5, 2, 3, 4, 6]
+    for lo, hi in zip(mags[:-1], mags[1:]):
+        m = 0.5 * (lo + hi)
+        assert _significant_bits(m) <= 3
+        for sb in _ue4m3_values():
+            assert float(F32(m) * F32(sb)) == m * sb
+
+
+def test_int4_scale_midpoints_are_exact():
+    # fp16 scale decision: amax against 7 m, m the midpoint of adjacent fp16 values:
+    # 3.5 (lo + hi) has at most 15 significant bits, exact in fp32
+    h = np.arange(0x0000, 0x7BFF, dtype=np.uint16).view(np.float16).astype(np.float64)
+    m7 = 3.5 * (h[:-1] + h[1:])
+    assert np.array_equal(m7.astype(np.float32).astype(np.float64), m7)
+    assert max(_significant_bits(x) for x in m7[::97]) <= 15
